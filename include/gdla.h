@@ -1,0 +1,141 @@
+/*
+ * gdla.h - C ABI of the GDLA forward core for NVIDIA B200 (sm_100a).
+ *
+ * Grouped Differential Latent Attention (GDLA), as described for the Motif 3
+ * model (aitrends.kr/articles/94908, "314B MoE 언어 모델 Motif 3의 구조와 학습
+ * 시스템", GDLA paragraphs; metalmedia.ai digest of arXiv 2608.09119, Table 1):
+ *
+ *   For every KV head j, GROUP = 4 signal query heads (4j..4j+3) and one noise
+ *   query head (j) attend with causal softmax attention over the same K_j
+ *   (dim 192) and V_j (dim 128), either over the full causal context or over
+ *   a sliding window. With H_S,i and H_N,j the attention outputs,
+ *       D_i     = H_S,i - lambda[t, i] * H_N,j          (j = i / 4)
+ *       out_i   = sigmoid(gate_logits[t, i, :]) * D_i   (element-wise)
+ *   and out is rounded once, to nearest even, to bf16.
+ *
+ * Readings where the pages are silent: lambda is one fp32 scalar per (token,
+ * signal head) in (0, 1), precomputed by the caller as sigmoid(x W^lambda);
+ * the softmax scale is 1/sqrt(192); a window of W keys includes the query
+ * itself (keys t-W+1 .. t); nothing follows the subtract except the gate.
+ * q and k arrive after any rotary embedding; the latent up-projection, the
+ * lambda and gate projections and the output projection are ordinary GEMMs
+ * outside this library.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensors are dense, row-major, caller-owned DEVICE memory unless a
+ *    comment says HOST. Tensor base pointers must be 16-byte aligned.
+ *  - bf16 is IEEE bfloat16 (1-8-7); lambda is fp32.
+ *  - The library allocates no memory, keeps no state between calls and may
+ *    be called from several host threads at once.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream). GDLA_OK means every kernel was enqueued; a CUDA launch
+ *    failure is reported as GDLA_ERR_CUDA.
+ *  - Arguments are checked on the host before anything is launched; on an
+ *    error nothing is launched and no output is written.
+ *  - Results are deterministic (no atomics, fixed reduction order).
+ *  - Output rows that belong to no sequence are never written.
+ */
+#ifndef GDLA_H
+#define GDLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDLA_GROUP 4          /* signal heads per noise / KV head (g) */
+#define GDLA_DQK 192          /* query-key head dim */
+#define GDLA_DV 128           /* value head dim */
+#define GDLA_MAX_KV_HEADS 64  /* largest num_kv_heads accepted */
+#define GDLA_VERSION 1
+
+typedef enum {
+    GDLA_OK = 0,
+    GDLA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, negative size, bad batch */
+    GDLA_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels handle (e.g. > 64 KV heads) */
+    GDLA_ERR_WORKSPACE = 3,    /* decode workspace missing or too small */
+    GDLA_ERR_CUDA = 4          /* a CUDA call or kernel launch failed */
+} gdla_status_t;
+
+/*
+ * Packed varlen prefill (GDLA core, full causal or sliding window).
+ * Defined by the GDLA query-path paragraph of aitrends.kr/articles/94908
+ * (D = H_S - lambda (.) Repeat_g(H_N), then the query-based gate) with the
+ * head grouping of its group-ratio paragraph.
+ *
+ * N = sum(seqlens). Sequence b occupies packed rows [s_b, s_b + seqlens[b]).
+ *   q_sig        bf16 [N, 4*num_kv_heads, 192]
+ *   q_noise      bf16 [N, num_kv_heads, 192]
+ *   k            bf16 [N, num_kv_heads, 192]
+ *   v            bf16 [N, num_kv_heads, 128]
+ *   lambda       fp32 [N, 4*num_kv_heads], values in (0, 1)
+ *   gate_logits  bf16 [N, 4*num_kv_heads, 128]
+ *   out          bf16 [N, 4*num_kv_heads, 128], written
+ *   batch        number of sequences, >= 1
+ *   seqlens      HOST int32 [batch], each >= 0 (empty sequences are skipped)
+ *   num_kv_heads 1 .. GDLA_MAX_KV_HEADS
+ *   window       <= 0: full causal; > 0: query t sees keys t-window+1 .. t
+ *   stream       cudaStream_t to enqueue on
+ * Errors: GDLA_ERR_INVALID_ARG for a null or non-16-byte-aligned pointer
+ * (when N > 0), batch < 1, a negative length or N >= 2^31;
+ * GDLA_ERR_UNSUPPORTED for num_kv_heads out of range; GDLA_ERR_CUDA if a
+ * launch fails. N == 0 returns GDLA_OK without launching.
+ */
+gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k, const void *v,
+                            const float *lambda, const void *gate_logits, void *out,
+                            int batch, const int32_t *seqlens, int num_kv_heads, int window,
+                            void *stream);
+
+/*
+ * Bytes of device workspace gdla_attn_decode needs for these sizes (0 when
+ * no split-KV pass is used). Returns 0 for invalid sizes as well; the
+ * workspace must be 256-byte aligned.
+ */
+size_t gdla_decode_workspace_bytes(int batch, int num_kv_heads, int max_seqlen_k, int window);
+
+/*
+ * Varlen decode: one new query token per sequence, attending over that
+ * sequence's KV cache (the cache already holds the new token's key and value,
+ * so the query sits at position L_b - 1). Same method as gdla_attn_fwd (the
+ * KV-cache motivation is the aitrends.kr/articles/94908 paragraph contrasting
+ * self-attention and MLA's compressed KV cache).
+ *   q_sig        bf16 [batch, 4*num_kv_heads, 192]
+ *   q_noise      bf16 [batch, num_kv_heads, 192]
+ *   k_cache      bf16 [Nk, num_kv_heads, 192], sequences packed back to back
+ *   v_cache      bf16 [Nk, num_kv_heads, 128]
+ *   cu_seqlens_k DEVICE int32 [batch + 1]: sequence b owns cache rows
+ *                cu[b] .. cu[b+1]-1; every L_b = cu[b+1]-cu[b] must be in
+ *                1 .. max_seqlen_k (a violating sequence's output is zeroed)
+ *   max_seqlen_k HOST upper bound on every L_b, >= 1 (sizes the split plan)
+ *   lambda       fp32 [batch, 4*num_kv_heads]
+ *   gate_logits  bf16 [batch, 4*num_kv_heads, 128]
+ *   out          bf16 [batch, 4*num_kv_heads, 128], written
+ *   window       <= 0: full context; > 0: the last `window` cache rows
+ *   workspace    DEVICE scratch of at least
+ *                gdla_decode_workspace_bytes(batch, num_kv_heads,
+ *                max_seqlen_k, window) bytes, 256-byte aligned (may be NULL
+ *                when that is 0); its contents need no initialisation
+ * Errors: GDLA_ERR_INVALID_ARG (null/misaligned pointers, batch < 1,
+ * max_seqlen_k < 1), GDLA_ERR_UNSUPPORTED (num_kv_heads out of range),
+ * GDLA_ERR_WORKSPACE (workspace NULL or smaller than required),
+ * GDLA_ERR_CUDA (launch failure).
+ */
+gdla_status_t gdla_attn_decode(const void *q_sig, const void *q_noise, const void *k_cache,
+                               const void *v_cache, const int32_t *cu_seqlens_k, int max_seqlen_k,
+                               const float *lambda, const void *gate_logits, void *out,
+                               int batch, int num_kv_heads, int window,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/* Static, human-readable name of a status code. */
+const char *gdla_status_string(gdla_status_t status);
+
+/* GDLA_VERSION of the loaded library. */
+int gdla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDLA_H */

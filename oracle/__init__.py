@@ -1,0 +1,151 @@
+"""GDLA forward oracle (fp64, CPU): TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+legs of ``bench.py`` may import this package. The CUDA product path never
+imports, links or calls it, and the two share no code.
+
+The arithmetic lives in ``gdla_oracle.c`` (plain C, double precision); this
+module only compiles it on demand and marshals numpy arrays through ctypes.
+Parity status per function:
+
+* ``prefill`` - pinned (closed forms, invariants, a library special case and
+  brute force; see ``tests/test_oracle_pins.py``).
+* ``decode`` - pinned through the decode == last prefill row identity and the
+  same closed forms.
+
+The choice of lambda granularity (one scalar per token and signal head), the
+absence of any normalisation after the subtract and the 1/sqrt(192) softmax
+scale are readings where the pages are silent; no page value pins them.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdla_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libgdla_oracle.so")
+_lib = None
+_lock = threading.Lock()
+
+GROUP = 4
+DQK = 192
+DV = 128
+
+
+def build(force: bool = False) -> str:
+    """Compile gdla_oracle.c into libgdla_oracle.so (gcc, -O2, pthreads)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                               "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            p = ctypes.c_void_p
+            lib.gdla_oracle_prefill.argtypes = [p, p, p, p, p, p, ctypes.c_int, ctypes.c_int, p,
+                                                ctypes.c_int, p, ctypes.c_int64, p, ctypes.c_int]
+            lib.gdla_oracle_prefill.restype = ctypes.c_int
+            lib.gdla_oracle_decode.argtypes = [p, p, p, p, p, p, p, ctypes.c_int, ctypes.c_int,
+                                               ctypes.c_int, p, ctypes.c_int]
+            lib.gdla_oracle_decode.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _bits(a, shape_tail, name):
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError(f"{name}: expected bf16 bit patterns as uint16, got {a.dtype}")
+    if tuple(a.shape[1:]) != tuple(shape_tail):
+        raise ValueError(f"{name}: expected trailing shape {shape_tail}, got {a.shape}")
+    return a
+
+
+def _ptr(a):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def prefill(q_sig, q_noise, k, v, lam, gate, seqlens, window, rows=None, num_threads=None):
+    """Packed varlen GDLA prefill in fp64.
+
+    q_sig [N, 4H, 192], q_noise [N, H, 192], k [N, H, 192], v [N, H, 128] and
+    gate [N, 4H, 128] are uint16 arrays of bf16 bits; lam is float32 [N, 4H].
+    ``rows`` selects packed token indices (default: all N). Returns float64
+    [len(rows), 4H, 128].
+    """
+    hkv = q_noise.shape[1]
+    hs = GROUP * hkv
+    q_sig = _bits(q_sig, (hs, DQK), "q_sig")
+    q_noise = _bits(q_noise, (hkv, DQK), "q_noise")
+    k = _bits(k, (hkv, DQK), "k")
+    v = _bits(v, (hkv, DV), "v")
+    gate = _bits(gate, (hs, DV), "gate")
+    lam = np.ascontiguousarray(lam, dtype=np.float32)
+    seqlens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    n = int(seqlens.sum())
+    for name, a in (("q_sig", q_sig), ("q_noise", q_noise), ("k", k), ("v", v), ("gate", gate), ("lambda", lam)):
+        if a.shape[0] != n:
+            raise ValueError(f"{name}: leading dim {a.shape[0]} != sum(seqlens) {n}")
+    if lam.shape != (n, hs):
+        raise ValueError(f"lambda: expected shape {(n, hs)}, got {lam.shape}")
+    if rows is None:
+        rows = np.arange(n, dtype=np.int64)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    out = np.zeros((rows.shape[0], hs, DV), dtype=np.float64)
+    nt = int(num_threads or default_threads())
+    rc = _load().gdla_oracle_prefill(_ptr(q_sig), _ptr(q_noise), _ptr(k), _ptr(v), _ptr(lam), _ptr(gate),
+                                     hkv, int(seqlens.shape[0]), _ptr(seqlens), int(window),
+                                     _ptr(rows), int(rows.shape[0]), _ptr(out), nt)
+    if rc != 0:
+        raise ValueError("gdla_oracle_prefill rejected its arguments")
+    return out
+
+
+def decode(q_sig, q_noise, k_cache, v_cache, cu_seqlens_k, lam, gate, window, num_threads=None):
+    """Varlen GDLA decode in fp64: one query per sequence at position L_b - 1.
+
+    q_sig [B, 4H, 192], q_noise [B, H, 192], gate [B, 4H, 128], lam [B, 4H];
+    k_cache [Nk, H, 192] and v_cache [Nk, H, 128] packed by cu_seqlens_k [B+1].
+    Returns float64 [B, 4H, 128].
+    """
+    hkv = q_noise.shape[1]
+    hs = GROUP * hkv
+    q_sig = _bits(q_sig, (hs, DQK), "q_sig")
+    q_noise = _bits(q_noise, (hkv, DQK), "q_noise")
+    k_cache = _bits(k_cache, (hkv, DQK), "k_cache")
+    v_cache = _bits(v_cache, (hkv, DV), "v_cache")
+    gate = _bits(gate, (hs, DV), "gate")
+    lam = np.ascontiguousarray(lam, dtype=np.float32)
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens_k, dtype=np.int64))
+    b = cu.shape[0] - 1
+    if q_sig.shape[0] != b or q_noise.shape[0] != b or gate.shape[0] != b or lam.shape != (b, hs):
+        raise ValueError("decode: per-sequence inputs must have leading dim B = len(cu_seqlens_k) - 1")
+    if cu[-1] > k_cache.shape[0] or cu[-1] > v_cache.shape[0]:
+        raise ValueError("decode: cache shorter than cu_seqlens_k[-1]")
+    out = np.zeros((b, hs, DV), dtype=np.float64)
+    nt = int(num_threads or default_threads())
+    rc = _load().gdla_oracle_decode(_ptr(q_sig), _ptr(q_noise), _ptr(k_cache), _ptr(v_cache), _ptr(cu),
+                                    _ptr(lam), _ptr(gate), b, hkv, int(window), _ptr(out), nt)
+    if rc != 0:
+        raise ValueError("gdla_oracle_decode rejected its arguments")
+    return out

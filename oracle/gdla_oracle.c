@@ -1,0 +1,297 @@
+/*
+ * GDLA forward oracle: plain, slow, fp64 CPU implementation of the Grouped
+ * Differential Latent Attention core.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only tests/, __graft_entry__.smoke() and the CPU
+ * baseline leg of bench.py may load this library. The CUDA library never calls
+ * it and shares no code, header or constant with it.
+ *
+ * What it follows (aitrends.kr/articles/94908, "314B MoE 언어 모델 Motif 3의
+ * 구조와 학습 시스템", GDLA paragraphs):
+ *  - the two attention paths (signal and noise) share one KV head, and the
+ *    noise output is subtracted from the signal output:
+ *        D_t = H_{S,t} - lambda_t (.) Repeat_g(H_{N,t})
+ *    followed by the query-based element-wise output gate ("GDLA query path"
+ *    paragraph);
+ *  - 80 query heads / 16 KV heads, 64 signal + 16 noise, dqk = 192, dv = 128
+ *    ("GDLA head configuration" paragraph; also Table 1 of the metalmedia.ai
+ *    digest of arXiv 2608.09119);
+ *  - group ratio g = 4, n_N = n_H/(g+1), n_S = g n_N; each signal head is
+ *    paired with the noise head of its own group; lambda_t = sigmoid(x_t W^l)
+ *    lies in (0, 1) ("group ratio" paragraph);
+ *  - full causal attention, or sliding-window attention over 128 tokens
+ *    (Table 1 "Hybrid GDLA (1 full / 3 sliding-window)"; idailynews article,
+ *    hybrid-attention paragraph).
+ *
+ * Readings taken where the pages are silent (each stated once here):
+ *  - lambda is one fp32 scalar per (token, signal head), broadcast over dv;
+ *  - Repeat_g is contiguous: noise head j serves signal heads 4j..4j+3, and
+ *    both use KV head j;
+ *  - the softmax scale is 1/sqrt(192);
+ *  - a window of W keys includes the query itself: keys u in [t-W+1, t];
+ *    window <= 0 means full causal;
+ *  - the gate is out = sigmoid(gate_logit) * D, element-wise per (token,
+ *    signal head, d); nothing else (no per-head norm) follows the subtract;
+ *  - decode: the single query of sequence b sits at position L_b - 1 and the
+ *    cache already holds its key and value.
+ *
+ * Arithmetic: every bf16 input is widened exactly to double, every fp32 lambda
+ * is widened exactly to double, and all arithmetic is in double with no tiling
+ * or reordering beyond the sums written below.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define GROUP 4     /* signal heads per noise head (g) */
+#define DQK 192     /* query/key head dim */
+#define DV 128      /* value head dim */
+
+static double bf16_to_double(uint16_t x) {
+    uint32_t bits = ((uint32_t)x) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/*
+ * One softmax-attention head for one query row:
+ *   s_u = (q . k_u) / sqrt(192),  w_u = exp(s_u - max_u s_u),
+ *   H = sum_u w_u v_u / sum_u w_u,
+ * over the keys u = 0..nkeys-1 whose rows start at k_rows + u*kstride and
+ * v_rows + u*vstride. `scores` has room for nkeys doubles.
+ */
+static void attend(const uint16_t *q, const uint16_t *k_rows, const uint16_t *v_rows,
+                   long kstride, long vstride, long nkeys, double *scores, double *h) {
+    double qd[DQK];
+    for (int d = 0; d < DQK; ++d) qd[d] = bf16_to_double(q[d]);
+    const double root = sqrt((double)DQK);
+    double smax = -INFINITY;
+    for (long u = 0; u < nkeys; ++u) {
+        const uint16_t *kr = k_rows + u * kstride;
+        double s = 0.0;
+        for (int d = 0; d < DQK; ++d) s += qd[d] * bf16_to_double(kr[d]);
+        s = s / root;
+        scores[u] = s;
+        if (s > smax) smax = s;
+    }
+    double den = 0.0;
+    for (int d = 0; d < DV; ++d) h[d] = 0.0;
+    for (long u = 0; u < nkeys; ++u) {
+        const uint16_t *vr = v_rows + u * vstride;
+        double w = exp(scores[u] - smax);
+        den += w;
+        for (int d = 0; d < DV; ++d) h[d] += w * bf16_to_double(vr[d]);
+    }
+    for (int d = 0; d < DV; ++d) h[d] /= den;
+}
+
+/*
+ * One output row of one group: the 4 signal heads and the noise head of group
+ * j attend over the same keys; then D_i = H_S,i - lambda_i * H_N and
+ * out_i = D_i / (1 + exp(-g_i)).
+ *   qs      : 4 signal query rows (4*DQK, consecutive heads 4j..4j+3)
+ *   qn      : the noise query row of group j
+ *   k_rows, v_rows : first visible key/value row of group j
+ *   lam     : 4 lambda values for heads 4j..4j+3
+ *   gate    : 4 x DV gate logits
+ *   out     : 4 x DV doubles
+ */
+static void group_row(const uint16_t *qs, const uint16_t *qn, const uint16_t *k_rows,
+                      const uint16_t *v_rows, long kstride, long vstride, long nkeys,
+                      const float *lam, const uint16_t *gate, double *scores, double *out) {
+    double hn[DV], hs[DV];
+    attend(qn, k_rows, v_rows, kstride, vstride, nkeys, scores, hn);
+    for (int i = 0; i < GROUP; ++i) {
+        attend(qs + (long)i * DQK, k_rows, v_rows, kstride, vstride, nkeys, scores, hs);
+        const double l = (double)lam[i];
+        for (int d = 0; d < DV; ++d) {
+            const double dd = hs[d] - l * hn[d];
+            const double g = bf16_to_double(gate[(long)i * DV + d]);
+            out[(long)i * DV + d] = dd / (1.0 + exp(-g));
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Prefill                                                                  */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t *q_sig, *q_noise, *k, *v, *gate;
+    const float *lambda;
+    int hkv, window;
+    const int64_t *row_token;  /* packed token index of each requested row */
+    const int64_t *row_seq_start; /* packed index of the row's sequence start */
+    int64_t num_rows;
+    double *out;               /* [num_rows, 4*hkv, DV] */
+    long max_keys;
+    int nthreads, tid;
+} prefill_job_t;
+
+static void *prefill_worker(void *arg) {
+    prefill_job_t *J = (prefill_job_t *)arg;
+    const int hs = GROUP * J->hkv;
+    double *scores = (double *)malloc(sizeof(double) * (size_t)(J->max_keys > 0 ? J->max_keys : 1));
+    if (!scores) return (void *)1;
+    const int64_t ntasks = J->num_rows * J->hkv;
+    for (int64_t task = J->tid; task < ntasks; task += J->nthreads) {
+        const int64_t r = task / J->hkv;
+        const int j = (int)(task % J->hkv);
+        const int64_t n = J->row_token[r];        /* packed token index */
+        const int64_t s0 = J->row_seq_start[r];   /* sequence start */
+        const int64_t t = n - s0;                 /* position in sequence */
+        int64_t lo = 0;
+        if (J->window > 0 && t - J->window + 1 > 0) lo = t - J->window + 1;
+        const long nkeys = (long)(t - lo + 1);
+        const long kstride = (long)J->hkv * DQK, vstride = (long)J->hkv * DV;
+        const uint16_t *krow = J->k + (s0 + lo) * kstride + (long)j * DQK;
+        const uint16_t *vrow = J->v + (s0 + lo) * vstride + (long)j * DV;
+        const uint16_t *qs = J->q_sig + (n * hs + (long)GROUP * j) * DQK;
+        const uint16_t *qn = J->q_noise + (n * J->hkv + j) * DQK;
+        const float *lam = J->lambda + n * hs + GROUP * j;
+        const uint16_t *gate = J->gate + (n * hs + (long)GROUP * j) * DV;
+        double *out = J->out + (r * hs + (long)GROUP * j) * DV;
+        group_row(qs, qn, krow, vrow, kstride, vstride, nkeys, lam, gate, scores, out);
+    }
+    free(scores);
+    return NULL;
+}
+
+static int run_threads(void *(*fn)(void *), void *jobs, size_t job_size, int nthreads) {
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!th) return -1;
+    int rc = 0, started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        if (pthread_create(&th[i], NULL, fn, (char *)jobs + (size_t)i * job_size) != 0) { rc = -1; break; }
+        ++started;
+    }
+    for (int i = 0; i < started; ++i) {
+        void *ret = NULL;
+        pthread_join(th[i], &ret);
+        if (ret != NULL) rc = -1;
+    }
+    free(th);
+    return rc;
+}
+
+/*
+ * Packed varlen prefill. Inputs are laid out exactly as the CUDA library's
+ * (row-major, N = sum(seqlens)):
+ *   q_sig [N, 4*hkv, 192] bf16 bits, q_noise [N, hkv, 192], k [N, hkv, 192],
+ *   v [N, hkv, 128], lambda [N, 4*hkv] fp32, gate [N, 4*hkv, 128] bf16 bits.
+ * rows: the packed token indices to evaluate (num_rows of them); out receives
+ * [num_rows, 4*hkv, 128] doubles. Returns 0, or -1 on a bad argument or an
+ * allocation/thread failure.
+ */
+int gdla_oracle_prefill(const uint16_t *q_sig, const uint16_t *q_noise, const uint16_t *k,
+                        const uint16_t *v, const float *lambda, const uint16_t *gate,
+                        int hkv, int batch, const int32_t *seqlens, int window,
+                        const int64_t *rows, int64_t num_rows, double *out, int nthreads) {
+    if (hkv < 1 || batch < 0 || num_rows < 0 || nthreads < 1) return -1;
+    int64_t total = 0;
+    long max_len = 0;
+    for (int b = 0; b < batch; ++b) {
+        if (seqlens[b] < 0) return -1;
+        total += seqlens[b];
+        if (seqlens[b] > max_len) max_len = seqlens[b];
+    }
+    int64_t *seq_start = (int64_t *)malloc(sizeof(int64_t) * (size_t)(num_rows > 0 ? num_rows : 1));
+    if (!seq_start) return -1;
+    for (int64_t r = 0; r < num_rows; ++r) {
+        const int64_t n = rows[r];
+        if (n < 0 || n >= total) { free(seq_start); return -1; }
+        int64_t s0 = 0;
+        for (int b = 0; b < batch; ++b) {
+            if (n < s0 + seqlens[b]) break;
+            s0 += seqlens[b];
+        }
+        seq_start[r] = s0;
+    }
+    prefill_job_t *jobs = (prefill_job_t *)malloc(sizeof(prefill_job_t) * (size_t)nthreads);
+    if (!jobs) { free(seq_start); return -1; }
+    for (int i = 0; i < nthreads; ++i) {
+        prefill_job_t J = {q_sig, q_noise, k, v, gate, lambda, hkv, window, rows, seq_start,
+                           num_rows, out, max_len, nthreads, i};
+        jobs[i] = J;
+    }
+    int rc = run_threads(prefill_worker, jobs, sizeof(prefill_job_t), nthreads);
+    free(jobs);
+    free(seq_start);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Decode                                                                   */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t *q_sig, *q_noise, *k, *v, *gate;
+    const float *lambda;
+    const int64_t *cu;  /* [batch+1] packed cache offsets */
+    int batch, hkv, window;
+    double *out;        /* [batch, 4*hkv, DV] */
+    long max_keys;
+    int nthreads, tid;
+} decode_job_t;
+
+static void *decode_worker(void *arg) {
+    decode_job_t *J = (decode_job_t *)arg;
+    const int hs = GROUP * J->hkv;
+    double *scores = (double *)malloc(sizeof(double) * (size_t)(J->max_keys > 0 ? J->max_keys : 1));
+    if (!scores) return (void *)1;
+    const int64_t ntasks = (int64_t)J->batch * J->hkv;
+    for (int64_t task = J->tid; task < ntasks; task += J->nthreads) {
+        const int64_t b = task / J->hkv;
+        const int j = (int)(task % J->hkv);
+        const int64_t s0 = J->cu[b];
+        const int64_t len = J->cu[b + 1] - s0;
+        const int64_t t = len - 1;              /* the query's own position */
+        int64_t lo = 0;
+        if (J->window > 0 && t - J->window + 1 > 0) lo = t - J->window + 1;
+        const long nkeys = (long)(t - lo + 1);
+        const long kstride = (long)J->hkv * DQK, vstride = (long)J->hkv * DV;
+        const uint16_t *krow = J->k + (s0 + lo) * kstride + (long)j * DQK;
+        const uint16_t *vrow = J->v + (s0 + lo) * vstride + (long)j * DV;
+        const uint16_t *qs = J->q_sig + (b * hs + (long)GROUP * j) * DQK;
+        const uint16_t *qn = J->q_noise + (b * J->hkv + j) * DQK;
+        const float *lam = J->lambda + b * hs + GROUP * j;
+        const uint16_t *gate = J->gate + (b * hs + (long)GROUP * j) * DV;
+        double *out = J->out + (b * hs + (long)GROUP * j) * DV;
+        group_row(qs, qn, krow, vrow, kstride, vstride, nkeys, lam, gate, scores, out);
+    }
+    free(scores);
+    return NULL;
+}
+
+/*
+ * Varlen decode: one query per sequence at position L_b - 1.
+ *   q_sig [B, 4*hkv, 192], q_noise [B, hkv, 192], k_cache [Nk, hkv, 192],
+ *   v_cache [Nk, hkv, 128] (sequence b owns rows cu[b]..cu[b+1]-1),
+ *   lambda [B, 4*hkv] fp32, gate [B, 4*hkv, 128]; out [B, 4*hkv, 128] doubles.
+ * Every L_b must be >= 1. Returns 0, or -1 on a bad argument.
+ */
+int gdla_oracle_decode(const uint16_t *q_sig, const uint16_t *q_noise, const uint16_t *k_cache,
+                       const uint16_t *v_cache, const int64_t *cu_seqlens_k, const float *lambda,
+                       const uint16_t *gate, int batch, int hkv, int window, double *out,
+                       int nthreads) {
+    if (hkv < 1 || batch < 0 || nthreads < 1) return -1;
+    long max_len = 0;
+    for (int b = 0; b < batch; ++b) {
+        const int64_t len = cu_seqlens_k[b + 1] - cu_seqlens_k[b];
+        if (len < 1) return -1;
+        if (len > max_len) max_len = (long)len;
+    }
+    decode_job_t *jobs = (decode_job_t *)malloc(sizeof(decode_job_t) * (size_t)nthreads);
+    if (!jobs) return -1;
+    for (int i = 0; i < nthreads; ++i) {
+        decode_job_t J = {q_sig, q_noise, k_cache, v_cache, gate, lambda, cu_seqlens_k,
+                          batch, hkv, window, out, max_len, nthreads, i};
+        jobs[i] = J;
+    }
+    int rc = run_threads(decode_worker, jobs, sizeof(decode_job_t), nthreads);
+    free(jobs);
+    return rc;
+}

@@ -1,0 +1,11 @@
+"""GDLA (Grouped Differential Latent Attention) forward core for NVIDIA B200.
+
+Python binding of the C-ABI library ``libgdla.so`` (hand-written sm_100a CUDA
+kernels). PyTorch supplies device memory and streams; the computation happens
+only in the library. See ``include/gdla.h`` for the ABI.
+"""
+from .ops import (DQK, DV, GROUP, GDLAError, attn_decode, attn_fwd, decode_workspace_bytes, device_error,
+                  library)
+
+__all__ = ["attn_fwd", "attn_decode", "decode_workspace_bytes", "device_error", "library", "GDLAError",
+           "GROUP", "DQK", "DV"]

@@ -1,0 +1,232 @@
+// gdla_api.cu - the C ABI declared in include/gdla.h: argument checks, the
+// prefill tile plan, the decode split plan, TMA tensor maps and the launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <memory>
+#include <mutex>
+#include <vector>
+
+#include "gdla.h"
+#include "gdla_internal.h"
+#include "gdla_ptx.cuh"
+
+namespace gdla {
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 3-D bf16 tensor [d2][d1][d0] (d0 contiguous), 128-byte swizzled boxes.
+bool make_map(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1,
+              uint32_t b2) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct TileItem {
+    int cost;  // key tiles the q-tile visits
+    int seq;
+    int qt;
+};
+
+}  // namespace
+
+DecodePlan make_decode_plan(int batch, int hkv, int max_seqlen_k, int window, int num_cache_rows) {
+    DecodePlan p{};
+    p.batch = batch;
+    p.hkv = hkv;
+    p.window = window;
+    p.max_seqlen_k = max_seqlen_k;
+    p.num_cache_rows = num_cache_rows;
+    const int eff = (window > 0) ? std::min(window, max_seqlen_k) : max_seqlen_k;
+    int ns = std::max(1, (eff + kDecodeMinSplitKeys - 1) / kDecodeMinSplitKeys);
+    ns = std::min(ns, kDecodeMaxSplits);
+    int keys = (eff + ns - 1) / ns;
+    keys = (keys + 63) / 64 * 64;
+    p.split_keys = keys;
+    p.num_splits = (eff + keys - 1) / keys;
+    p.ml_offset_floats = static_cast<long long>(batch) * hkv * p.num_splits * 5 * 128;
+    return p;
+}
+
+size_t decode_workspace_bytes(const DecodePlan &p) {
+    if (p.num_splits <= 1) return 0;
+    return static_cast<size_t>(p.batch) * p.hkv * p.num_splits * 5 * (128 + 2) * sizeof(float);
+}
+
+}  // namespace gdla
+
+using namespace gdla;
+
+extern "C" {
+
+gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k, const void *v,
+                            const float *lambda, const void *gate_logits, void *out, int batch,
+                            const int32_t *seqlens, int num_kv_heads, int window, void *stream) {
+    if (batch < 1 || seqlens == nullptr) return GDLA_ERR_INVALID_ARG;
+    if (num_kv_heads < 1 || num_kv_heads > GDLA_MAX_KV_HEADS) return GDLA_ERR_UNSUPPORTED;
+    long long n_total = 0;
+    for (int b = 0; b < batch; ++b) {
+        if (seqlens[b] < 0) return GDLA_ERR_INVALID_ARG;
+        n_total += seqlens[b];
+    }
+    if (n_total >= (1ll << 31)) return GDLA_ERR_INVALID_ARG;
+    if (n_total == 0) return GDLA_OK;
+    if (!aligned16(q_sig) || !aligned16(q_noise) || !aligned16(k) || !aligned16(v) || !aligned16(lambda) ||
+        !aligned16(gate_logits) || !aligned16(out))
+        return GDLA_ERR_INVALID_ARG;
+
+    const int hkv = num_kv_heads;
+    const int T = kPrefillTileTokens;
+    // ---- tile plan: every (sequence, q-tile), heaviest first ----
+    std::vector<TileItem> items;
+    std::vector<int> seq_start(batch);
+    {
+        long long s0 = 0;
+        for (int b = 0; b < batch; ++b) {
+            seq_start[b] = static_cast<int>(s0);
+            const int L = seqlens[b];
+            s0 += L;
+            const int nqt = (L + T - 1) / T;
+            for (int qt = 0; qt < nqt; ++qt) {
+                const int t0 = qt * T;
+                const int lo = (window > 0) ? std::max(0, t0 - window + 1) : 0;
+                const int hi = std::min(L, t0 + T);
+                items.push_back({(hi - lo + kPrefillKeyTile - 1) / kPrefillKeyTile, b, qt});
+            }
+        }
+    }
+    std::stable_sort(items.begin(), items.end(), [](const TileItem &a, const TileItem &b) {
+        if (a.cost != b.cost) return a.cost > b.cost;
+        if (a.seq != b.seq) return a.seq < b.seq;
+        return a.qt > b.qt;
+    });
+
+    PrefillLaunch L{};
+    const uint64_t N = static_cast<uint64_t>(n_total);
+    if (!make_map(&L.tm_qs, q_sig, 192, 4 * hkv, N, 64, 4, T) || !make_map(&L.tm_qn, q_noise, 192, hkv, N, 64, 1, T) ||
+        !make_map(&L.tm_k, k, 192, hkv, N, 64, 1, kPrefillKeyTile) ||
+        !make_map(&L.tm_v, v, 128, hkv, N, 64, 1, kPrefillKeyTile))
+        return GDLA_ERR_CUDA;
+    L.lambda = lambda;
+    L.gate = static_cast<const __nv_bfloat16 *>(gate_logits);
+    L.out = static_cast<__nv_bfloat16 *>(out);
+
+    std::unique_ptr<PrefillPlan> plan(new PrefillPlan());
+    std::vector<int> local(batch, -1);
+    size_t pos = 0;
+    while (pos < items.size()) {
+        PrefillPlan &P = *plan;
+        P.n_items = 0;
+        P.hkv = hkv;
+        P.window = window;
+        int n_seq = 0;
+        std::vector<int> used;
+        while (pos < items.size() && P.n_items < kPlanMaxItems) {
+            const TileItem &it = items[pos];
+            if (local[it.seq] < 0) {
+                if (n_seq == kPlanMaxSeqs) break;
+                local[it.seq] = n_seq;
+                P.seq_start[n_seq] = seq_start[it.seq];
+                P.seq_len[n_seq] = seqlens[it.seq];
+                used.push_back(it.seq);
+                ++n_seq;
+            }
+            P.items[P.n_items++] = (static_cast<uint32_t>(local[it.seq]) << kItemSeqShift) |
+                                   static_cast<uint32_t>(it.qt);
+            ++pos;
+        }
+        for (int s : used) local[s] = -1;
+        if (launch_prefill(L, P, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDLA_ERR_CUDA;
+    }
+    return GDLA_OK;
+}
+
+size_t gdla_decode_workspace_bytes(int batch, int num_kv_heads, int max_seqlen_k, int window) {
+    if (batch < 1 || num_kv_heads < 1 || num_kv_heads > GDLA_MAX_KV_HEADS || max_seqlen_k < 1) return 0;
+    return decode_workspace_bytes(make_decode_plan(batch, num_kv_heads, max_seqlen_k, window, 1));
+}
+
+gdla_status_t gdla_attn_decode(const void *q_sig, const void *q_noise, const void *k_cache, const void *v_cache,
+                               const int32_t *cu_seqlens_k, int num_cache_rows, int max_seqlen_k,
+                               const float *lambda, const void *gate_logits, void *out, int batch, int num_kv_heads,
+                               int window, void *workspace, size_t workspace_bytes, void *stream) {
+    if (batch < 1 || num_cache_rows < 1 || max_seqlen_k < 1) return GDLA_ERR_INVALID_ARG;
+    if (num_kv_heads < 1 || num_kv_heads > GDLA_MAX_KV_HEADS) return GDLA_ERR_UNSUPPORTED;
+    if (!aligned16(q_sig) || !aligned16(q_noise) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(lambda) || !aligned16(gate_logits) || !aligned16(out) || cu_seqlens_k == nullptr ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+        return GDLA_ERR_INVALID_ARG;
+    const DecodePlan plan = make_decode_plan(batch, num_kv_heads, max_seqlen_k, window, num_cache_rows);
+    const size_t need = decode_workspace_bytes(plan);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need ||
+                     (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+        return GDLA_ERR_WORKSPACE;
+    DecodeLaunch L{};
+    const uint64_t nk = static_cast<uint64_t>(num_cache_rows);
+    if (!make_map(&L.tm_k, k_cache, 192, num_kv_heads, nk, 64, 1, 64) ||
+        !make_map(&L.tm_v, v_cache, 128, num_kv_heads, nk, 64, 1, 64))
+        return GDLA_ERR_CUDA;
+    L.q_sig = static_cast<const __nv_bfloat16 *>(q_sig);
+    L.q_noise = static_cast<const __nv_bfloat16 *>(q_noise);
+    L.cu_seqlens_k = cu_seqlens_k;
+    L.lambda = lambda;
+    L.gate = static_cast<const __nv_bfloat16 *>(gate_logits);
+    L.out = static_cast<__nv_bfloat16 *>(out);
+    L.ws = static_cast<float *>(workspace);
+    if (launch_decode(L, plan, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDLA_ERR_CUDA;
+    return GDLA_OK;
+}
+
+int gdla_device_error(int clear) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return -1;
+    if (clear) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return -1;
+    }
+    return v;
+}
+
+const char *gdla_status_string(gdla_status_t status) {
+    switch (status) {
+        case GDLA_OK: return "GDLA_OK";
+        case GDLA_ERR_INVALID_ARG: return "GDLA_ERR_INVALID_ARG: null, misaligned or out-of-range argument";
+        case GDLA_ERR_UNSUPPORTED: return "GDLA_ERR_UNSUPPORTED: sizes outside what the kernels handle";
+        case GDLA_ERR_WORKSPACE: return "GDLA_ERR_WORKSPACE: decode workspace missing, misaligned or too small";
+        case GDLA_ERR_CUDA: return "GDLA_ERR_CUDA: a CUDA call or kernel launch failed";
+    }
+    return "GDLA: unknown status";
+}
+
+int gdla_version(void) { return GDLA_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,72 @@
+// gdla_internal.h - launch plans shared between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdla {
+
+// Prefill: one CTA tile = 24 tokens x 5 heads = 120 of the 128 MMA rows.
+constexpr int kPrefillTileTokens = 24;
+constexpr int kPrefillKeyTile = 128;
+constexpr int kPlanMaxSeqs = 256;    // sequences per launch (more are split across launches)
+constexpr int kPlanMaxItems = 6144;  // q-tiles per launch
+constexpr int kItemSeqShift = 20;
+constexpr uint32_t kItemTileMask = (1u << kItemSeqShift) - 1u;
+
+// Passed by value (constant bank): the q-tiles of one launch, heaviest first.
+struct PrefillPlan {
+    int n_items;
+    int hkv;
+    int window;
+    int pad_;
+    int seq_start[kPlanMaxSeqs];  // packed row of each sequence's first token
+    int seq_len[kPlanMaxSeqs];
+    uint32_t items[kPlanMaxItems];  // (local sequence << kItemSeqShift) | q-tile index
+};
+
+struct PrefillLaunch {
+    CUtensorMap tm_qs, tm_qn, tm_k, tm_v;
+    const float *lambda;
+    const __nv_bfloat16 *gate;
+    __nv_bfloat16 *out;
+};
+
+cudaError_t launch_prefill(const PrefillLaunch &launch, const PrefillPlan &plan, cudaStream_t stream);
+int prefill_smem_bytes();
+
+// Decode: split-KV.
+constexpr int kDecodeMaxSplits = 64;
+constexpr int kDecodeMinSplitKeys = 1024;
+
+struct DecodePlan {
+    int batch;
+    int hkv;
+    int window;
+    int max_seqlen_k;
+    int num_cache_rows;
+    int num_splits;
+    int split_keys;        // keys per split (multiple of 64)
+    long long ml_offset_floats;  // start of the (m, l) area in the workspace, in floats
+};
+
+struct DecodeLaunch {
+    CUtensorMap tm_k, tm_v;
+    const __nv_bfloat16 *q_sig, *q_noise;
+    const int32_t *cu_seqlens_k;
+    const float *lambda;
+    const __nv_bfloat16 *gate;
+    __nv_bfloat16 *out;
+    float *ws;
+};
+
+cudaError_t launch_decode(const DecodeLaunch &launch, const DecodePlan &plan, cudaStream_t stream);
+int decode_smem_bytes();
+
+// Host-side decode split plan (shared by the workspace query and the launch).
+DecodePlan make_decode_plan(int batch, int hkv, int max_seqlen_k, int window, int num_cache_rows);
+size_t decode_workspace_bytes(const DecodePlan &plan);
+
+}  // namespace gdla

@@ -1,0 +1,157 @@
+"""ctypes binding of libgdla.so: argument marshalling only.
+
+Every step of the GDLA core runs in the library's CUDA kernels; PyTorch only
+provides device memory and the current CUDA stream. There is no fallback: if
+libgdla.so is missing or cannot be loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import numpy as np
+import torch
+
+from . import _build
+
+GROUP, DQK, DV = 4, 192, 128
+MAX_KV_HEADS = 64
+
+STATUS = {0: "GDLA_OK", 1: "GDLA_ERR_INVALID_ARG", 2: "GDLA_ERR_UNSUPPORTED", 3: "GDLA_ERR_WORKSPACE",
+          4: "GDLA_ERR_CUDA"}
+EXPORTED = ("gdla_attn_fwd", "gdla_decode_workspace_bytes", "gdla_attn_decode", "gdla_device_error",
+            "gdla_status_string", "gdla_version")
+
+_lib = None
+_lock = threading.Lock()
+
+
+class GDLAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {library().gdla_status_string(status).decode()}")
+
+
+def library():
+    """The loaded libgdla.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.LIB_PATH
+            if not os.path.exists(path):
+                raise RuntimeError(f"{path} is missing; build it with `python -m "
+                                   f"differential_latent_attention_b200._build` (no fallback path exists)")
+            lib = ctypes.CDLL(path)
+            p, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+            lib.gdla_attn_fwd.argtypes = [p, p, p, p, p, p, p, i, p, i, i, p]
+            lib.gdla_attn_fwd.restype = i
+            lib.gdla_decode_workspace_bytes.argtypes = [i, i, i, i]
+            lib.gdla_decode_workspace_bytes.restype = sz
+            lib.gdla_attn_decode.argtypes = [p, p, p, p, p, i, i, p, p, p, i, i, i, p, sz, p]
+            lib.gdla_attn_decode.restype = i
+            lib.gdla_device_error.argtypes = [i]
+            lib.gdla_device_error.restype = i
+            lib.gdla_status_string.argtypes = [i]
+            lib.gdla_status_string.restype = ctypes.c_char_p
+            lib.gdla_version.argtypes = []
+            lib.gdla_version.restype = i
+            _lib = lib
+    return _lib
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(t, name, dtype, shape):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def attn_fwd(q_sig, q_noise, k, v, lam, gate, seqlens, window=0, out=None, stream=None):
+    """Packed varlen GDLA prefill (calls ``gdla_attn_fwd``).
+
+    q_sig [N, 4H, 192], q_noise [N, H, 192], k [N, H, 192], v [N, H, 128] and
+    gate [N, 4H, 128] are bf16 CUDA tensors, lam [N, 4H] fp32; ``seqlens`` is a
+    host sequence of per-sequence lengths summing to N. Returns out [N, 4H, 128]
+    bf16 (written into ``out`` when given).
+    """
+    lens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32).reshape(-1))
+    n = int(lens.astype(np.int64).sum())
+    hkv = q_noise.shape[1] if q_noise.dim() == 3 else -1
+    hs = GROUP * hkv
+    _check(q_sig, "q_sig", torch.bfloat16, (n, hs, DQK))
+    _check(q_noise, "q_noise", torch.bfloat16, (n, hkv, DQK))
+    _check(k, "k", torch.bfloat16, (n, hkv, DQK))
+    _check(v, "v", torch.bfloat16, (n, hkv, DV))
+    _check(lam, "lam", torch.float32, (n, hs))
+    _check(gate, "gate", torch.bfloat16, (n, hs, DV))
+    if out is None:
+        out = torch.empty((n, hs, DV), dtype=torch.bfloat16, device=q_sig.device)
+    _check(out, "out", torch.bfloat16, (n, hs, DV))
+    st = library().gdla_attn_fwd(_ptr(q_sig), _ptr(q_noise), _ptr(k), _ptr(v), _ptr(lam), _ptr(gate), _ptr(out),
+                                 int(lens.shape[0]), lens.ctypes.data_as(ctypes.c_void_p), hkv, int(window),
+                                 _stream(stream))
+    if st != 0:
+        raise GDLAError(st, "gdla_attn_fwd")
+    return out
+
+
+def decode_workspace_bytes(batch, num_kv_heads, max_seqlen_k, window=0):
+    return int(library().gdla_decode_workspace_bytes(int(batch), int(num_kv_heads), int(max_seqlen_k),
+                                                     int(window)))
+
+
+def attn_decode(q_sig, q_noise, k_cache, v_cache, cu_seqlens_k, max_seqlen_k, lam, gate, window=0, out=None,
+                workspace=None, stream=None):
+    """Varlen GDLA decode (calls ``gdla_attn_decode``).
+
+    One query per sequence: q_sig [B, 4H, 192], q_noise [B, H, 192], lam [B, 4H],
+    gate [B, 4H, 128]; k_cache [Nk, H, 192] and v_cache [Nk, H, 128] hold the
+    sequences back to back as given by the int32 CUDA tensor cu_seqlens_k [B+1].
+    ``workspace`` (uint8 CUDA tensor) is allocated here when not given.
+    """
+    b = q_sig.shape[0]
+    hkv = q_noise.shape[1] if q_noise.dim() == 3 else -1
+    hs = GROUP * hkv
+    nk = k_cache.shape[0]
+    _check(q_sig, "q_sig", torch.bfloat16, (b, hs, DQK))
+    _check(q_noise, "q_noise", torch.bfloat16, (b, hkv, DQK))
+    _check(k_cache, "k_cache", torch.bfloat16, (nk, hkv, DQK))
+    _check(v_cache, "v_cache", torch.bfloat16, (nk, hkv, DV))
+    _check(cu_seqlens_k, "cu_seqlens_k", torch.int32, (b + 1,))
+    _check(lam, "lam", torch.float32, (b, hs))
+    _check(gate, "gate", torch.bfloat16, (b, hs, DV))
+    if out is None:
+        out = torch.empty((b, hs, DV), dtype=torch.bfloat16, device=q_sig.device)
+    _check(out, "out", torch.bfloat16, (b, hs, DV))
+    need = decode_workspace_bytes(b, hkv, max_seqlen_k, window)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_sig.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = library().gdla_attn_decode(_ptr(q_sig), _ptr(q_noise), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens_k),
+                                    int(nk), int(max_seqlen_k), _ptr(lam), _ptr(gate), _ptr(out), int(b), hkv,
+                                    int(window), _ptr(workspace), ws_bytes, _stream(stream))
+    if st != 0:
+        raise GDLAError(st, "gdla_attn_decode")
+    return out
+
+
+def device_error(clear=True) -> int:
+    """Code recorded by a kernel whose bounded wait ran out (0 = none); synchronises."""
+    return int(library().gdla_device_error(1 if clear else 0))

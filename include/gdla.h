@@ -25,8 +25,9 @@
  *  - All tensors are dense, row-major, caller-owned DEVICE memory unless a
  *    comment says HOST. Tensor base pointers must be 16-byte aligned.
  *  - bf16 is IEEE bfloat16 (1-8-7); lambda is fp32.
- *  - The library allocates no memory, keeps no state between calls and may
- *    be called from several host threads at once.
+ *  - The library allocates no memory, keeps no state between calls (apart
+ *    from the device-side failure word, see gdla_device_error) and may be
+ *    called from several host threads at once.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
  *    default stream). GDLA_OK means every kernel was enqueued; a CUDA launch
  *    failure is reported as GDLA_ERR_CUDA.
@@ -43,6 +44,12 @@
 
 #ifdef __cplusplus
 extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GDLA_API __attribute__((visibility("default")))
+#else
+#define GDLA_API
 #endif
 
 #define GDLA_GROUP 4          /* signal heads per noise / KV head (g) */
@@ -83,7 +90,7 @@ typedef enum {
  * GDLA_ERR_UNSUPPORTED for num_kv_heads out of range; GDLA_ERR_CUDA if a
  * launch fails. N == 0 returns GDLA_OK without launching.
  */
-gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k, const void *v,
+GDLA_API gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *k, const void *v,
                             const float *lambda, const void *gate_logits, void *out,
                             int batch, const int32_t *seqlens, int num_kv_heads, int window,
                             void *stream);
@@ -93,7 +100,7 @@ gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *
  * no split-KV pass is used). Returns 0 for invalid sizes as well; the
  * workspace must be 256-byte aligned.
  */
-size_t gdla_decode_workspace_bytes(int batch, int num_kv_heads, int max_seqlen_k, int window);
+GDLA_API size_t gdla_decode_workspace_bytes(int batch, int num_kv_heads, int max_seqlen_k, int window);
 
 /*
  * Varlen decode: one new query token per sequence, attending over that
@@ -107,7 +114,10 @@ size_t gdla_decode_workspace_bytes(int batch, int num_kv_heads, int max_seqlen_k
  *   v_cache      bf16 [Nk, num_kv_heads, 128]
  *   cu_seqlens_k DEVICE int32 [batch + 1]: sequence b owns cache rows
  *                cu[b] .. cu[b+1]-1; every L_b = cu[b+1]-cu[b] must be in
- *                1 .. max_seqlen_k (a violating sequence's output is zeroed)
+ *                1 .. max_seqlen_k and cu[b+1] <= num_cache_rows (a
+ *                sequence that violates this gets an all-zero output)
+ *   num_cache_rows HOST number of rows Nk in k_cache / v_cache, >= 1; reads
+ *                never go past it
  *   max_seqlen_k HOST upper bound on every L_b, >= 1 (sizes the split plan)
  *   lambda       fp32 [batch, 4*num_kv_heads]
  *   gate_logits  bf16 [batch, 4*num_kv_heads, 128]
@@ -118,21 +128,31 @@ size_t gdla_decode_workspace_bytes(int batch, int num_kv_heads, int max_seqlen_k
  *                max_seqlen_k, window) bytes, 256-byte aligned (may be NULL
  *                when that is 0); its contents need no initialisation
  * Errors: GDLA_ERR_INVALID_ARG (null/misaligned pointers, batch < 1,
- * max_seqlen_k < 1), GDLA_ERR_UNSUPPORTED (num_kv_heads out of range),
+ * num_cache_rows < 1, max_seqlen_k < 1), GDLA_ERR_UNSUPPORTED (num_kv_heads out of range),
  * GDLA_ERR_WORKSPACE (workspace NULL or smaller than required),
  * GDLA_ERR_CUDA (launch failure).
  */
-gdla_status_t gdla_attn_decode(const void *q_sig, const void *q_noise, const void *k_cache,
-                               const void *v_cache, const int32_t *cu_seqlens_k, int max_seqlen_k,
+GDLA_API gdla_status_t gdla_attn_decode(const void *q_sig, const void *q_noise, const void *k_cache,
+                               const void *v_cache, const int32_t *cu_seqlens_k, int num_cache_rows,
+                               int max_seqlen_k,
                                const float *lambda, const void *gate_logits, void *out,
                                int batch, int num_kv_heads, int window,
                                void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Device-side failure word. Every wait inside the kernels is bounded (about
+ * one second of SM clock); a wait that runs out makes its CTA wind down and
+ * records a nonzero code here instead of hanging the GPU. This call
+ * synchronises the current device, returns the recorded code (0 = none) and,
+ * if `clear` is nonzero, resets it. Returns -1 if the device cannot be read.
+ */
+GDLA_API int gdla_device_error(int clear);
+
 /* Static, human-readable name of a status code. */
-const char *gdla_status_string(gdla_status_t status);
+GDLA_API const char *gdla_status_string(gdla_status_t status);
 
 /* GDLA_VERSION of the loaded library. */
-int gdla_version(void);
+GDLA_API int gdla_version(void);
 
 #ifdef __cplusplus
 }

@@ -1,0 +1,76 @@
+"""GPU parity of gdla_attn_decode (through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import differential_latent_attention_b200 as gdla
+import gdla_inputs as gi
+import oracle
+from _parity import assert_close, decode_host_args, gpu_decode, gpu_prefill, host_args
+
+pytestmark = pytest.mark.gpu
+
+EDGE_LENS = (1, 2, 63, 64, 65, 127, 128, 129, 1023, 1024, 1025, 2047, 2048, 2049, 5000)
+
+
+def _check(lengths, hkv, window, seed, max_len=None):
+    d = gi.make_decode_inputs(lengths, hkv, seed, device="cuda")
+    max_len = int(max(lengths)) if max_len is None else max_len
+    out = gpu_decode(d, max_len, window)
+    torch.cuda.synchronize()
+    assert gdla.device_error() == 0
+    ref = oracle.decode(*decode_host_args(d), window)
+    return assert_close(out.float().cpu().numpy(), ref, f"decode lengths={lengths} window={window}")
+
+
+@pytest.mark.parametrize("window", [0, 1, 128, 129, 3000])
+def test_edge_lengths(window):
+    _check(EDGE_LENS, 2, window, 50 + window)
+
+
+def test_split_boundaries():
+    # max_seqlen_k 5000 -> 5 splits of 1024 keys; lengths at split edges +-1
+    _check((1023, 1024, 1025, 2048, 2049, 4095, 4096, 4097, 5000), 1, 0, 51, max_len=5000)
+
+
+def test_max_len_larger_than_needed():
+    _check((700, 1300), 3, 0, 52, max_len=40000)
+
+
+def test_decode_equals_last_prefill_row():
+    lengths = (3, 700, 2500)
+    t = gi.make_prefill_inputs(lengths, 2, 53, device="cuda")
+    last = torch.as_tensor(np.cumsum(lengths) - 1, device="cuda")
+    cu = torch.as_tensor(np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32), device="cuda")
+    pre = gpu_prefill(t, lengths, 0)
+    d = {"q_sig": t["q_sig"][last].contiguous(), "q_noise": t["q_noise"][last].contiguous(),
+         "k_cache": t["k"], "v_cache": t["v"], "cu_seqlens_k": cu, "lam": t["lam"][last].contiguous(),
+         "gate": t["gate"][last].contiguous()}
+    dec = gpu_decode(d, max(lengths), 0)
+    torch.cuda.synchronize()
+    assert_close(dec.float().cpu().numpy(), pre[last].double().cpu().numpy(), "decode vs prefill last row")
+
+
+def test_invalid_lengths_give_zero_output():
+    lengths = (10, 20)
+    d = gi.make_decode_inputs(lengths, 1, 54, device="cuda")
+    cu = d["cu_seqlens_k"].clone()
+    cu[1] = cu[0]          # sequence 0 empty, sequence 1 then 30 rows long
+    d["cu_seqlens_k"] = cu
+    out = gpu_decode(d, 20, 0)        # 30 > max_seqlen_k for sequence 1 as well
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out.float()) == 0
+
+
+def test_deterministic():
+    d = gi.make_decode_inputs((3000, 5000, 17), 2, 55, device="cuda")
+    a = gpu_decode(d, 5000, 0).clone()
+    b = gpu_decode(d, 5000, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.parametrize("w", [gi.DECODE_FULL, gi.DECODE_W128], ids=lambda w: w.name)
+def test_decode_B64_H16(w):
+    lengths = w.kv_lengths()
+    _check(tuple(int(x) for x in lengths), w.num_kv_heads, w.window, w.seed, max_len=32768)

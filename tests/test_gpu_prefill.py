@@ -1,0 +1,110 @@
+"""GPU parity of gdla_attn_fwd (through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import differential_latent_attention_b200 as gdla
+import gdla_inputs as gi
+import oracle
+from _parity import assert_close, check_prefill, gpu_prefill, host_args
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_all_rows():
+    w = gi.TINY
+    check_prefill(w.seqlens, w.num_kv_heads, w.window, w.seed)
+
+
+EDGE_SEQS = (1, 63, 64, 65, 127, 128, 129, 23, 24, 25, 0, 47, 48, 49, 300)
+
+
+@pytest.mark.parametrize("window", [0, 1, 2, 24, 127, 128, 129, 4096])
+def test_ragged_batch_all_rows(window):
+    check_prefill(EDGE_SEQS, 2, window, 100 + max(window, 0))
+
+
+@pytest.mark.parametrize("hkv", [1, 3, 5])
+def test_kv_head_counts(hkv):
+    check_prefill((200, 77), hkv, 0, 7)
+
+
+def test_several_key_tiles_and_ragged_tail():
+    # 1000 tokens: 8 key tiles of 128, a ragged last q-tile (1000 = 41*24 + 16)
+    check_prefill((1000,), 2, 0, 8)
+    check_prefill((1000,), 2, 128, 9)
+
+
+def test_every_row_written_and_deterministic():
+    seqlens = (5, 130, 1, 64)
+    t = gi.make_prefill_inputs(seqlens, 2, 11, device="cuda")
+    out = torch.full((sum(seqlens), 8, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gpu_prefill(t, seqlens, 0, out=out)
+    first = out.clone()
+    gpu_prefill(t, seqlens, 0, out=out)
+    torch.cuda.synchronize()
+    assert torch.isfinite(first.float()).all()
+    assert torch.equal(first.view(torch.int16), out.view(torch.int16))
+
+
+def test_empty_batch_is_a_no_op():
+    """Zero tokens: the call returns GDLA_OK without launching anything."""
+    import ctypes
+    lib = gdla.library()
+    lens = np.zeros(2, dtype=np.int32)
+    buf = torch.empty(64, dtype=torch.uint8, device="cuda")
+    p = ctypes.c_void_p(buf.data_ptr())
+    assert lib.gdla_attn_fwd(p, p, p, p, p, p, p, 2, lens.ctypes.data_as(ctypes.c_void_p), 1, 0, None) == 0
+
+
+def test_identical_paths_cancel_exactly():
+    """Signal queries equal to their noise query and lambda = 1: the signal and
+    noise rows of a tile see identical inputs, so D = 0 exactly on the GPU too."""
+    seqlens = (150, 40)
+    t = gi.make_prefill_inputs(seqlens, 2, 12, device="cuda")
+    t["q_sig"] = t["q_noise"].repeat_interleave(4, dim=1).contiguous()
+    t["lam"] = torch.ones_like(t["lam"])
+    out = gpu_prefill(t, seqlens, 0)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out.float()) == 0
+
+
+def test_lambda_zero_gate_open_is_gqa_attention():
+    """lambda = 0, gate logit 40: the GPU output is plain causal GQA attention,
+    checked against torch's SDPA (float64, CPU) rather than the oracle."""
+    import torch.nn.functional as F
+    seqlens = (300,)
+    t = gi.make_prefill_inputs(seqlens, 2, 13, device="cuda")
+    t["lam"] = torch.zeros_like(t["lam"])
+    t["gate"] = torch.full_like(t["gate"], 40.0)
+    out = gpu_prefill(t, seqlens, 0).float().cpu().numpy()
+    q = t["q_sig"].double().cpu().permute(1, 0, 2)[None]
+    k = t["k"].double().cpu().permute(1, 0, 2)[None]
+    v = t["v"].double().cpu().permute(1, 0, 2)[None]
+    ref = F.scaled_dot_product_attention(q, k, v, is_causal=True, enable_gqa=True)[0].permute(1, 0, 2).numpy()
+    assert_close(out, ref, "lambda=0 vs SDPA")
+
+
+def test_prefill_full_T4096_sampled_rows():
+    """The bench's own workload and launch: T=4096, 16 KV groups, full causal."""
+    w = gi.PREFILL_FULL
+    rows = gi.sample_rows(w.seqlens, 512, seed=1, must_include=(0, 1, 23, 24, 127, 128, 4095))
+    check_prefill(w.seqlens, w.num_kv_heads, w.window, w.seed, rows=rows)
+
+
+def test_swa_B2_T32768_sampled_rows():
+    w = gi.SWA
+    rows = gi.sample_rows(w.seqlens, 512, seed=2, must_include=(0, 1, 126, 127, 128, 129))
+    check_prefill(w.seqlens, w.num_kv_heads, w.window, w.seed, rows=rows)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("layer", [0, 1, 2, 3])
+def test_hybrid_T65536_layers_sampled_rows(layer):
+    w = gi.HYBRID_LAYERS[layer]
+    rows = gi.sample_rows(w.seqlens, 512, seed=40 + layer, must_include=(0, 1, 127, 128, 65535))
+    check_prefill(w.seqlens, w.num_kv_heads, w.window, w.seed, rows=rows)
+
+
+def test_no_device_error_recorded():
+    assert gdla.device_error(clear=True) == 0

@@ -1,0 +1,403 @@
+#!/usr/bin/env python
+"""Benchmark of the GDLA forward core (libgdla.so) on B200.
+
+Headline: packed prefill, batch 1, T = 4096, 64 signal + 16 noise query heads
+over 16 KV heads (dqk 192, dv 128), full causal, in TFLOP/s of algorithmic
+work (80 heads x (2*192 + 2*128) flops per visible query/key pair). The same
+JSON line carries the sliding-window-128 prefill and the varlen decode
+workloads (tokens/s and HBM GB/s) under "extra".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gdla|reference]
+
+N > 1 runs under torch.distributed.run, one rank per GPU: every rank runs the
+same workload on its own GPU (independent problems, no collective on the data
+path), timing is the max over ranks and "value" counts the work of all ranks.
+``--impl reference`` times the fp64 CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import gdla_inputs as gi  # noqa: E402
+
+METRIC = "GDLA fwd TFLOP/s (full causal) & tokens/s (SWA-128, decode) vs B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 512 << 20
+FLOPS_PER_PAIR_HEAD = 2 * 192 + 2 * 128
+PREFILL_KERNEL = "gdla_prefill_kernel"
+
+
+# ------------------------------------------------------------------ workloads
+def prefill_flops(w: gi.PrefillWorkload) -> float:
+    return float(w.visible_pairs()) * 5 * w.num_kv_heads * FLOPS_PER_PAIR_HEAD
+
+
+def prefill_bytes(w: gi.PrefillWorkload) -> float:
+    hkv, hs = w.num_kv_heads, 4 * w.num_kv_heads
+    per_token = 2 * (hs * 192 + hkv * 192 + hkv * 192 + hkv * 128 + hs * 128 + hs * 128) + 4 * hs
+    return float(w.tokens) * per_token
+
+
+def decode_bytes(lengths, hkv, window) -> float:
+    hs = 4 * hkv
+    keys = sum(min(int(l), window) if window > 0 else int(l) for l in lengths)
+    per_query = 2 * (hs * 192 + hkv * 192 + hs * 128 + hs * 128) + 4 * hs
+    return float(keys) * hkv * (192 + 128) * 2 + len(lengths) * per_query
+
+
+def decode_flops(lengths, hkv, window) -> float:
+    keys = sum(min(int(l), window) if window > 0 else int(l) for l in lengths)
+    return float(keys) * 5 * hkv * FLOPS_PER_PAIR_HEAD
+
+
+# ------------------------------------------------------------------ plumbing
+def dist_info():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    """Max of a float over ranks (identity for one rank)."""
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"]))}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "differential_latent_attention_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch recorded in profiles/ by an ncu capture, or None if
+    there is none or the kernel sources changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}__{workload}.txt")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_t = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
+    m_h = re.search(r"^kernel_sources_sha256_16:\s*([0-9a-f]+)", text, re.M)
+    if not m_t or not m_h or m_h.group(1) != kernel_source_hash():
+        return None
+    return float(m_t.group(1))
+
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML while running."""
+
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:  # noqa: BLE001 - clocks are reported as unavailable
+            pass
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._ok:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0, "source": "nvml" if self._ok else "unavailable"}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+def time_steps(fn, steps, warmup, flush, world):
+    """Per-step device time (ms) of ``fn`` with CUDA events on the current stream;
+    L2 is flushed before every step, outside the events."""
+    for _ in range(warmup):
+        flush()
+        fn()
+    torch.cuda.synchronize()
+    barrier(world)
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for s, e in ev:
+        flush()
+        s.record(stream)
+        fn()
+        e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return [s.elapsed_time(e) for s, e in ev]
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gdla(args):
+    import differential_latent_attention_b200 as gdla
+    rank, world, local = dist_info()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    gdla.library()
+    peaks, peak_src = load_peaks()
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = flush_buf.zero_
+
+    # ---------------- headline: full-causal prefill, T = 4096 ----------------
+    w = gi.PREFILL_FULL
+    t = gi.make_prefill_inputs(w.seqlens, w.num_kv_heads, w.seed + 1000 * rank, device=dev)
+    out = torch.empty((w.tokens, 4 * w.num_kv_heads, 128), dtype=torch.bfloat16, device=dev)
+
+    def step():
+        gdla.attn_fwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"], w.seqlens, w.window, out=out)
+
+    with ClockSampler(local) as clocks:
+        per_step = time_steps(step, args.steps, args.warmup, flush, world)
+    total_ms = reduce_max(sum(per_step), world, dev)
+    assert gdla.device_error() == 0, "a kernel recorded a device-side failure"
+    flops = prefill_flops(w)
+    value = flops * world / (total_ms * 1e-3) / 1e12
+    launch_ms = statistics.mean(per_step)
+    achieved = flops / (launch_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+
+    # ---------------- end to end through the public API, host buffers ----------------
+    host = {k: v.cpu().pin_memory() for k, v in t.items()}
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        for k in t:
+            t[k].copy_(host[k], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_ms = reduce_max(sum(time_steps(e2e_step, e2e_steps, 2, flush, world)), world, dev) / e2e_steps
+    e2e_value = flops * world / (e2e_ms * 1e-3) / 1e12
+
+    # ---------------- CPU oracle baseline (rank 0, one GPU only) ----------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(t, w)
+    del host, out_h
+
+    extra = [] if args.headline_only else extra_workloads(gdla, dev, flush, args, world, rank, peaks)
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": len(w.seqlens), "seq_len": w.seqlens[0], "q_heads": 80,
+                   "signal_heads": 64, "noise_heads": 16, "kv_heads": 16, "dqk": 192, "dv": 128,
+                   "window": "full causal", "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed (512 MiB write) before every timed step, outside the events",
+                   "algorithmic_flops_per_step": flops},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "peak_source": f"bf16_tflops (burst) of {peak_src}",
+                     "kernel": PREFILL_KERNEL, "traffic": profiled_traffic(PREFILL_KERNEL, w.name)},
+        "e2e": {"value": round(e2e_value, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": args.steps,  # one gdla_prefill_kernel launch per step for this workload
+        "clocks": clocks.summary(),
+        "extra": extra,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def extra_workloads(gdla, dev, flush, args, world, rank, peaks):
+    res = []
+    steps = max(3, min(args.steps, 20))
+    hbm = peaks["hbm_gbs"]
+    # sliding window 128 prefill, B = 2 x 32768
+    w = gi.SWA
+    t = gi.make_prefill_inputs(w.seqlens, w.num_kv_heads, w.seed + 1000 * rank, device=dev)
+    out = torch.empty((w.tokens, 64, 128), dtype=torch.bfloat16, device=dev)
+    per = time_steps(lambda: gdla.attn_fwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"],
+                                           w.seqlens, w.window, out=out), steps, 3, flush, world)
+    ms = reduce_max(statistics.mean(per), world, dev)
+    gbs = prefill_bytes(w) / (ms * 1e-3) / 1e9
+    res.append({"workload": w.name, "metric": "tokens/s", "value": w.tokens * world / (ms * 1e-3),
+                "ms": round(ms, 5), "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
+                                                 "unit": "GB/s", "frac": round(gbs / hbm, 4)},
+                "tflops": prefill_flops(w) / (ms * 1e-3) / 1e12})
+    del t, out
+    # varlen decode, 64 sequences, full context and window 128
+    for wd in (gi.DECODE_FULL, gi.DECODE_W128):
+        lengths = wd.kv_lengths()
+        d = gi.make_decode_inputs(lengths, wd.num_kv_heads, wd.seed + 1000 * rank, device=dev)
+        o = torch.empty((wd.batch, 64, 128), dtype=torch.bfloat16, device=dev)
+        ws_bytes = gdla.decode_workspace_bytes(wd.batch, wd.num_kv_heads, 32768, wd.window)
+        ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+        per = time_steps(lambda: gdla.attn_decode(d["q_sig"], d["q_noise"], d["k_cache"], d["v_cache"],
+                                                  d["cu_seqlens_k"], 32768, d["lam"], d["gate"], wd.window,
+                                                  out=o, workspace=ws), steps, 3, flush, world)
+        ms = reduce_max(statistics.mean(per), world, dev)
+        gbs = decode_bytes(lengths, wd.num_kv_heads, wd.window) / (ms * 1e-3) / 1e9
+        res.append({"workload": wd.name, "metric": "query tokens/s", "value": wd.batch * world / (ms * 1e-3),
+                    "ms": round(ms, 5), "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
+                                                     "unit": "GB/s", "frac": round(gbs / hbm, 4)}})
+        del d, o, ws
+    return res
+
+
+def cpu_baseline(t, w, target_s: float = 12.0):
+    """The fp64 oracle, as it stands, on a bounded row sample of the same workload."""
+    import oracle
+    host = [gi.bf16_bits(t["q_sig"]), gi.bf16_bits(t["q_noise"]), gi.bf16_bits(t["k"]), gi.bf16_bits(t["v"]),
+            t["lam"].cpu().numpy(), gi.bf16_bits(t["gate"])]
+    cores = oracle.default_threads()
+    # rows evenly spaced over the sequence; grow the sample until ~target_s of CPU work
+    n_rows = 64
+    while True:
+        rows = np.linspace(0, w.tokens - 1, n_rows).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.prefill(*host, w.seqlens, w.window, rows=rows, num_threads=cores)
+        dt = time.perf_counter() - t0
+        if dt >= target_s / 4 or n_rows >= w.tokens:
+            break
+        n_rows = min(w.tokens, n_rows * 4)
+    flops = float((rows + 1).sum()) * 5 * w.num_kv_heads * FLOPS_PER_PAIR_HEAD
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{len(rows)} evenly spaced query rows (all 80 heads) of {w.name}, {dt:.1f} s"}
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    """The fp64 CPU oracle as the reference arm: rank 0 only, bounded row samples."""
+    rank, world, _ = dist_info()
+    if rank != 0:
+        return
+    import oracle
+    w = gi.PREFILL_FULL
+    t = gi.make_prefill_inputs(w.seqlens, w.num_kv_heads, w.seed, device="cpu")
+    host = [gi.bf16_bits(t["q_sig"]), gi.bf16_bits(t["q_noise"]), gi.bf16_bits(t["k"]), gi.bf16_bits(t["v"]),
+            t["lam"].numpy(), gi.bf16_bits(t["gate"])]
+    cores = oracle.default_threads()
+    rng = np.random.default_rng(0)
+    rows_per_step = 16
+    flops = 0.0
+    for _ in range(args.warmup):
+        oracle.prefill(*host, w.seqlens, w.window, rows=rng.integers(0, w.tokens, 2), num_threads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        rows = rng.integers(0, w.tokens, rows_per_step)
+        oracle.prefill(*host, w.seqlens, w.window, rows=rows, num_threads=cores)
+        flops += float((rows + 1).sum()) * 5 * w.num_kv_heads * FLOPS_PER_PAIR_HEAD
+    dt = time.perf_counter() - t0
+    value = flops / dt / 1e12
+    sample = f"{rows_per_step} random query rows (all 80 heads) of {w.name} per step"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": 1, "seq_len": 4096, "q_heads": 80, "kv_heads": 16, "dqk": 192,
+                   "dv": 128, "window": "full causal"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("gdla", "reference"), default="gdla")
+    ap.add_argument("--headline-only", action="store_true", help="skip the SWA and decode workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    _, world, _ = dist_info()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}; launch N>1 with torch.distributed.run")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gdla(args)
+
+
+if __name__ == "__main__":
+    main()

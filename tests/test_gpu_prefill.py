@@ -58,15 +58,16 @@ def test_empty_batch_is_a_no_op():
 
 
 def test_identical_paths_cancel_exactly():
-    """Signal queries equal to their noise query and lambda = 1: the signal and
-    noise rows of a tile see identical inputs, so D = 0 exactly on the GPU too."""
+    """Signal queries equal to their noise query and lambda = 1: D = 0 up to the
+    rounding of the tensor-core accumulation, which may differ by an ulp between
+    MMA rows (a wrong noise/KV group pairing would leave O(1) outputs)."""
     seqlens = (150, 40)
     t = gi.make_prefill_inputs(seqlens, 2, 12, device="cuda")
     t["q_sig"] = t["q_noise"].repeat_interleave(4, dim=1).contiguous()
     t["lam"] = torch.ones_like(t["lam"])
     out = gpu_prefill(t, seqlens, 0)
     torch.cuda.synchronize()
-    assert torch.count_nonzero(out.float()) == 0
+    assert out.float().abs().max().item() <= 1e-5
 
 
 def test_lambda_zero_gate_open_is_gqa_attention():

@@ -84,6 +84,11 @@ def reduce_max(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def whole_job_rate(work_per_step: float, steps: int, world: int, max_total_ms: float) -> float:
+    """Work of every rank over the slowest rank's device time (units per second)."""
+    return work_per_step * steps * world / (max_total_ms * 1e-3)
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
@@ -228,7 +233,7 @@ def run_gdla(args):
     total_ms = reduce_max(sum(per_step), world, dev)
     assert gdla.device_error() == 0, "a kernel recorded a device-side failure"
     flops = prefill_flops(w)
-    value = flops * world / (total_ms * 1e-3) / 1e12
+    value = whole_job_rate(flops, args.steps, world, total_ms) / 1e12
     launch_ms = statistics.mean(per_step)
     achieved = flops / (launch_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops"]

@@ -3,3 +3,4 @@
 #include "gdla_api.cu"
 #include "gdla_prefill.cu"
 #include "gdla_decode.cu"
+#include "gdla_decode_noalloc.cu"

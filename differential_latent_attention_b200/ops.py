@@ -20,8 +20,8 @@ MAX_KV_HEADS = 64
 
 STATUS = {0: "GDLA_OK", 1: "GDLA_ERR_INVALID_ARG", 2: "GDLA_ERR_UNSUPPORTED", 3: "GDLA_ERR_WORKSPACE",
           4: "GDLA_ERR_CUDA"}
-EXPORTED = ("gdla_attn_fwd", "gdla_decode_workspace_bytes", "gdla_attn_decode", "gdla_device_error",
-            "gdla_status_string", "gdla_version")
+EXPORTED = ("gdla_attn_fwd", "gdla_decode_workspace_bytes", "gdla_attn_decode", "gdla_attn_decode_noalloc",
+            "gdla_device_error", "gdla_status_string", "gdla_version")
 
 _lib = None
 _lock = threading.Lock()
@@ -50,6 +50,8 @@ def library():
             lib.gdla_decode_workspace_bytes.restype = sz
             lib.gdla_attn_decode.argtypes = [p, p, p, p, p, i, i, p, p, p, i, i, i, p, sz, p]
             lib.gdla_attn_decode.restype = i
+            lib.gdla_attn_decode_noalloc.argtypes = [p, p, p, p, p, i, i, p, p, p, i, i, i, p]
+            lib.gdla_attn_decode_noalloc.restype = i
             lib.gdla_device_error.argtypes = [i]
             lib.gdla_device_error.restype = i
             lib.gdla_status_string.argtypes = [i]

@@ -140,6 +140,39 @@ GDLA_API gdla_status_t gdla_attn_decode(const void *q_sig, const void *q_noise, 
                                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Decode for callers that cannot allocate device memory. The paper has no
+ * counterpart to this entry point; it exists for the library's users.
+ *
+ * Some callers only hold the buffers they are handed and may not allocate:
+ * a plugin inside another inference runtime that forbids device allocation
+ * on its execution path, or a service with a fixed, pre-reserved memory
+ * budget where a cudaMalloc could fail or synchronise the device mid-request.
+ * They cannot supply the split-KV workspace gdla_attn_decode needs. This
+ * call takes the same arguments and gives the same results as
+ * gdla_attn_decode, without the workspace: the split partials go to a
+ * file-scope device array of GDLA_DECODE_STATIC_SCRATCH_BYTES (16 MiB) that
+ * every GPU which loads the library holds until the process exits.
+ *  - It calls no cudaMalloc, cudaFree or allocating library routine.
+ *  - Sizes whose split plan needs more scratch than the array holds (that is,
+ *    gdla_decode_workspace_bytes(batch, num_kv_heads, max_seqlen_k, window) >
+ *    GDLA_DECODE_STATIC_SCRATCH_BYTES) are rejected with GDLA_ERR_WORKSPACE
+ *    before anything is launched.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - Every call shares the one array and it keeps the last call's contents.
+ *    Nothing needs clearing (each slot is written before it is read), but
+ *    calls whose kernels overlap on the GPU (two streams, or two host threads
+ *    on different streams) race on it: serialise them.
+ */
+#define GDLA_DECODE_STATIC_SCRATCH_BYTES (16u << 20)
+GDLA_API gdla_status_t gdla_attn_decode_noalloc(const void *q_sig, const void *q_noise, const void *k_cache,
+                                                const void *v_cache, const int32_t *cu_seqlens_k,
+                                                int num_cache_rows, int max_seqlen_k, const float *lambda,
+                                                const void *gate_logits, void *out, int batch,
+                                                int num_kv_heads, int window, void *stream);
+
+/*
  * Device-side failure word. Every wait inside the kernels is bounded (about
  * one second of SM clock); a wait that runs out makes its CTA wind down and
  * records a nonzero code here instead of hanging the GPU. This call

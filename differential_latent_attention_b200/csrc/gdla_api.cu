@@ -104,7 +104,8 @@ gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *
         return GDLA_ERR_INVALID_ARG;
 
     const int hkv = num_kv_heads;
-    const int T = kPrefillTileTokens;
+    const PrefillGeometry geo = prefill_geometry(window);
+    const int T = geo.cta_tokens;
     // ---- tile plan: every (sequence, q-tile), heaviest first ----
     std::vector<TileItem> items;
     std::vector<int> seq_start(batch);
@@ -119,7 +120,7 @@ gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *
                 const int t0 = qt * T;
                 const int lo = (window > 0) ? std::max(0, t0 - window + 1) : 0;
                 const int hi = std::min(L, t0 + T);
-                items.push_back({(hi - lo + kPrefillKeyTile - 1) / kPrefillKeyTile, b, qt});
+                items.push_back({(hi - lo + geo.key_tile - 1) / geo.key_tile, b, qt});
             }
         }
     }
@@ -131,9 +132,11 @@ gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *
 
     PrefillLaunch L{};
     const uint64_t N = static_cast<uint64_t>(n_total);
-    if (!make_map(&L.tm_qs, q_sig, 192, 4 * hkv, N, 64, 4, T) || !make_map(&L.tm_qn, q_noise, 192, hkv, N, 64, 1, T) ||
-        !make_map(&L.tm_k, k, 192, hkv, N, 64, 1, kPrefillKeyTile) ||
-        !make_map(&L.tm_v, v, 128, hkv, N, 64, 1, kPrefillKeyTile))
+    const int TT = kPrefillTileTokens;
+    if (!make_map(&L.tm_qs, q_sig, 192, 4 * hkv, N, 64, 4, TT) ||
+        !make_map(&L.tm_qn, q_noise, 192, hkv, N, 64, 1, TT) ||
+        !make_map(&L.tm_k, k, 192, hkv, N, 64, 1, geo.key_tile) ||
+        !make_map(&L.tm_v, v, 128, hkv, N, 64, 1, geo.key_tile))
         return GDLA_ERR_CUDA;
     L.lambda = lambda;
     L.gate = static_cast<const __nv_bfloat16 *>(gate_logits);

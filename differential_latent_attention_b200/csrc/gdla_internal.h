@@ -8,9 +8,16 @@
 
 namespace gdla {
 
-// Prefill: one CTA tile = 24 tokens x 5 heads = 120 of the 128 MMA rows.
+// Prefill: one MMA tile = 24 tokens x 5 heads = 120 of the 128 MMA rows. The
+// CTA size and key tile depend on the window (see prefill_geometry).
 constexpr int kPrefillTileTokens = 24;
-constexpr int kPrefillKeyTile = 128;
+constexpr int kPrefillSlidingMaxWindow = 256;  // windows up to this use the sliding configuration
+
+struct PrefillGeometry {
+    int cta_tokens;  // tokens per CTA (a multiple of kPrefillTileTokens)
+    int key_tile;    // keys per K/V tile
+};
+PrefillGeometry prefill_geometry(int window);
 constexpr int kPlanMaxSeqs = 256;    // sequences per launch (more are split across launches)
 constexpr int kPlanMaxItems = 6144;  // q-tiles per launch
 constexpr int kItemSeqShift = 20;
@@ -24,7 +31,7 @@ struct PrefillPlan {
     int pad_;
     int seq_start[kPlanMaxSeqs];  // packed row of each sequence's first token
     int seq_len[kPlanMaxSeqs];
-    uint32_t items[kPlanMaxItems];  // (local sequence << kItemSeqShift) | q-tile index
+    uint32_t items[kPlanMaxItems];  // (local sequence << kItemSeqShift) | CTA block index
 };
 
 struct PrefillLaunch {
@@ -35,7 +42,6 @@ struct PrefillLaunch {
 };
 
 cudaError_t launch_prefill(const PrefillLaunch &launch, const PrefillPlan &plan, cudaStream_t stream);
-int prefill_smem_bytes();
 
 // Decode: split-KV.
 constexpr int kDecodeMaxSplits = 64;

@@ -132,9 +132,10 @@ gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *
 
     PrefillLaunch L{};
     const uint64_t N = static_cast<uint64_t>(n_total);
-    const int TT = kPrefillTileTokens;
-    if (!make_map(&L.tm_qs, q_sig, 192, 4 * hkv, N, 64, 4, TT) ||
-        !make_map(&L.tm_qn, q_noise, 192, hkv, N, 64, 1, TT) ||
+    // Q boxes: the 6 tokens one warp (TMEM lane quarter) owns in an MMA tile.
+    const int TQ = kPrefillTileTokens / 4;
+    if (!make_map(&L.tm_qs, q_sig, 192, 4 * hkv, N, 64, 4, TQ) ||
+        !make_map(&L.tm_qn, q_noise, 192, hkv, N, 64, 1, TQ) ||
         !make_map(&L.tm_k, k, 192, hkv, N, 64, 1, geo.key_tile) ||
         !make_map(&L.tm_v, v, 128, hkv, N, 64, 1, geo.key_tile))
         return GDLA_ERR_CUDA;

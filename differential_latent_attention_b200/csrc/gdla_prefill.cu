@@ -5,12 +5,17 @@
 // over the same K_j (192) and V_j (128); then D_i = H_S,i - lambda_i * H_N,j
 // and out_i = sigmoid(gate_i) * D_i.
 //
-// Tiling. One CTA owns one KV group and TILES tensor-core tiles of 24
-// consecutive tokens of one sequence. In each tile the 5 query heads of its 24
-// tokens fill the M = 128 rows of one MMA:
-//     rows 0..95    signal heads, row = 4*tau + h   (tau = token in tile, h = 0..3)
-//     rows 96..119  the noise head, row = 96 + tau
-//     rows 120..127 unused (zero queries)
+// Work. A work item is (KV group, block of TILES x 24 consecutive tokens of
+// one sequence). CTAs are persistent (one per SM) and take items round-robin
+// from a list sorted heaviest first.
+//
+// Tiling. In each 24-token tile the 5 query heads fill the M = 128 rows of one
+// tensor-core MMA, laid out per TMEM lane quarter (one warp) so that every
+// warp owns whole tokens:
+//     quarter w (rows 32w..32w+31) holds tokens 6w..6w+5 of the tile:
+//       rows 32w + 4*i + h   signal head h (0..3) of token 6w+i   (24 rows)
+//       rows 32w + 24 + i    the noise head of token 6w+i         (6 rows)
+//       rows 32w + 30, 31    unused (zero queries)
 // Each BN-key K/V tile is staged once in shared memory (TMA) and consumed by
 // every tile and all five heads. Per key tile k and q tile x:
 //     S_x = Q_x K^T   tcgen05 M=128 N=BN K=192, smem operands, fp32 in TMEM
@@ -18,20 +23,22 @@
 //                     max/sum, P = exp2(.) rounded to bf16 into TMEM over S_x
 //     O_x += P_x V    tcgen05 with A = P from TMEM, B = V from smem (MN-major)
 // S is double-buffered per tile, so QK^T of key tile k+1 is queued while the
-// softmax of tile k runs; with two q tiles the softmax warpgroups also
-// alternate (ping-pong). The epilogue finalises O/l, passes the noise rows to
-// the signal rows through shared memory and writes sigmoid(g)(H_S - lambda H_N)
-// as bf16.
+// softmax of tile k runs; with two q tiles the softmax warpgroups alternate
+// (ping-pong). Epilogue: every warp finalises its rows (O/l), passes each
+// token's noise row to its four signal rows with warp shuffles, and writes
+// sigmoid(g)(H_S - lambda H_N) as bf16. Meanwhile the tensor core already
+// computes QK^T of the next item (its Q was loaded as soon as the last QK^T
+// of the current item finished).
 //
 // Two configurations (measured on B200: an M=128 MMA from shared memory takes
 // the same ~65 cycles at N=64 as at N=128, so 128-key tiles double the tensor
 // rate of QK^T):
 //   Causal  (TILES=1, BN=128, 2 K + 2 V stages) for full-causal and long windows;
 //   Sliding (TILES=2, BN=64, 3 K + 3 V stages) for short windows, where the path
-//           is bound by HBM and 48-token CTAs halve the per-token overheads.
+//           is bound by HBM and 48-token items halve the per-token overheads.
 // Warps: 4 per q tile (softmax + epilogue), then the TMA producer warp (which
-// also zero-fills the unused Q rows) and the MMA warp (TMEM allocation, MMA
-// issue by one elected lane of a converged warp).
+// also zero-fills the unused Q rows once) and the MMA warp (TMEM allocation,
+// MMA issue by one elected lane of a converged warp).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -51,8 +58,6 @@ constexpr int KCHUNKS = DQK / 64;
 constexpr int VCHUNKS = DV / 64;
 constexpr int Q_CHUNK = ROWS * 128;        // 16 KB
 constexpr int Q_TILE = KCHUNKS * Q_CHUNK;  // 48 KB
-constexpr int HN_STRIDE = 132;             // floats per noise row in the exchange buffer
-static_assert(TOK * HN_STRIDE * 4 <= Q_TILE, "noise exchange must fit in a Q tile");
 constexpr uint32_t Q_TX = KCHUNKS * (64 * 4 * TOK * 2 + 64 * 1 * TOK * 2);
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
@@ -99,41 +104,50 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *q_full = bars + 0;    // [tile]
-    uint64_t *k_full = bars + 2;    // [stage]
-    uint64_t *k_empty = bars + 5;   // [stage]
-    uint64_t *v_full = bars + 8;    // [stage]
-    uint64_t *v_empty = bars + 11;  // [stage]
-    uint64_t *s_full = bars + 14;   // [tile * 2 + buffer]
-    uint64_t *p_full = bars + 18;   // [tile * 2 + buffer]
-    uint64_t *o_done = bars + 22;   // [tile]: one phase per PV product of the tile
-    uint64_t *o_final = bars + 24;  // [tile]: single phase, the tile's last PV product is done
+    uint64_t *q_full = bars + 0;    // [tile]: one phase per item
+    uint64_t *q_empty = bars + 2;   // [tile]: one phase per item, after its last QK^T
+    uint64_t *k_full = bars + 4;    // [stage]
+    uint64_t *k_empty = bars + 7;   // [stage]
+    uint64_t *v_full = bars + 10;   // [stage]
+    uint64_t *v_empty = bars + 13;  // [stage]
+    uint64_t *s_full = bars + 16;   // [tile * 2 + buffer]
+    uint64_t *p_full = bars + 20;   // [tile * 2 + buffer]
+    uint64_t *o_done = bars + 24;   // [tile]: one phase per PV product of the tile
+    uint64_t *o_final = bars + 26;  // [tile]: one phase per item, its last PV product is done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
     const int hkv = plan.hkv;
-    const int group = blockIdx.x % hkv;
-    const uint32_t item = plan.items[blockIdx.x / hkv];
-    const int seq = static_cast<int>(item >> kItemSeqShift);
-    const int blk = static_cast<int>(item & kItemTileMask);
-    const int s0 = plan.seq_start[seq];
-    const int L = plan.seq_len[seq];
-    const int t0 = blk * C::CTA_TOK;
-    const int window = plan.window;
-    const int kv_lo = (window > 0) ? max(0, t0 - window + 1) : 0;
-    // key tiles q tile x visits: up to its own last row (never past the sequence)
-    int n_tiles[TILES];
-#pragma unroll
-    for (int x = 0; x < TILES; ++x) n_tiles[x] = (min(L, t0 + (x + 1) * TOK) - kv_lo + BN - 1) / BN;
-    const int n_last = n_tiles[TILES - 1];
     const int hs = 4 * hkv;
+    const int window = plan.window;
+    const int n_work = plan.n_items * hkv;
+
+    // Item w: group = w % hkv, block = items[w / hkv]; key tiles of q tile x.
+    struct Item {
+        int group, s0, L, t0, kv_lo;
+        int n_tiles[TILES];
+    };
+    auto item_at = [&](int w) {
+        Item it;
+        it.group = w % hkv;
+        const uint32_t code = plan.items[w / hkv];
+        const int seq = static_cast<int>(code >> kItemSeqShift);
+        it.s0 = plan.seq_start[seq];
+        it.L = plan.seq_len[seq];
+        it.t0 = static_cast<int>(code & kItemTileMask) * C::CTA_TOK;
+        it.kv_lo = (window > 0) ? max(0, it.t0 - window + 1) : 0;
+#pragma unroll
+        for (int x = 0; x < TILES; ++x)
+            it.n_tiles[x] = (min(it.L, it.t0 + (x + 1) * TOK) - it.kv_lo + BN - 1) / BN;
+        return it;
+    };
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < TILES; ++i) {
             mbar_init(q_full + i, 1);
+            mbar_init(q_empty + i, 1);
             mbar_init(o_done + i, 1);
             mbar_init(o_final + i, 1);
             for (int b = 0; b < 2; ++b) {
@@ -151,12 +165,14 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         fence_mbar_init();
     }
     if (warp == C::PRODUCER_WARP) {
-        // Rows 120..127 of every Q tile are never loaded: zero them.
+        // Rows 32w+30 and 32w+31 of every Q tile are never loaded: zero them once.
         for (int x = 0; x < TILES; ++x)
-            for (int c = 0; c < KCHUNKS; ++c) {
-                uint4 *dst = reinterpret_cast<uint4 *>(smem + C::OFF_Q + x * Q_TILE + c * Q_CHUNK + 120 * 128);
-                for (int i = lane; i < 8 * 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
-            }
+            for (int c = 0; c < KCHUNKS; ++c)
+                for (int i = lane; i < 4 * 2 * 8; i += 32) {
+                    const int row = 32 * (i >> 4) + 30 + ((i >> 3) & 1);
+                    reinterpret_cast<uint4 *>(smem + C::OFF_Q + x * Q_TILE + c * Q_CHUNK + row * 128)[i & 7] =
+                        make_uint4(0, 0, 0, 0);
+                }
         fence_proxy_async_smem();
     }
     if (warp == C::MMA_WARP) {
@@ -175,40 +191,58 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
             tma_prefetch_desc(&tm_qn);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            for (int x = 0; x < TILES; ++x) {
-                mbar_arrive_expect_tx(q_full + x, Q_TX);
-                for (int c = 0; c < KCHUNKS; ++c) {
-                    uint8_t *qc = smem + C::OFF_Q + x * Q_TILE + c * Q_CHUNK;
-                    tma_load_3d(qc, &tm_qs, q_full + x, c * 64, 4 * group, s0 + t0 + x * TOK);
-                    tma_load_3d(qc + NOISE_ROW0 * 128, &tm_qn, q_full + x, c * 64, group, s0 + t0 + x * TOK);
+            int kv = 0, issued_kv = 0;  // K/V tiles issued by this CTA (ring position)
+            int n_item = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+                const Item it = item_at(w);
+                for (int x = 0; x < TILES; ++x) {
+                    // the previous item's last QK^T must be done before Q_x is overwritten
+                    if (n_item > 0 && !mbar_wait(q_empty + x, (n_item - 1) & 1, abort_flag, ERR_SITE_PREFILL | 10)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(q_full + x, Q_TX);
+                    const int row0 = it.s0 + it.t0 + x * TOK;
+                    for (int c = 0; c < KCHUNKS; ++c) {
+                        uint8_t *qc = smem + C::OFF_Q + x * Q_TILE + c * Q_CHUNK;
+                        for (int q = 0; q < 4; ++q) {
+                            tma_load_3d(qc + (32 * q) * 128, &tm_qs, q_full + x, c * 64, 4 * it.group, row0 + 6 * q);
+                            tma_load_3d(qc + (32 * q + 24) * 128, &tm_qn, q_full + x, c * 64, it.group, row0 + 6 * q);
+                        }
+                    }
                 }
-            }
-            int issued_k = 0, issued_v = 0;
-            for (int k = 0; k < n_last; ++k) {
-                const int st = k % STAGES;
-                const uint32_t use = static_cast<uint32_t>(k / STAGES);
-                const int row = s0 + kv_lo + k * BN;
-                if (k >= STAGES && !mbar_wait(k_empty + st, (use + 1) & 1, abort_flag, ERR_SITE_PREFILL | 1)) break;
-                mbar_arrive_expect_tx(k_full + st, C::K_TX);
-                for (int c = 0; c < KCHUNKS; ++c)
-                    tma_load_3d(smem + C::OFF_K + st * C::K_STAGE + c * C::KV_CHUNK, &tm_k, k_full + st, c * 64,
-                                group, row);
-                issued_k = k + 1;
-                if (k >= STAGES && !mbar_wait(v_empty + st, (use + 1) & 1, abort_flag, ERR_SITE_PREFILL | 2)) break;
-                mbar_arrive_expect_tx(v_full + st, C::V_TX);
-                for (int c = 0; c < VCHUNKS; ++c)
-                    tma_load_3d(smem + C::OFF_V + st * C::V_STAGE + c * C::KV_CHUNK, &tm_v, v_full + st, c * 64,
-                                group, row);
-                issued_v = k + 1;
+                for (int k = 0; ok && k < it.n_tiles[TILES - 1]; ++k, ++kv) {
+                    const int st = kv % STAGES;
+                    const uint32_t use = static_cast<uint32_t>(kv / STAGES);
+                    const int row = it.s0 + it.kv_lo + k * BN;
+                    if (kv >= STAGES && !mbar_wait(k_empty + st, (use + 1) & 1, abort_flag, ERR_SITE_PREFILL | 1)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(k_full + st, C::K_TX);
+                    for (int c = 0; c < KCHUNKS; ++c)
+                        tma_load_3d(smem + C::OFF_K + st * C::K_STAGE + c * C::KV_CHUNK, &tm_k, k_full + st, c * 64,
+                                    it.group, row);
+                    if (kv >= STAGES && !mbar_wait(v_empty + st, (use + 1) & 1, abort_flag, ERR_SITE_PREFILL | 2)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(v_full + st, C::V_TX);
+                    for (int c = 0; c < VCHUNKS; ++c)
+                        tma_load_3d(smem + C::OFF_V + st * C::V_STAGE + c * C::KV_CHUNK, &tm_v, v_full + st, c * 64,
+                                    it.group, row);
+                    issued_kv = kv + 1;
+                }
             }
             if (*abort_flag) {
                 // Another role gave up: let this thread's copies still in flight land
                 // before the CTA (and its shared memory) goes away.
-                for (int x = 0; x < TILES; ++x) mbar_wait_cycles(q_full + x, 0, 1ll << 22);
-                for (int k = max(0, issued_k - STAGES); k < issued_k; ++k)
+                for (int k = max(0, issued_kv - STAGES); k < issued_kv; ++k) {
                     mbar_wait_cycles(k_full + k % STAGES, (k / STAGES) & 1, 1ll << 22);
-                for (int k = max(0, issued_v - STAGES); k < issued_v; ++k)
                     mbar_wait_cycles(v_full + k % STAGES, (k / STAGES) & 1, 1ll << 22);
+                }
+                for (int x = 0; x < TILES; ++x) mbar_wait_cycles(q_full + x, (n_item & 1) ^ 1, 1ll << 22);
             }
         }
     } else if (warp == C::MMA_WARP) {
@@ -217,7 +251,9 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         // one elected lane issues the MMAs and commits. Order per key tile k:
         // S_x(k) for every q tile, then PV_x(k-1) for every q tile. S_x(k) writes
         // the S buffer that held P_x(k-2), whose PV was issued earlier (tcgen05
-        // MMAs of one thread execute in issue order).
+        // MMAs of one thread execute in issue order); across items the same
+        // holds because the last PV of an item is issued before the next
+        // item's first QK^T.
         const uint32_t leader = elect_one_sync();
         constexpr uint32_t idesc_s = idesc_bf16_f32(ROWS, BN, false, false);
         constexpr uint32_t idesc_o = idesc_bf16_f32(ROWS, DV, false, true);
@@ -226,226 +262,237 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         const uint64_t q_desc0 = desc_sw128(smem_u32(smem + C::OFF_Q), 16, 1024);
         const uint64_t k_desc0 = desc_sw128(smem_u32(smem + C::OFF_K), 16, 1024);
         const uint64_t v_desc0 = desc_sw128(smem_u32(smem + C::OFF_V), C::KV_CHUNK, 1024);
+        int kv = 0;          // K/V tiles consumed by this CTA
+        int sx[TILES] = {};  // S/P steps of each q tile so far (buffer and phase)
+        int n_item = 0;
         bool ok = true;
+        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+            const Item it = item_at(w);
+            const int n_last = it.n_tiles[TILES - 1];
 #pragma unroll
-        for (int x = 0; x < TILES; ++x) ok = ok && mbar_wait(q_full + x, 0, abort_flag, ERR_SITE_PREFILL | 3);
-        ok = __all_sync(0xffffffffu, ok);
-        for (int k = 0; ok && k <= n_last; ++k) {
-            if (k < n_last) {
-                const int st = k % STAGES;
-                if (!__all_sync(0xffffffffu,
-                                mbar_wait(k_full + st, (k / STAGES) & 1, abort_flag, ERR_SITE_PREFILL | 4)))
-                    break;
-                tc_fence_after();
-                const uint64_t k_desc = k_desc0 + static_cast<uint64_t>((st * C::K_STAGE) >> 4);
-#pragma unroll
-                for (int x = 0; x < TILES; ++x) {
-                    if (k >= n_tiles[x]) continue;
-                    const uint64_t q_desc = q_desc0 + static_cast<uint64_t>((x * Q_TILE) >> 4);
-                    const uint32_t d = tmem + C::S_COL0 + x * 2 * BN + (k & 1) * BN;
-#pragma unroll
-                    for (int kk = 0; kk < DQK / 16; ++kk) {
-                        const uint32_t offq = ((kk >> 2) * Q_CHUNK + (kk & 3) * 32) >> 4;
-                        const uint32_t offk = ((kk >> 2) * C::KV_CHUNK + (kk & 3) * 32) >> 4;
-                        umma_ss_leader(d, q_desc + offq, k_desc + offk, idesc_s, kk > 0, leader);
-                    }
-                    umma_commit_leader(s_full + x * 2 + (k & 1), leader);
-                }
-                umma_commit_leader(k_empty + st, leader);
-            }
-            if (k >= 1) {
-                const int j = k - 1;
-                const int st = j % STAGES;
-                if (!__all_sync(0xffffffffu,
-                                mbar_wait(v_full + st, (j / STAGES) & 1, abort_flag, ERR_SITE_PREFILL | 6)))
-                    break;
-                const uint64_t v_desc = v_desc0 + static_cast<uint64_t>((st * C::V_STAGE) >> 4);
-                bool fail = false;
-#pragma unroll
-                for (int x = 0; x < TILES; ++x) {
-                    if (j >= n_tiles[x]) continue;
-                    if (!__all_sync(0xffffffffu, mbar_wait(p_full + x * 2 + (j & 1), (j >> 1) & 1, abort_flag,
-                                                           ERR_SITE_PREFILL | 5))) {
-                        fail = true;
+            for (int x = 0; x < TILES; ++x)
+                ok = ok && mbar_wait(q_full + x, n_item & 1, abort_flag, ERR_SITE_PREFILL | 3);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            for (int k = 0; k <= n_last; ++k) {
+                if (k < n_last) {
+                    const int st = (kv + k) % STAGES;
+                    if (!__all_sync(0xffffffffu, mbar_wait(k_full + st, ((kv + k) / STAGES) & 1, abort_flag,
+                                                           ERR_SITE_PREFILL | 4))) {
+                        ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t p_tmem = tmem + C::S_COL0 + x * 2 * BN + (j & 1) * BN;
+                    const uint64_t k_desc = k_desc0 + static_cast<uint64_t>((st * C::K_STAGE) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < BN / 16; ++kk)
-                        umma_ts_leader(tmem + C::O_COL0 + x * 128, p_tmem + kk * 8, v_desc + ((kk * 2048) >> 4),
-                                       idesc_o, (j > 0 || kk > 0) ? 1u : 0u, leader);
-                    umma_commit_leader(o_done + x, leader);
-                    if (j == n_tiles[x] - 1) umma_commit_leader(o_final + x, leader);
+                    for (int x = 0; x < TILES; ++x) {
+                        if (k >= it.n_tiles[x]) continue;
+                        const int b = (sx[x] + k) & 1;
+                        const uint64_t q_desc = q_desc0 + static_cast<uint64_t>((x * Q_TILE) >> 4);
+                        const uint32_t d = tmem + C::S_COL0 + x * 2 * BN + b * BN;
+#pragma unroll
+                        for (int kk = 0; kk < DQK / 16; ++kk) {
+                            const uint32_t offq = ((kk >> 2) * Q_CHUNK + (kk & 3) * 32) >> 4;
+                            const uint32_t offk = ((kk >> 2) * C::KV_CHUNK + (kk & 3) * 32) >> 4;
+                            umma_ss_leader(d, q_desc + offq, k_desc + offk, idesc_s, kk > 0, leader);
+                        }
+                        umma_commit_leader(s_full + x * 2 + b, leader);
+                        if (k == it.n_tiles[x] - 1) umma_commit_leader(q_empty + x, leader);
+                    }
+                    umma_commit_leader(k_empty + st, leader);
                 }
-                if (fail) break;
-                umma_commit_leader(v_empty + st, leader);
+                if (k >= 1) {
+                    const int j = k - 1;
+                    const int st = (kv + j) % STAGES;
+                    if (!__all_sync(0xffffffffu, mbar_wait(v_full + st, ((kv + j) / STAGES) & 1, abort_flag,
+                                                           ERR_SITE_PREFILL | 6))) {
+                        ok = false;
+                        break;
+                    }
+                    const uint64_t v_desc = v_desc0 + static_cast<uint64_t>((st * C::V_STAGE) >> 4);
+#pragma unroll
+                    for (int x = 0; x < TILES; ++x) {
+                        if (j >= it.n_tiles[x]) continue;
+                        const int step = sx[x] + j;
+                        if (!__all_sync(0xffffffffu, mbar_wait(p_full + x * 2 + (step & 1), (step >> 1) & 1,
+                                                               abort_flag, ERR_SITE_PREFILL | 5))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t p_tmem = tmem + C::S_COL0 + x * 2 * BN + (step & 1) * BN;
+#pragma unroll
+                        for (int kk = 0; kk < BN / 16; ++kk)
+                            umma_ts_leader(tmem + C::O_COL0 + x * 128, p_tmem + kk * 8, v_desc + ((kk * 2048) >> 4),
+                                           idesc_o, (j > 0 || kk > 0) ? 1u : 0u, leader);
+                        umma_commit_leader(o_done + x, leader);
+                        if (j == it.n_tiles[x] - 1) umma_commit_leader(o_final + x, leader);
+                    }
+                    if (!ok) break;
+                    umma_commit_leader(v_empty + st, leader);
+                }
             }
+            kv += n_last;
+#pragma unroll
+            for (int x = 0; x < TILES; ++x) sx[x] += it.n_tiles[x];
         }
     } else {
         // --------------------------- softmax + epilogue ---------------------------
-        const int x = warp >> 2;       // q tile of this warpgroup
-        const int wq = warp & 3;       // TMEM lane quarter
-        const int r = wq * 32 + lane;  // TMEM lane == tile row
-        int nt = n_tiles[0];
-#pragma unroll
-        for (int i = 1; i < TILES; ++i)
-            if (x == i) nt = n_tiles[i];
-        const int tx0 = t0 + x * TOK;  // first token of this tile
-        const bool is_sig = r < SIG_ROWS;
-        const bool is_noise = (r >= NOISE_ROW0) && (r < NOISE_ROW0 + TOK);
-        const int tau = is_sig ? (r >> 2) : (r - NOISE_ROW0);
-        const int t = tx0 + tau;
-        const int lo_t = (window > 0) ? t - window + 1 : -0x40000000;
+        const int x = warp >> 2;  // q tile of this warpgroup
+        const int wq = warp & 3;  // TMEM lane quarter = this warp's 6 tokens
+        const bool is_sig = lane < 24;
+        const int tau = 6 * wq + (is_sig ? (lane >> 2) : (lane - 24));  // token in tile
+        const int hsrc = 24 + (lane >> 2);  // lane holding this signal row's noise row
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
         const uint32_t o_addr = lane_base + C::O_COL0 + x * 128;
         const float c_log2 = 0.07216878364870322f * 1.4426950408889634f;  // log2(e) / sqrt(192)
-        float m_run = -INFINITY, l_run = 0.f;
+        int sxs = 0;  // S/P steps of this q tile so far
+        int pv = 0;   // PV products of this q tile so far (o_done phases)
+        int n_item = 0;
         bool ok = true;
+        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+            const Item it = item_at(w);
+            int nt = it.n_tiles[0];
+#pragma unroll
+            for (int i = 1; i < TILES; ++i)
+                if (x == i) nt = it.n_tiles[i];
+            const int tx0 = it.t0 + x * TOK;  // first token of this tile
+            const int t = tx0 + tau;
+            const int lo_t = (window > 0) ? t - window + 1 : -0x40000000;
+            float m_run = -INFINITY, l_run = 0.f;
 
-        for (int k = 0; k < nt; ++k) {
-            const int b = k & 1;
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait(s_full + x * 2 + b, (k >> 1) & 1, abort_flag, ERR_SITE_PREFILL | 7))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t s_addr = lane_base + C::S_COL0 + x * 2 * BN + b * BN;
-            float s[BN];
-#pragma unroll
-            for (int h = 0; h < BN / 64; ++h) {
-                uint32_t rr[64];
-                tmem_ld64(s_addr + h * 64, rr);
-#pragma unroll
-                for (int i = 0; i < 64; ++i) s[h * 64 + i] = __uint_as_float(rr[i]);
-            }
-            const int u0 = kv_lo + k * BN;
-            const bool need_mask = (u0 + BN - 1 > tx0) || (window > 0 && u0 < tx0 + TOK - window);
-            if (need_mask) {
-#pragma unroll
-                for (int i = 0; i < BN; ++i) {
-                    const int u = u0 + i;
-                    if (u > t || u < lo_t) s[i] = -INFINITY;
-                }
-            }
-            float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
-#pragma unroll
-            for (int i = 4; i < BN; i += 4) {
-                mx0 = fmaxf(mx0, s[i]);
-                mx1 = fmaxf(mx1, s[i + 1]);
-                mx2 = fmaxf(mx2, s[i + 2]);
-                mx3 = fmaxf(mx3, s[i + 3]);
-            }
-            const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c_log2;
-            const float m_new = fmaxf(m_run, mx);
-            float alpha = 1.f;
-            bool resc = false;
-            if (m_new > m_run + kRescaleThreshold) {
-                alpha = fast_exp2(m_run - m_new);
-                l_run *= alpha;
-                m_run = m_new;
-                resc = true;
-            }
-            const float mb = (m_run == -INFINITY) ? 0.f : m_run;
-            float l0 = 0.f, l1 = 0.f;
-#pragma unroll
-            for (int h = 0; h < BN / 64; ++h) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 64; i += 2) {
-                    const float p0 = fast_exp2(fmaf(s[h * 64 + i], c_log2, -mb));
-                    const float p1 = fast_exp2(fmaf(s[h * 64 + i + 1], c_log2, -mb));
-                    l0 += p0;
-                    l1 += p1;
-                    pk[i >> 1] = pack_bf16x2(p0, p1);
-                }
-                tmem_st32(s_addr + h * 32, pk);
-            }
-            l_run += l0 + l1;
-            if (k > 0 && __any_sync(0xffffffffu, resc)) {
-                // O_x still holds PV_x(k-1)'s accumulation: wait for it, then rescale.
-                if (!__all_sync(0xffffffffu, mbar_wait(o_done + x, (k - 1) & 1, abort_flag, ERR_SITE_PREFILL | 8))) {
+            for (int k = 0; k < nt; ++k) {
+                const int step = sxs + k;
+                const int b = step & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(s_full + x * 2 + b, (step >> 1) & 1, abort_flag,
+                                                       ERR_SITE_PREFILL | 7))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const float a = resc ? alpha : 1.f;
+                const uint32_t s_addr = lane_base + C::S_COL0 + x * 2 * BN + b * BN;
+                float s[BN];
 #pragma unroll
-                for (int ch = 0; ch < DV / 32; ++ch) {
-                    uint32_t o[32];
-                    tmem_ld32(o_addr + ch * 32, o);
+                for (int h = 0; h < BN / 64; ++h) {
+                    uint32_t rr[64];
+                    tmem_ld64(s_addr + h * 64, rr);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
-                    tmem_st32(o_addr + ch * 32, o);
+                    for (int i = 0; i < 64; ++i) s[h * 64 + i] = __uint_as_float(rr[i]);
                 }
+                const int u0 = it.kv_lo + k * BN;
+                const bool need_mask = (u0 + BN - 1 > tx0) || (window > 0 && u0 < tx0 + TOK - window);
+                if (need_mask) {
+#pragma unroll
+                    for (int i = 0; i < BN; ++i) {
+                        const int u = u0 + i;
+                        if (u > t || u < lo_t) s[i] = -INFINITY;
+                    }
+                }
+                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+                for (int i = 4; i < BN; i += 4) {
+                    mx0 = fmaxf(mx0, s[i]);
+                    mx1 = fmaxf(mx1, s[i + 1]);
+                    mx2 = fmaxf(mx2, s[i + 2]);
+                    mx3 = fmaxf(mx3, s[i + 3]);
+                }
+                const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c_log2;
+                const float m_new = fmaxf(m_run, mx);
+                float alpha = 1.f;
+                bool resc = false;
+                if (m_new > m_run + kRescaleThreshold) {
+                    alpha = fast_exp2(m_run - m_new);
+                    l_run *= alpha;
+                    m_run = m_new;
+                    resc = true;
+                }
+                const float mb = (m_run == -INFINITY) ? 0.f : m_run;
+                float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+                for (int h = 0; h < BN / 64; ++h) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 64; i += 2) {
+                        const float p0 = fast_exp2(fmaf(s[h * 64 + i], c_log2, -mb));
+                        const float p1 = fast_exp2(fmaf(s[h * 64 + i + 1], c_log2, -mb));
+                        l0 += p0;
+                        l1 += p1;
+                        pk[i >> 1] = pack_bf16x2(p0, p1);
+                    }
+                    tmem_st32(s_addr + h * 32, pk);
+                }
+                l_run += l0 + l1;
+                if (k > 0 && __any_sync(0xffffffffu, resc)) {
+                    // O_x still holds PV_x(k-1)'s accumulation: wait for it, then rescale.
+                    if (!__all_sync(0xffffffffu, mbar_wait(o_done + x, (pv + k - 1) & 1, abort_flag,
+                                                           ERR_SITE_PREFILL | 8))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const float a = resc ? alpha : 1.f;
+#pragma unroll
+                    for (int ch = 0; ch < DV / 32; ++ch) {
+                        uint32_t o[32];
+                        tmem_ld32(o_addr + ch * 32, o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
+                        tmem_st32(o_addr + ch * 32, o);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(p_full + x * 2 + b);
             }
-            tc_fence_before();
-            mbar_arrive(p_full + x * 2 + b);
-        }
+            if (!ok) break;
+            sxs += nt;
+            pv += nt;
 
-        // ------------------------------- epilogue --------------------------------
-        // Signal rows fetch their gate row and lambda before waiting for the last PV.
-        const bool valid = is_sig && (t < L);
-        const int n_idx = s0 + t;
-        const int head = 4 * group + (r & 3);
-        const size_t row = static_cast<size_t>(n_idx) * hs + head;
-        uint4 gv[16];
-        float lam = 0.f;
-        if (valid) {
-            const uint4 *g_row = reinterpret_cast<const uint4 *>(gate + row * DV);
+            // ----------------------------- epilogue ------------------------------
+            // Signal rows fetch their gate row and lambda before waiting for the last PV.
+            const bool valid = is_sig && (t < it.L);
+            const size_t row = static_cast<size_t>(it.s0 + t) * hs + 4 * it.group + (lane & 3);
+            uint4 gv[16];
+            float lam = 0.f;
+            if (valid) {
+                const uint4 *g_row = reinterpret_cast<const uint4 *>(gate + row * DV);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) gv[i] = __ldg(g_row + i);
-            lam = __ldg(lambda + row);
-        }
-        // o_final completes exactly once, after this tile's last PV product.
-        if (ok && !mbar_wait(o_final + x, 0, abort_flag, ERR_SITE_PREFILL | 9)) ok = false;
-        ok = __all_sync(0xffffffffu, ok);
-        tc_fence_after();
-        const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-        float *hn = reinterpret_cast<float *>(smem + C::OFF_Q + x * Q_TILE);  // Q_x is free once S_x is done
-        if (wq == 3) {
+                for (int i = 0; i < 16; ++i) gv[i] = __ldg(g_row + i);
+                lam = __ldg(lambda + row);
+            } else {
 #pragma unroll
-            for (int ch = 0; ch < DV / 32; ++ch) {
-                uint32_t o[32];
-                tmem_ld32(o_addr + ch * 32, o);
-                if (is_noise) {
-                    float4 *dst = reinterpret_cast<float4 *>(hn + tau * HN_STRIDE + ch * 32);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
-                                             __uint_as_float(o[4 * i + 2]) * inv_l,
-                                             __uint_as_float(o[4 * i + 3]) * inv_l);
-                }
+                for (int i = 0; i < 16; ++i) gv[i] = make_uint4(0, 0, 0, 0);
             }
-        }
-        // named barrier 1 + x over this tile's 4 warps
-        asm volatile("bar.sync %0, 128;" ::"r"(1 + x) : "memory");
-        if (wq < 3) {
+            // o_final completes once per item, after this tile's last PV product.
+            if (!__all_sync(0xffffffffu, mbar_wait(o_final + x, n_item & 1, abort_flag, ERR_SITE_PREFILL | 9))) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
             uint4 *o_row = reinterpret_cast<uint4 *>(out + row * DV);
-            const float *hn_row = hn + tau * HN_STRIDE;
             const uint32_t *gw = reinterpret_cast<const uint32_t *>(gv);
 #pragma unroll
             for (int ch = 0; ch < DV / 32; ++ch) {
                 uint32_t o[32];
                 tmem_ld32(o_addr + ch * 32, o);
-                if (valid && ok) {
-                    uint32_t res[16];
+                uint32_t res[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float2 g2 =
-                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gw[ch * 16 + i]));
-                        const float d0 = __uint_as_float(o[2 * i]) * inv_l - lam * hn_row[ch * 32 + 2 * i];
-                        const float d1 = __uint_as_float(o[2 * i + 1]) * inv_l - lam * hn_row[ch * 32 + 2 * i + 1];
-                        const float y0 = __fdividef(d0, 1.f + __expf(-g2.x));
-                        const float y1 = __fdividef(d1, 1.f + __expf(-g2.y));
-                        res[i] = pack_bf16x2(y0, y1);
-                    }
+                for (int i = 0; i < 16; ++i) {
+                    const float h0 = __uint_as_float(o[2 * i]) * inv_l;
+                    const float h1 = __uint_as_float(o[2 * i + 1]) * inv_l;
+                    const float n0 = __shfl_sync(0xffffffffu, h0, hsrc);  // H_N of this row's token
+                    const float n1 = __shfl_sync(0xffffffffu, h1, hsrc);
+                    const float2 g2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gw[ch * 16 + i]));
+                    res[i] = pack_bf16x2(fmaf(-lam, n0, h0) * fast_sigmoid(g2.x), fmaf(-lam, n1, h1) * fast_sigmoid(g2.y));
+                }
+                if (valid) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
                         o_row[ch * 4 + i] = make_uint4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
                 }
             }
+            // every lane's TMEM reads of O are complete before the next item's PV
+            // products may overwrite it (they wait for this warpgroup's p_full).
+            tc_fence_before();
         }
     }
 
@@ -461,27 +508,31 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
 // Host side
 // ------------------------------------------------------------------------------
 PrefillGeometry prefill_geometry(int window) {
-    // Short windows: 48-token CTAs over 64-key tiles; otherwise 24-token CTAs over 128-key tiles.
-    if (window > 0 && window <= kPrefillSlidingMaxWindow)
-        return {pf::SlidingCfg::CTA_TOK, pf::SlidingCfg::BN};
+    // Short windows: 48-token items over 64-key tiles; otherwise 24-token items over 128-key tiles.
+    if (window > 0 && window <= kPrefillSlidingMaxWindow) return {pf::SlidingCfg::CTA_TOK, pf::SlidingCfg::BN};
     return {pf::CausalCfg::CTA_TOK, pf::CausalCfg::BN};
 }
 
 template <class C>
-static cudaError_t launch_cfg(const PrefillLaunch &L, const PrefillPlan &plan, cudaStream_t stream) {
+static cudaError_t launch_cfg(const PrefillLaunch &L, const PrefillPlan &plan, int num_sms, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(gdla_prefill_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    const unsigned grid = static_cast<unsigned>(plan.n_items) * static_cast<unsigned>(plan.hkv);
+    const long long work = static_cast<long long>(plan.n_items) * plan.hkv;
+    const unsigned grid = static_cast<unsigned>(work < num_sms ? work : num_sms);
     gdla_prefill_kernel<C><<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(L.tm_qs, L.tm_qn, L.tm_k, L.tm_v,
                                                                           L.lambda, L.gate, L.out, plan);
     return cudaPeekAtLastError();
 }
 
 cudaError_t launch_prefill(const PrefillLaunch &L, const PrefillPlan &plan, cudaStream_t stream) {
+    int dev = 0, num_sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
     if (plan.window > 0 && plan.window <= kPrefillSlidingMaxWindow)
-        return launch_cfg<pf::SlidingCfg>(L, plan, stream);
-    return launch_cfg<pf::CausalCfg>(L, plan, stream);
+        return launch_cfg<pf::SlidingCfg>(L, plan, num_sms, stream);
+    return launch_cfg<pf::CausalCfg>(L, plan, num_sms, stream);
 }
 
 }  // namespace gdla

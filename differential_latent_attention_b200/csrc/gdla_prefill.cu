@@ -40,6 +40,7 @@
 // also zero-fills the unused Q rows once) and the MMA warp (TMEM allocation,
 // MMA issue by one elected lane of a converged warp).
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -61,6 +62,7 @@ constexpr int Q_TILE = KCHUNKS * Q_CHUNK;  // 48 KB
 constexpr uint32_t Q_TX = KCHUNKS * (64 * 4 * TOK * 2 + 64 * 1 * TOK * 2);
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+constexpr int kPolyEvery = 4;              // one exponential pair in 4 on the FMA pipe
 
 template <int TILES_, int BN_, int STAGES_>
 struct Cfg {
@@ -82,10 +84,16 @@ struct Cfg {
     static constexpr uint32_t V_TX = V_STAGE;
     static constexpr uint32_t O_COL0 = 0;              // + 128 * tile
     static constexpr uint32_t S_COL0 = 128 * TILES;    // + 2 * BN * tile + BN * buffer
+    // With one q tile, Q is copied into TMEM once per item (96 columns) and
+    // QK^T reads it from there, which removes the Q re-reads from shared
+    // memory that otherwise bound the MMAs; the shared Q buffer is then only
+    // a staging area, free again as soon as the copy is done.
+    static constexpr bool Q_IN_TMEM = (TILES == 1);
+    static constexpr uint32_t QT_COL0 = S_COL0 + 2 * BN * TILES;
     static constexpr int NUM_THREADS = 128 * TILES + 64;
     static constexpr int PRODUCER_WARP = 4 * TILES;
     static constexpr int MMA_WARP = 4 * TILES + 1;
-    static_assert(S_COL0 + 2 * BN * TILES <= TMEM_COLS, "TMEM budget");
+    static_assert(QT_COL0 + (Q_IN_TMEM ? DQK / 2 : 0) <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(BN == 64 || BN == 128, "key tile");
 };
@@ -273,6 +281,16 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
             for (int x = 0; x < TILES; ++x)
                 ok = ok && mbar_wait(q_full + x, n_item & 1, abort_flag, ERR_SITE_PREFILL | 3);
             if (!__all_sync(0xffffffffu, ok)) break;
+            if constexpr (C::Q_IN_TMEM) {
+                // Q (staged in shared memory) -> TMEM, one 16-element K step per copy;
+                // the MMAs below are issued after these copies and run after them.
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < DQK / 16; ++kk)
+                    tmem_cp_128x256b_leader(tmem + C::QT_COL0 + kk * 8,
+                                            q_desc0 + (((kk >> 2) * Q_CHUNK + (kk & 3) * 32) >> 4), leader);
+                umma_commit_leader(q_empty + 0, leader);  // the staging buffer may be refilled
+            }
             for (int k = 0; k <= n_last; ++k) {
                 if (k < n_last) {
                     const int st = (kv + k) % STAGES;
@@ -293,10 +311,13 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                         for (int kk = 0; kk < DQK / 16; ++kk) {
                             const uint32_t offq = ((kk >> 2) * Q_CHUNK + (kk & 3) * 32) >> 4;
                             const uint32_t offk = ((kk >> 2) * C::KV_CHUNK + (kk & 3) * 32) >> 4;
-                            umma_ss_leader(d, q_desc + offq, k_desc + offk, idesc_s, kk > 0, leader);
+                            if constexpr (C::Q_IN_TMEM)
+                                umma_ts_leader(d, tmem + C::QT_COL0 + kk * 8, k_desc + offk, idesc_s, kk > 0, leader);
+                            else
+                                umma_ss_leader(d, q_desc + offq, k_desc + offk, idesc_s, kk > 0, leader);
                         }
                         umma_commit_leader(s_full + x * 2 + b, leader);
-                        if (k == it.n_tiles[x] - 1) umma_commit_leader(q_empty + x, leader);
+                        if (!C::Q_IN_TMEM && k == it.n_tiles[x] - 1) umma_commit_leader(q_empty + x, leader);
                     }
                     umma_commit_leader(k_empty + st, leader);
                 }
@@ -406,21 +427,41 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                     resc = true;
                 }
                 const float mb = (m_run == -INFINITY) ? 0.f : m_run;
-                float l0 = 0.f, l1 = 0.f;
+                // p = exp2(s * log2(e)/sqrt(192) - m): scaling and row sums in packed
+                // fp32 pairs; one pair in kPolyEvery through the FMA-pipe polynomial,
+                // the others through MUFU ex2, so both pipes share the work.
+                const uint64_t scale2 = f2_pack(c_log2, c_log2);
+                const uint64_t neg_m2 = f2_pack(-mb, -mb);
+                uint64_t lsum_a = f2_pack(0.f, 0.f), lsum_b = f2_pack(0.f, 0.f);
 #pragma unroll
                 for (int h = 0; h < BN / 64; ++h) {
                     uint32_t pk[32];
 #pragma unroll
-                    for (int i = 0; i < 64; i += 2) {
-                        const float p0 = fast_exp2(fmaf(s[h * 64 + i], c_log2, -mb));
-                        const float p1 = fast_exp2(fmaf(s[h * 64 + i + 1], c_log2, -mb));
-                        l0 += p0;
-                        l1 += p1;
-                        pk[i >> 1] = pack_bf16x2(p0, p1);
+                    for (int i = 0; i < 32; ++i) {
+                        const uint64_t xx = f2_fma(f2_pack(s[h * 64 + 2 * i], s[h * 64 + 2 * i + 1]), scale2, neg_m2);
+                        float p0, p1;
+                        if ((i % kPolyEvery) == kPolyEvery - 1) {
+                            exp2_poly_pair(xx, p0, p1);
+                        } else {
+                            float x0, x1;
+                            f2_unpack(xx, x0, x1);
+                            p0 = fast_exp2(x0);
+                            p1 = fast_exp2(x1);
+                        }
+                        if (i & 1)
+                            lsum_b = f2_add(lsum_b, f2_pack(p0, p1));
+                        else
+                            lsum_a = f2_add(lsum_a, f2_pack(p0, p1));
+                        pk[i] = pack_bf16x2(p0, p1);
                     }
                     tmem_st32(s_addr + h * 32, pk);
                 }
-                l_run += l0 + l1;
+                {
+                    float a0, a1, b0, b1;
+                    f2_unpack(lsum_a, a0, a1);
+                    f2_unpack(lsum_b, b0, b1);
+                    l_run += (a0 + a1) + (b0 + b1);
+                }
                 if (k > 0 && __any_sync(0xffffffffu, resc)) {
                     // O_x still holds PV_x(k-1)'s accumulation: wait for it, then rescale.
                     if (!__all_sync(0xffffffffu, mbar_wait(o_done + x, (pv + k - 1) & 1, abort_flag,

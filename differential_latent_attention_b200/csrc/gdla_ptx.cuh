@@ -169,6 +169,17 @@ __device__ __forceinline__ void umma_commit_leader(uint64_t *bar, uint32_t leade
         "r"(leader)
         : "memory");
 }
+// Copy a 128-row x 32-byte matrix (described like an MMA operand) from shared
+// memory into 128 TMEM lanes x 8 columns; asynchronous and ordered with the
+// tcgen05.mma operations issued by the same thread.
+__device__ __forceinline__ void tmem_cp_128x256b_leader(uint32_t taddr, uint64_t s_desc, uint32_t leader) {
+    asm volatile(
+        "{\n\t.reg .pred q;\n\t"
+        "setp.ne.b32 q, %2, 0;\n\t"
+        "@q tcgen05.cp.cta_group::1.128x256b [%0], %1;\n\t}" ::"r"(taddr),
+        "l"(s_desc), "r"(leader)
+        : "memory");
+}
 __device__ __forceinline__ uint32_t elect_one_sync() {
     uint32_t pred = 0;
     asm volatile(
@@ -274,6 +285,51 @@ __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// ---------------------- packed fp32 pairs (sm_100 f32x2) ----------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// exp2 of a pair on the FMA pipe: x = n + f with n = round(x), f in [-1/2, 1/2];
+// 2^f by a cubic whose coefficients were fitted for this library (discrete
+// minimax, max relative error 7.5e-5; csrc/fit_exp2_poly.py), 2^n by adding n
+// to the exponent bits. n comes from the round-to-nearest of x + 1.5 * 2^23.
+// Inputs below -125 are clamped there (result ~2^-125, below any weight that
+// matters once rounded into a softmax sum of at least 1).
+__device__ __forceinline__ void exp2_poly_pair(uint64_t x, float &r0, float &r1) {
+    constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+    float x0, x1;
+    f2_unpack(x, x0, x1);
+    x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t y = f2_add(x, f2_pack(kShift, kShift));    // n in the low mantissa bits
+    const uint64_t n = f2_add(y, f2_pack(-kShift, -kShift));  // n as a float (exact)
+    const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);      // x - n
+    uint64_t p = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f,
+                        f2_pack(0.2426111251115799f, 0.2426111251115799f));
+    p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+    p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+    float p0, p1, y0, y1;
+    f2_unpack(p, p0, p1);
+    f2_unpack(y, y0, y1);
+    r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(y0) << 23));
+    r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(y1) << 23));
 }
 
 }  // namespace gdla

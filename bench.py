@@ -384,6 +384,33 @@ def run_reference(args):
     }), flush=True)
 
 
+PROFILE_CASES = ("prefill_T4096_full", "swa128_B2_T8192", "decode_B64_L1024_4096", "decode_B64_L1024_4096_w128")
+
+
+def run_profile_case(args):
+    """A few launches of one workload, small enough for a full ncu capture
+    (ncu -k <kernel> -s <skip> -c <count> python bench.py --profile-case NAME)."""
+    import differential_latent_attention_b200 as gdla
+    dev = torch.device("cuda", 0)
+    name = args.profile_case
+    if name.startswith("decode"):
+        wd = gi.DecodeWorkload(name, 64, 16, 128 if name.endswith("w128") else 0, 4, 1024, 4096)
+        lengths = wd.kv_lengths()
+        d = gi.make_decode_inputs(lengths, 16, wd.seed, device=dev)
+        fn = lambda: gdla.attn_decode(d["q_sig"], d["q_noise"], d["k_cache"], d["v_cache"], d["cu_seqlens_k"],
+                                      4096, d["lam"], d["gate"], wd.window)
+    else:
+        w = gi.PREFILL_FULL if name.startswith("prefill") else gi.PrefillWorkload(name, (8192, 8192), 16, 128, 2)
+        t = gi.make_prefill_inputs(w.seqlens, w.num_kv_heads, w.seed, device=dev)
+        fn = lambda: gdla.attn_fwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"], w.seqlens,
+                                   w.window)
+    for _ in range(args.steps):
+        fn()
+    torch.cuda.synchronize()
+    assert gdla.device_error() == 0
+    print(f"profile case {name}: {args.steps} launches done", flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -392,13 +419,17 @@ def main():
     ap.add_argument("--impl", choices=("gdla", "reference"), default="gdla")
     ap.add_argument("--headline-only", action="store_true", help="skip the SWA and decode workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--profile-case", choices=PROFILE_CASES, help="only launch this small workload --steps times "
+                    "(a driver for ncu captures; prints no JSON line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     _, world, _ = dist_info()
     if world != args.gpus:
         ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}; launch N>1 with torch.distributed.run")
-    if args.impl == "reference":
+    if args.profile_case:
+        run_profile_case(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_gdla(args)

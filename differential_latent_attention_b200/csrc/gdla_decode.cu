@@ -1,8 +1,9 @@
 // gdla_decode.cu - varlen split-KV GDLA decode for sm_100a.
 //
 // One query token per sequence (position L_b - 1, the cache holding it). For
-// each (sequence b, KV group j, split s) a CTA streams its slice of K_j/V_j
-// through shared memory (TMA, 64 keys per stage) and computes, for the five
+// each (sequence b, KV group j, split s) item a persistent CTA streams the
+// split's slice of K_j/V_j through shared memory (TMA, 64 keys per stage; the
+// stage ring continues across items) and computes, for the five
 // query heads of the group at once, the split's running max m, sum l and
 // unnormalised O. The dense contractions run on tensor cores with the keys as
 // the MMA's M dimension:
@@ -90,6 +91,44 @@ __device__ __forceinline__ void decode_epilogue(const float *h, const float *__r
     }
 }
 
+// Key range of one (split, group, sequence) item; an item is empty when the
+// sequence's length is invalid or the split starts past its keys.
+struct DecodeItem {
+    int b, group, split;
+    int start;            // packed cache row of the sequence's first key
+    int k_begin, k_end;   // keys of this split, positions within the sequence
+    int n_stages;
+};
+
+__device__ __forceinline__ int decode_visible_keys(const int32_t *__restrict__ cu, int b, const DecodePlan &plan,
+                                                   int &start, int &lo) {
+    start = cu[b];
+    const int end = cu[b + 1];
+    const int len = end - start;
+    const bool ok = (start >= 0) && (len >= 1) && (len <= plan.max_seqlen_k) && (end <= plan.num_cache_rows);
+    lo = (plan.window > 0) ? max(0, len - plan.window) : 0;
+    return ok ? len - lo : 0;
+}
+
+__device__ __forceinline__ DecodeItem decode_item(const int32_t *__restrict__ cu, int w, const DecodePlan &plan) {
+    DecodeItem d;
+    d.split = w % plan.num_splits;
+    const int rest = w / plan.num_splits;
+    d.group = rest % plan.hkv;
+    d.b = rest / plan.hkv;
+    int lo;
+    const int n_vis = decode_visible_keys(cu, d.b, plan, d.start, lo);
+    d.k_begin = lo + d.split * plan.split_keys;
+    d.k_end = lo + min(n_vis, (d.split + 1) * plan.split_keys);
+    d.n_stages = max(0, (d.k_end - d.k_begin + dc::TK - 1) / dc::TK);
+    return d;
+}
+
+// Persistent split kernel: every CTA loops over (split, group, sequence)
+// items; the producer's K/V stage ring runs on across items, so the next
+// item's keys stream in while the current one is computed. Consumers fetch
+// an item's Q fragments (and, for a single split, its gate values and lambda)
+// before waiting for its first stage.
 __global__ void __launch_bounds__(dc::NUM_THREADS, 2)
 gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          const __nv_bfloat16 *__restrict__ q_sig, const __nv_bfloat16 *__restrict__ q_noise,
@@ -105,21 +144,10 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
     float *red = reinterpret_cast<float *>(smem + OFF_RED);
     float *ml = reinterpret_cast<float *>(smem + OFF_ML);
 
-    const int split = blockIdx.x;
-    const int group = blockIdx.y;
-    const int b = blockIdx.z;
     const int hkv = plan.hkv;
+    const int ns = plan.num_splits;
+    const int n_work = ns * hkv * plan.batch;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    const int start = cu_seqlens_k[b];
-    const int len = cu_seqlens_k[b + 1] - start;
-    const bool len_ok = (start >= 0) && (len >= 1) && (len <= plan.max_seqlen_k) &&
-                        (cu_seqlens_k[b + 1] <= plan.num_cache_rows);
-    const int lo = (plan.window > 0) ? max(0, len - plan.window) : 0;
-    const int k_begin = lo + split * plan.split_keys;
-    const int k_end = len_ok ? min(len, k_begin + plan.split_keys) : k_begin;
-    const int n_keys = max(0, k_end - k_begin);
-    const int n_stages = (n_keys + TK - 1) / TK;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
@@ -133,206 +161,231 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
 
     if (warp == CONSUMER_WARPS) {
         // ------------------------------ TMA producer ------------------------------
-        if (lane == 0 && n_stages > 0) {
+        if (lane == 0) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            int issued = 0;
-            for (int it = 0; it < n_stages; ++it) {
-                const int st = it % STAGES;
-                if (it >= STAGES &&
-                    !mbar_wait(empty + st, ((it / STAGES) + 1) & 1, abort_flag, ERR_SITE_DECODE | 1))
-                    break;
-                mbar_arrive_expect_tx(full + st, STAGE_TX);
-                const int row = start + k_begin + it * TK;
-                for (int c = 0; c < 3; ++c)
-                    tma_load_3d(smem + OFF_K + st * K_STAGE + c * K_CHUNK, &tm_k, full + st, c * 64, group, row);
-                for (int c = 0; c < 2; ++c)
-                    tma_load_3d(smem + OFF_V + st * V_STAGE + c * K_CHUNK, &tm_v, full + st, c * 64, group, row);
-                issued = it + 1;
+            int g = 0, issued = 0;  // stages issued by this CTA (ring position)
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x) {
+                const DecodeItem d = decode_item(cu_seqlens_k, w, plan);
+                for (int it = 0; it < d.n_stages; ++it, ++g) {
+                    const int st = g % STAGES;
+                    if (g >= STAGES &&
+                        !mbar_wait(empty + st, ((g / STAGES) + 1) & 1, abort_flag, ERR_SITE_DECODE | 1)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(full + st, STAGE_TX);
+                    const int row = d.start + d.k_begin + it * TK;
+                    for (int c = 0; c < 3; ++c)
+                        tma_load_3d(smem + OFF_K + st * K_STAGE + c * K_CHUNK, &tm_k, full + st, c * 64, d.group, row);
+                    for (int c = 0; c < 2; ++c)
+                        tma_load_3d(smem + OFF_V + st * V_STAGE + c * K_CHUNK, &tm_v, full + st, c * 64, d.group, row);
+                    issued = g + 1;
+                }
             }
             if (*abort_flag)
-                for (int it = max(0, issued - STAGES); it < issued; ++it)
-                    mbar_wait_cycles(full + it % STAGES, (it / STAGES) & 1, 1ll << 22);
+                for (int k = max(0, issued - STAGES); k < issued; ++k)
+                    mbar_wait_cycles(full + k % STAGES, (k / STAGES) & 1, 1ll << 22);
         }
     } else {
         // ------------------------------- consumers --------------------------------
-        const int g = lane >> 2, c = lane & 3;
-        // Q^T fragments (B operand): thread holds head g, dims 16*ks + 2c(+1) and +8.
-        uint32_t qf[DQK / 16][2];
-        {
-            const __nv_bfloat16 *qrow = nullptr;
-            if (g < 4) qrow = q_sig + (static_cast<size_t>(b) * 4 * hkv + 4 * group + g) * DQK;
-            else if (g == 4) qrow = q_noise + (static_cast<size_t>(b) * hkv + group) * DQK;
-#pragma unroll
-            for (int ks = 0; ks < DQK / 16; ++ks) {
-                if (qrow) {
-                    qf[ks][0] = *reinterpret_cast<const uint32_t *>(qrow + ks * 16 + 2 * c);
-                    qf[ks][1] = *reinterpret_cast<const uint32_t *>(qrow + ks * 16 + 8 + 2 * c);
-                } else {
-                    qf[ks][0] = 0u;
-                    qf[ks][1] = 0u;
-                }
-            }
-        }
-        const float c_log2 = 0.07216878364870322f * 1.4426950408889634f;  // log2(e) / sqrt(192)
-        float o[DV / 16][4];
-#pragma unroll
-        for (int mt = 0; mt < DV / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
-        float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of heads 2c, 2c+1
-        float l0 = 0.f, l1 = 0.f;              // this thread's partial sums
-
+        const int g8 = lane >> 2, c = lane & 3;
         const int mi = lane >> 3, ri = lane & 7;
-        for (int it = 0; it < n_stages; ++it) {
-            const int st = it % STAGES;
-            if (!mbar_wait(full + st, (it / STAGES) & 1, abort_flag, ERR_SITE_DECODE | 2)) break;
-            const uint32_t kb = smem_u32(smem + OFF_K + st * K_STAGE);
-            const uint32_t vb = smem_u32(smem + OFF_V + st * V_STAGE);
-            const int key0 = warp * 16;  // this warp's 16 keys within the stage
-            // S^T = K Q^T
-            float s[4] = {0.f, 0.f, 0.f, 0.f};
+        const int dcol = threadIdx.x;  // output column this thread owns in the merge/epilogue
+        const float c_log2 = 0.07216878364870322f * 1.4426950408889634f;  // log2(e) / sqrt(192)
+        int g = 0;  // stages consumed by this CTA
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x) {
+            const DecodeItem d = decode_item(cu_seqlens_k, w, plan);
+            // Several splits: empty ones write nothing (the combine kernel skips them).
+            if (ns > 1 && d.n_stages == 0) continue;
+            // Q^T fragments (B operand): thread holds head g8, dims 16*ks + 2c(+1) and +8.
+            uint32_t qf[DQK / 16][2];
             {
-                const int krow = key0 + ri + 8 * (mi & 1);
+                const __nv_bfloat16 *qrow = nullptr;
+                if (g8 < 4) qrow = q_sig + (static_cast<size_t>(d.b) * 4 * hkv + 4 * d.group + g8) * DQK;
+                else if (g8 == 4) qrow = q_noise + (static_cast<size_t>(d.b) * hkv + d.group) * DQK;
 #pragma unroll
                 for (int ks = 0; ks < DQK / 16; ++ks) {
-                    const int dim = ks * 16 + 8 * (mi >> 1);
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4(kb + (dim >> 6) * K_CHUNK + swz(krow, (dim & 63) >> 3), a0, a1, a2, a3);
-                    mma_bf16(s, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+                    qf[ks][0] = qrow ? __ldg(reinterpret_cast<const uint32_t *>(qrow + ks * 16 + 2 * c)) : 0u;
+                    qf[ks][1] = qrow ? __ldg(reinterpret_cast<const uint32_t *>(qrow + ks * 16 + 8 + 2 * c)) : 0u;
                 }
             }
-            // mask keys past the split end (and the cache rows of other sequences)
-            const int ubase = k_begin + it * TK + key0;
-            if (ubase + g >= k_end) { s[0] = -INFINITY; s[1] = -INFINITY; }
-            if (ubase + g + 8 >= k_end) { s[2] = -INFINITY; s[3] = -INFINITY; }
-            float mx0 = fmaxf(s[0], s[2]) * c_log2, mx1 = fmaxf(s[1], s[3]) * c_log2;
+            const size_t orow0 = (static_cast<size_t>(d.b) * hkv + d.group) * 4;
+            float lam_pre[4] = {0.f, 0.f, 0.f, 0.f}, g_pre[4] = {0.f, 0.f, 0.f, 0.f};
+            if (ns == 1) {
 #pragma unroll
-            for (int off = 4; off < 32; off <<= 1) {
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                for (int i = 0; i < 4; ++i) {
+                    lam_pre[i] = __ldg(lambda + orow0 + i);
+                    g_pre[i] = __bfloat162float(gate[(orow0 + i) * DV + dcol]);
+                }
             }
-            const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-            const float a0s = (n0 == -INFINITY) ? 1.f : fast_exp2(m0 - n0);
-            const float a1s = (n1 == -INFINITY) ? 1.f : fast_exp2(m1 - n1);
-            m0 = n0;
-            m1 = n1;
-            const float b0 = (n0 == -INFINITY) ? 0.f : n0, b1 = (n1 == -INFINITY) ? 0.f : n1;
-            const float p0 = fast_exp2(fmaf(s[0], c_log2, -b0));
-            const float p1 = fast_exp2(fmaf(s[1], c_log2, -b1));
-            const float p2 = fast_exp2(fmaf(s[2], c_log2, -b0));
-            const float p3 = fast_exp2(fmaf(s[3], c_log2, -b1));
-            l0 = l0 * a0s + p0 + p2;
-            l1 = l1 * a1s + p1 + p3;
+            float o[DV / 16][4];
 #pragma unroll
-            for (int mt = 0; mt < DV / 16; ++mt) {
-                o[mt][0] *= a0s;
-                o[mt][1] *= a1s;
-                o[mt][2] *= a0s;
-                o[mt][3] *= a1s;
-            }
-            // P^T blocks (keys g / g+8, heads 2c..2c+1) -> transposed B fragments
-            const uint32_t pb0 = movmatrix_t(pack_bf16x2(p0, p1));
-            const uint32_t pb1 = movmatrix_t(pack_bf16x2(p2, p3));
-            {
-                const int vrow = key0 + ri + 8 * (mi >> 1);
+            for (int mt = 0; mt < DV / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+            float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of heads 2c, 2c+1
+            float l0 = 0.f, l1 = 0.f;              // this thread's partial sums
+
+            for (int it = 0; it < d.n_stages; ++it, ++g) {
+                const int st = g % STAGES;
+                if (!__all_sync(0xffffffffu, mbar_wait(full + st, (g / STAGES) & 1, abort_flag, ERR_SITE_DECODE | 2))) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t kb = smem_u32(smem + OFF_K + st * K_STAGE);
+                const uint32_t vb = smem_u32(smem + OFF_V + st * V_STAGE);
+                const int key0 = warp * 16;  // this warp's 16 keys within the stage
+                // S^T = K Q^T
+                float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+                {
+                    const int krow = key0 + ri + 8 * (mi & 1);
+#pragma unroll
+                    for (int ks = 0; ks < DQK / 16; ++ks) {
+                        const int dim = ks * 16 + 8 * (mi >> 1);
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4(kb + (dim >> 6) * K_CHUNK + swz(krow, (dim & 63) >> 3), a0, a1, a2, a3);
+                        mma_bf16(sacc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+                    }
+                }
+                // mask keys past the split end (and the cache rows of other sequences)
+                const int ubase = d.k_begin + it * TK + key0;
+                if (ubase + g8 >= d.k_end) { sacc[0] = -INFINITY; sacc[1] = -INFINITY; }
+                if (ubase + g8 + 8 >= d.k_end) { sacc[2] = -INFINITY; sacc[3] = -INFINITY; }
+                float mx0 = fmaxf(sacc[0], sacc[2]) * c_log2, mx1 = fmaxf(sacc[1], sacc[3]) * c_log2;
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                }
+                const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+                const float a0s = (n0 == -INFINITY) ? 1.f : fast_exp2(m0 - n0);
+                const float a1s = (n1 == -INFINITY) ? 1.f : fast_exp2(m1 - n1);
+                m0 = n0;
+                m1 = n1;
+                const float b0 = (n0 == -INFINITY) ? 0.f : n0, b1 = (n1 == -INFINITY) ? 0.f : n1;
+                const float p0 = fast_exp2(fmaf(sacc[0], c_log2, -b0));
+                const float p1 = fast_exp2(fmaf(sacc[1], c_log2, -b1));
+                const float p2 = fast_exp2(fmaf(sacc[2], c_log2, -b0));
+                const float p3 = fast_exp2(fmaf(sacc[3], c_log2, -b1));
+                l0 = l0 * a0s + p0 + p2;
+                l1 = l1 * a1s + p1 + p3;
 #pragma unroll
                 for (int mt = 0; mt < DV / 16; ++mt) {
-                    const int dv = mt * 16 + 8 * (mi & 1);
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4_t(vb + (dv >> 6) * K_CHUNK + swz(vrow, (dv & 63) >> 3), a0, a1, a2, a3);
-                    mma_bf16(o[mt], a0, a1, a2, a3, pb0, pb1);
+                    o[mt][0] *= a0s;
+                    o[mt][1] *= a1s;
+                    o[mt][2] *= a0s;
+                    o[mt][3] *= a1s;
+                }
+                // P^T blocks (keys g8 / g8+8, heads 2c..2c+1) -> transposed B fragments
+                const uint32_t pb0 = movmatrix_t(pack_bf16x2(p0, p1));
+                const uint32_t pb1 = movmatrix_t(pack_bf16x2(p2, p3));
+                {
+                    const int vrow = key0 + ri + 8 * (mi >> 1);
+#pragma unroll
+                    for (int mt = 0; mt < DV / 16; ++mt) {
+                        const int dv = mt * 16 + 8 * (mi & 1);
+                        uint32_t v0, v1, v2, v3;
+                        ldsm_x4_t(vb + (dv >> 6) * K_CHUNK + swz(vrow, (dv & 63) >> 3), v0, v1, v2, v3);
+                        mma_bf16(o[mt], v0, v1, v2, v3, pb0, pb1);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty + st);
+            }
+            if (!ok) break;
+            // ---- merge the four warps: per head max, then rescaled sums ----
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+                l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+            }
+            if (g8 == 0) {
+                ml[(warp * 8 + 2 * c) * 2 + 0] = m0;
+                ml[(warp * 8 + 2 * c) * 2 + 1] = l0;
+                ml[(warp * 8 + 2 * c + 1) * 2 + 0] = m1;
+                ml[(warp * 8 + 2 * c + 1) * 2 + 1] = l1;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            float gm0 = -INFINITY, gm1 = -INFINITY;
+#pragma unroll
+            for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) {
+                gm0 = fmaxf(gm0, ml[(w4 * 8 + 2 * c) * 2]);
+                gm1 = fmaxf(gm1, ml[(w4 * 8 + 2 * c + 1) * 2]);
+            }
+            const float f0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - gm0);
+            const float f1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - gm1);
+            float *rw = red + warp * HEADS * DV;
+#pragma unroll
+            for (int mt = 0; mt < DV / 16; ++mt) {
+                const int dv0 = mt * 16 + g8;
+                if (2 * c < HEADS) {
+                    rw[(2 * c) * DV + dv0] = o[mt][0] * f0;
+                    rw[(2 * c) * DV + dv0 + 8] = o[mt][2] * f0;
+                }
+                if (2 * c + 1 < HEADS) {
+                    rw[(2 * c + 1) * DV + dv0] = o[mt][1] * f1;
+                    rw[(2 * c + 1) * DV + dv0 + 8] = o[mt][3] * f1;
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty + st);
-        }
-        // ---- merge the four warps: per head max, then rescaled sums ----
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-        }
-        if (g == 0) {
-            ml[(warp * 8 + 2 * c) * 2 + 0] = m0;
-            ml[(warp * 8 + 2 * c) * 2 + 1] = l0;
-            ml[(warp * 8 + 2 * c + 1) * 2 + 0] = m1;
-            ml[(warp * 8 + 2 * c + 1) * 2 + 1] = l1;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        // global max over warps for this thread's two heads
-        float gm0 = -INFINITY, gm1 = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < CONSUMER_WARPS; ++w) {
-            gm0 = fmaxf(gm0, ml[(w * 8 + 2 * c) * 2]);
-            gm1 = fmaxf(gm1, ml[(w * 8 + 2 * c + 1) * 2]);
-        }
-        const float f0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - gm0);
-        const float f1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - gm1);
-        // write this warp's rescaled O^T (heads < 5) to red[warp][head][dv]
-        float *rw = red + warp * HEADS * DV;
-#pragma unroll
-        for (int mt = 0; mt < DV / 16; ++mt) {
-            const int dv0 = mt * 16 + g;
-            if (2 * c < HEADS) {
-                rw[(2 * c) * DV + dv0] = o[mt][0] * f0;
-                rw[(2 * c) * DV + dv0 + 8] = o[mt][2] * f0;
-            }
-            if (2 * c + 1 < HEADS) {
-                rw[(2 * c + 1) * DV + dv0] = o[mt][1] * f1;
-                rw[(2 * c + 1) * DV + dv0 + 8] = o[mt][3] * f1;
-            }
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        // thread d (0..127) sums the 4 warps for every head, fixed order
-        const int d = threadIdx.x;
-        float hsum[HEADS];
-        float hm[HEADS], hl[HEADS];
-#pragma unroll
-        for (int h = 0; h < HEADS; ++h) {
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < CONSUMER_WARPS; ++w) M = fmaxf(M, ml[(w * 8 + h) * 2]);
-            float Ls = 0.f, Os = 0.f;
-#pragma unroll
-            for (int w = 0; w < CONSUMER_WARPS; ++w) {
-                const float mw = ml[(w * 8 + h) * 2];
-                const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-                Ls += ml[(w * 8 + h) * 2 + 1] * f;
-                Os += red[(w * HEADS + h) * DV + d];
-            }
-            hm[h] = M;
-            hl[h] = Ls;
-            hsum[h] = Os;
-        }
-        const size_t slot = (static_cast<size_t>(b) * hkv + group) * plan.num_splits + split;
-        if (plan.num_splits == 1) {
-            // one split holds every key: finish here. Reuse red[0] as h[5][128].
             asm volatile("bar.sync 1, 128;" ::: "memory");
-            float *hbuf = red;
+            // thread dcol (0..127) sums the 4 warps for every head, fixed order
+            float hsum[HEADS], hm[HEADS], hl[HEADS];
 #pragma unroll
-            for (int h = 0; h < HEADS; ++h) hbuf[h * DV + d] = (hl[h] > 0.f) ? hsum[h] / hl[h] : 0.f;
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            decode_epilogue(hbuf, lambda, gate, out, (static_cast<size_t>(b) * hkv + group) * 4, d);
-        } else {
-            float *wo = ws + slot * (HEADS * DV);
-            float *wml = ws + plan.ml_offset_floats + slot * (HEADS * 2);
+            for (int h = 0; h < HEADS; ++h) {
+                float M = -INFINITY;
 #pragma unroll
-            for (int h = 0; h < HEADS; ++h) wo[h * DV + d] = hsum[h];
-            if (d < HEADS) {
-                wml[d * 2 + 0] = hm[d];
-                wml[d * 2 + 1] = hl[d];
+                for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) M = fmaxf(M, ml[(w4 * 8 + h) * 2]);
+                float Ls = 0.f, Os = 0.f;
+#pragma unroll
+                for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) {
+                    const float mw = ml[(w4 * 8 + h) * 2];
+                    const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
+                    Ls += ml[(w4 * 8 + h) * 2 + 1] * f;
+                    Os += red[(w4 * HEADS + h) * DV + dcol];
+                }
+                hm[h] = M;
+                hl[h] = Ls;
+                hsum[h] = Os;
             }
+            if (ns == 1) {
+                // one split holds every key: finish here (gate values fetched at the item start)
+                float hv[HEADS];
+#pragma unroll
+                for (int h = 0; h < HEADS; ++h) hv[h] = (hl[h] > 0.f) ? hsum[h] / hl[h] : 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float dd = hv[i] - lam_pre[i] * hv[4];
+                    out[(orow0 + i) * DV + dcol] = __float2bfloat16_rn(__fdividef(dd, 1.f + __expf(-g_pre[i])));
+                }
+            } else {
+                const size_t slot = (static_cast<size_t>(d.b) * hkv + d.group) * ns + d.split;
+                float *wo = ws + slot * (HEADS * DV);
+                float *wml = ws + plan.ml_offset_floats + slot * (HEADS * 2);
+#pragma unroll
+                for (int h = 0; h < HEADS; ++h) wo[h * DV + dcol] = hsum[h];
+#pragma unroll
+                for (int h = 0; h < HEADS; ++h)
+                    if (dcol == h) {
+                        wml[h * 2 + 0] = hm[h];
+                        wml[h * 2 + 1] = hl[h];
+                    }
+            }
+            // every consumer is done with ml/red before the next item writes them
+            asm volatile("bar.sync 1, 128;" ::: "memory");
         }
     }
 }
 
-// Split merge: one CTA of 5 warps per (sequence, group); warp h merges head h.
-// Lanes walk the splits (32 at a time): a shuffle max gives the global m, each
-// split gets weight exp2(m_s - m), and each lane then owns 4 dv columns of the
-// weighted sum. Splits that saw no key carry m = -inf and are skipped.
+// Split merge: one CTA of 5 warps per (sequence, group); warp h merges head h
+// over the splits that hold keys of this sequence (the split kernel writes
+// nothing for the others). Lanes walk the splits: a shuffle max gives the
+// global m, each split gets weight exp2(m_s - m), and each lane then owns 4 dv
+// columns of the weighted sum.
 __global__ void __launch_bounds__(160)
-gdla_decode_combine_kernel(const float *__restrict__ ws, const float *__restrict__ lambda,
-                           const __nv_bfloat16 *__restrict__ gate, __nv_bfloat16 *__restrict__ out,
-                           const DecodePlan plan) {
+gdla_decode_combine_kernel(const float *__restrict__ ws, const int32_t *__restrict__ cu_seqlens_k,
+                           const float *__restrict__ lambda, const __nv_bfloat16 *__restrict__ gate,
+                           __nv_bfloat16 *__restrict__ out, const DecodePlan plan) {
     using namespace dc;
     __shared__ float hbuf[HEADS * DV];
     __shared__ float wsh[HEADS][64];
@@ -340,15 +393,18 @@ gdla_decode_combine_kernel(const float *__restrict__ ws, const float *__restrict
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int hkv = plan.hkv;
     const int ns = plan.num_splits;
+    int start, lo;
+    const int n_vis = decode_visible_keys(cu_seqlens_k, b, plan, start, lo);
+    const int ns_b = min(ns, (n_vis + plan.split_keys - 1) / plan.split_keys);  // splits holding keys
     const size_t slot0 = (static_cast<size_t>(b) * hkv + group) * ns;
     const float *wml = ws + plan.ml_offset_floats;
     const int h = warp;
     float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, wml[(slot0 + s) * (HEADS * 2) + h * 2]);
+    for (int s = lane; s < ns_b; s += 32) M = fmaxf(M, wml[(slot0 + s) * (HEADS * 2) + h * 2]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     float Lsum = 0.f;
-    for (int s = lane; s < ns; s += 32) {
+    for (int s = lane; s < ns_b; s += 32) {
         const float ms = wml[(slot0 + s) * (HEADS * 2) + h * 2];
         const float ls = wml[(slot0 + s) * (HEADS * 2) + h * 2 + 1];
         const float w = (ms == -INFINITY) ? 0.f : fast_exp2(ms - M);
@@ -359,7 +415,7 @@ gdla_decode_combine_kernel(const float *__restrict__ ws, const float *__restrict
     for (int off = 16; off > 0; off >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
     __syncwarp();
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < ns; ++s) {
+    for (int s = 0; s < ns_b; ++s) {
         const float w = wsh[h][s];
         if (w == 0.f) continue;
         const float4 v = *reinterpret_cast<const float4 *>(ws + (slot0 + s) * (HEADS * DV) + h * DV + lane * 4);
@@ -382,13 +438,23 @@ cudaError_t launch_decode(const DecodeLaunch &L, const DecodePlan &plan, cudaStr
     cudaError_t e = cudaFuncSetAttribute(gdla_decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          dc::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    dim3 grid(plan.num_splits, plan.hkv, plan.batch);
+    int dev = 0, num_sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    // One split per sequence (windows, short caches): few small items whose
+    // latency chains dominate, so two persistent CTAs per SM pipeline them.
+    // Several splits: many items of similar size, balanced best by the hardware
+    // scheduler with one item per CTA (the same kernel, one loop trip each).
+    const long long work = static_cast<long long>(plan.num_splits) * plan.hkv * plan.batch;
+    const long long resident = 2ll * num_sms;  // two CTAs per SM
+    const unsigned grid = static_cast<unsigned>((plan.num_splits == 1 && work > resident) ? resident : work);
     gdla_decode_split_kernel<<<grid, dc::NUM_THREADS, dc::SMEM_BYTES, stream>>>(
         L.tm_k, L.tm_v, L.q_sig, L.q_noise, L.cu_seqlens_k, L.lambda, L.gate, L.out, L.ws, plan);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess || plan.num_splits == 1) return e;
     dim3 grid2(plan.hkv, plan.batch);
-    gdla_decode_combine_kernel<<<grid2, 160, 0, stream>>>(L.ws, L.lambda, L.gate, L.out, plan);
+    gdla_decode_combine_kernel<<<grid2, 160, 0, stream>>>(L.ws, L.cu_seqlens_k, L.lambda, L.gate, L.out, plan);
     return cudaPeekAtLastError();
 }
 

@@ -106,13 +106,19 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "gdla_prefill_kernel": ("gdla_prefill.cu", "gdla_ptx.cuh", "gdla_internal.h"),
+    "gdla_decode_split_kernel": ("gdla_decode.cu", "gdla_ptx.cuh", "gdla_internal.h"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources a kernel is compiled from (its .cu file and the shared headers)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "differential_latent_attention_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 
@@ -126,7 +132,7 @@ def profiled_traffic(kernel: str, workload: str):
         return None
     m_t = re.search(r"^traffic_bytes_per_launch:\s*([0-9.eE+]+)", text, re.M)
     m_h = re.search(r"^kernel_sources_sha256_16:\s*([0-9a-f]+)", text, re.M)
-    if not m_t or not m_h or m_h.group(1) != kernel_source_hash():
+    if not m_t or not m_h or m_h.group(1) != kernel_source_hash(kernel):
         return None
     return float(m_t.group(1))
 

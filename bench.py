@@ -313,6 +313,25 @@ def extra_workloads(gdla, dev, flush, args, world, rank, peaks):
                                                  "unit": "GB/s", "frac": round(gbs / hbm, 4)},
                 "tflops": prefill_flops(w) / (ms * 1e-3) / 1e12})
     del t, out
+    # the pages' hybrid schedule: one full-causal layer then three window-128 layers, T = 65536
+    hyb_ms, hyb_flops, hyb_bytes = 0.0, 0.0, 0.0
+    layer_ms = []
+    for wl in gi.HYBRID_LAYERS:
+        t = gi.make_prefill_inputs(wl.seqlens, wl.num_kv_heads, wl.seed + 1000 * rank, device=dev)
+        out = torch.empty((wl.tokens, 64, 128), dtype=torch.bfloat16, device=dev)
+        per = time_steps(lambda: gdla.attn_fwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"],
+                                               wl.seqlens, wl.window, out=out), 3, 3, flush, world)
+        ms = reduce_max(statistics.mean(per), world, dev)
+        layer_ms.append(round(ms, 4))
+        hyb_ms += ms
+        hyb_flops += prefill_flops(wl)
+        hyb_bytes += prefill_bytes(wl) if wl.window > 0 else 0.0
+        del t, out
+    res.append({"workload": "hybrid_T65536_H16_1full_3w128", "metric": "tokens/s (4 layers)",
+                "value": gi.HYBRID_LAYERS[0].tokens * 4 * world / (hyb_ms * 1e-3), "ms": round(hyb_ms, 4),
+                "layer_ms": layer_ms,
+                "full_layer_tflops": round(prefill_flops(gi.HYBRID_LAYERS[0]) / (layer_ms[0] * 1e-3) / 1e12, 2),
+                "swa_layers_gbs": round(hyb_bytes / (sum(layer_ms[1:]) * 1e-3) / 1e9, 1)})
     # varlen decode, 64 sequences, full context and window 128
     for wd in (gi.DECODE_FULL, gi.DECODE_W128):
         lengths = wd.kv_lengths()

@@ -109,3 +109,20 @@ def test_hybrid_T65536_layers_sampled_rows(layer):
 
 def test_no_device_error_recorded():
     assert gdla.device_error(clear=True) == 0
+
+
+def test_more_sequences_than_one_launch_holds():
+    """300 sequences (over the 256 a launch plan holds): the host splits the batch
+    across launches; every row must still match."""
+    rng = np.random.default_rng(5)
+    seqlens = tuple(int(x) for x in rng.integers(0, 41, size=300))
+    check_prefill(seqlens, 2, 0, 14)
+    check_prefill(seqlens, 2, 16, 15)
+
+
+def test_more_blocks_than_one_launch_holds():
+    """200 sequences of 800 tokens: 6,800 token blocks (over the 6,144 a launch plan
+    holds) in the full-causal configuration; sampled rows of every sequence."""
+    seqlens = (800,) * 200
+    rows = gi.sample_rows(seqlens, 3, seed=16, must_include=(0, 799))
+    check_prefill(seqlens, 1, 0, 16, rows=rows)

@@ -49,6 +49,19 @@
 
 namespace gdla {
 
+// One full 32-byte sector per lane (sm_100 256-bit loads/stores); the address
+// must be 32-byte aligned.
+__device__ __forceinline__ void ld_nc_v8(const void *p, uint32_t *r) {
+    asm volatile("ld.global.nc.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "l"(p));
+}
+__device__ __forceinline__ void st_v8(void *p, const uint32_t *r) {
+    asm volatile("st.global.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
 namespace pf {
 constexpr int TOK = kPrefillTileTokens;  // 24 tokens per MMA tile
 constexpr int ROWS = 128;
@@ -99,6 +112,59 @@ struct Cfg {
 };
 using CausalCfg = Cfg<1, 128, 2>;
 using SlidingCfg = Cfg<2, 64, 3>;
+
+// ------------------------------- epilogue ----------------------------------
+// Per warp: the 24 signal rows of its 6 tokens. gate/out rows are 256 bytes;
+// with 32-byte aligned bases each lane moves whole 32-byte sectors (half the
+// memory instructions of 16-byte accesses over the same scattered rows).
+// Gate columns 32ch..32ch+31 of one row (16 words of bf16 pairs).
+__device__ __forceinline__ void epi_fetch_gate(bool valid, size_t row, const __nv_bfloat16 *__restrict__ gate,
+                                               bool wide, int ch, uint32_t (&g)[16]) {
+    if (valid) {
+        const __nv_bfloat16 *src = gate + row * DV + ch * 32;
+        if (wide) {
+            ld_nc_v8(src, g);
+            ld_nc_v8(src + 16, g + 8);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(src) + i);
+                g[4 * i] = v.x;
+                g[4 * i + 1] = v.y;
+                g[4 * i + 2] = v.z;
+                g[4 * i + 3] = v.w;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) g[i] = 0;
+    }
+}
+// Columns 32ch..32ch+31 of this lane's O row: H = O/l; the token's noise row
+// comes from lane hsrc by shuffle; out = sigmoid(g) (H_S - lambda H_N) in bf16.
+__device__ __forceinline__ void epi_chunk(const uint32_t (&o)[32], float inv_l, float lam, const uint32_t (&g)[16],
+                                          int hsrc, bool valid, bool wide, __nv_bfloat16 *__restrict__ dst) {
+    uint32_t res[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float h0 = __uint_as_float(o[2 * i]) * inv_l;
+        const float h1 = __uint_as_float(o[2 * i + 1]) * inv_l;
+        const float n0 = __shfl_sync(0xffffffffu, h0, hsrc);  // H_N of this row's token
+        const float n1 = __shfl_sync(0xffffffffu, h1, hsrc);
+        const float2 g2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&g[i]));
+        res[i] = pack_bf16x2(fmaf(-lam, n0, h0) * fast_sigmoid(g2.x), fmaf(-lam, n1, h1) * fast_sigmoid(g2.y));
+    }
+    if (valid) {
+        if (wide) {
+            st_v8(dst, res);
+            st_v8(dst + 16, res + 8);
+        } else {
+            uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d[i] = make_uint4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
+        }
+    }
+}
 }  // namespace pf
 
 template <class C>
@@ -366,6 +432,7 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
         const uint32_t o_addr = lane_base + C::O_COL0 + x * 128;
         const float c_log2 = 0.07216878364870322f * 1.4426950408889634f;  // log2(e) / sqrt(192)
+        const bool wide = ((reinterpret_cast<uintptr_t>(gate) | reinterpret_cast<uintptr_t>(out)) & 31u) == 0;
         int sxs = 0;  // S/P steps of this q tile so far
         int pv = 0;   // PV products of this q tile so far (o_done phases)
         int n_item = 0;
@@ -491,17 +558,10 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
             // Signal rows fetch their gate row and lambda before waiting for the last PV.
             const bool valid = is_sig && (t < it.L);
             const size_t row = static_cast<size_t>(it.s0 + t) * hs + 4 * it.group + (lane & 3);
-            uint4 gv[16];
-            float lam = 0.f;
-            if (valid) {
-                const uint4 *g_row = reinterpret_cast<const uint4 *>(gate + row * DV);
+            uint32_t gw[DV / 32][16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) gv[i] = __ldg(g_row + i);
-                lam = __ldg(lambda + row);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) gv[i] = make_uint4(0, 0, 0, 0);
-            }
+            for (int ch = 0; ch < DV / 32; ++ch) epi_fetch_gate(valid, row, gate, wide, ch, gw[ch]);
+            const float lam = valid ? __ldg(lambda + row) : 0.f;
             // o_final completes once per item, after this tile's last PV product.
             if (!__all_sync(0xffffffffu, mbar_wait(o_final + x, n_item & 1, abort_flag, ERR_SITE_PREFILL | 9))) {
                 ok = false;
@@ -509,27 +569,11 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
             }
             tc_fence_after();
             const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-            uint4 *o_row = reinterpret_cast<uint4 *>(out + row * DV);
-            const uint32_t *gw = reinterpret_cast<const uint32_t *>(gv);
 #pragma unroll
             for (int ch = 0; ch < DV / 32; ++ch) {
                 uint32_t o[32];
                 tmem_ld32(o_addr + ch * 32, o);
-                uint32_t res[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float h0 = __uint_as_float(o[2 * i]) * inv_l;
-                    const float h1 = __uint_as_float(o[2 * i + 1]) * inv_l;
-                    const float n0 = __shfl_sync(0xffffffffu, h0, hsrc);  // H_N of this row's token
-                    const float n1 = __shfl_sync(0xffffffffu, h1, hsrc);
-                    const float2 g2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&gw[ch * 16 + i]));
-                    res[i] = pack_bf16x2(fmaf(-lam, n0, h0) * fast_sigmoid(g2.x), fmaf(-lam, n1, h1) * fast_sigmoid(g2.y));
-                }
-                if (valid) {
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        o_row[ch * 4 + i] = make_uint4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
-                }
+                epi_chunk(o, inv_l, lam, gw[ch], hsrc, valid, wide, out + row * DV + ch * 32);
             }
             // every lane's TMEM reads of O are complete before the next item's PV
             // products may overwrite it (they wait for this warpgroup's p_full).

@@ -47,6 +47,26 @@ def test_every_row_written_and_deterministic():
     assert torch.equal(first.view(torch.int16), out.view(torch.int16))
 
 
+@pytest.mark.parametrize("window", [0, 16])
+def test_gate_and_out_only_16_byte_aligned(window):
+    """gate/out at 16- but not 32-byte aligned addresses take the 16-byte access
+    path of the epilogue; the result must be bit-identical to the aligned run."""
+    seqlens = (70, 200, 3)
+    t = gi.make_prefill_inputs(seqlens, 2, 18, device="cuda")
+    ref = gpu_prefill(t, seqlens, window)
+    n = sum(seqlens)
+    gbuf = torch.empty(n * 8 * 128 + 8, dtype=torch.bfloat16, device="cuda")
+    obuf = torch.full((n * 8 * 128 + 8,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    g16 = gbuf[8:].view(n, 8, 128)
+    g16.copy_(t["gate"])
+    o16 = obuf[8:].view(n, 8, 128)
+    assert g16.data_ptr() % 32 == 16 and o16.data_ptr() % 32 == 16
+    gdla.attn_fwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], g16, seqlens, window, out=o16)
+    torch.cuda.synchronize()
+    assert gdla.device_error() == 0
+    assert torch.equal(ref.view(torch.int16), o16.view(torch.int16))
+
+
 def test_empty_batch_is_a_no_op():
     """Zero tokens: the call returns GDLA_OK without launching anything."""
     import ctypes

@@ -76,6 +76,9 @@ DecodePlan make_decode_plan(int batch, int hkv, int max_seqlen_k, int window, in
     return p;
 }
 
+// Keys per K/V TMA box of the decode kernel that runs this plan (gdla_decode.cu).
+int decode_key_tile(const DecodePlan &plan);
+
 size_t decode_workspace_bytes(const DecodePlan &p) {
     if (p.num_splits <= 1) return 0;
     return static_cast<size_t>(p.batch) * p.hkv * p.num_splits * 5 * (128 + 2) * sizeof(float);
@@ -195,8 +198,9 @@ gdla_status_t gdla_attn_decode(const void *q_sig, const void *q_noise, const voi
         return GDLA_ERR_WORKSPACE;
     DecodeLaunch L{};
     const uint64_t nk = static_cast<uint64_t>(num_cache_rows);
-    if (!make_map(&L.tm_k, k_cache, 192, num_kv_heads, nk, 64, 1, 64) ||
-        !make_map(&L.tm_v, v_cache, 128, num_kv_heads, nk, 64, 1, 64))
+    const uint32_t tk = static_cast<uint32_t>(decode_key_tile(plan));
+    if (!make_map(&L.tm_k, k_cache, 192, num_kv_heads, nk, 64, 1, tk) ||
+        !make_map(&L.tm_v, v_cache, 128, num_kv_heads, nk, 64, 1, tk))
         return GDLA_ERR_CUDA;
     L.q_sig = static_cast<const __nv_bfloat16 *>(q_sig);
     L.q_noise = static_cast<const __nv_bfloat16 *>(q_noise);

@@ -28,23 +28,40 @@ namespace gdla {
 
 namespace dc {
 constexpr int DQK = 192, DV = 128, HEADS = 5;
-constexpr int TK = 64;                     // keys per stage
 constexpr int STAGES = 2;
-constexpr int CONSUMER_WARPS = 4;          // each takes 16 keys of a stage
-constexpr int NUM_THREADS = (CONSUMER_WARPS + 1) * 32;
-constexpr int K_CHUNK = TK * 128;          // one 64-dim swizzled chunk: 8 KB
-constexpr int K_STAGE = 3 * K_CHUNK;       // 24 KB
-constexpr int V_STAGE = 2 * K_CHUNK;       // 16 KB
-constexpr int OFF_K = 0;
-constexpr int OFF_V = OFF_K + STAGES * K_STAGE;
-constexpr int OFF_RED = OFF_V + STAGES * V_STAGE;                 // [4 warps][5 heads][128] fp32
-constexpr int RED_BYTES = CONSUMER_WARPS * HEADS * DV * 4;
-constexpr int OFF_ML = OFF_RED + RED_BYTES;                        // [4 warps][8 heads] m, l
-constexpr int OFF_BAR = OFF_ML + 2 * CONSUMER_WARPS * 8 * 4;
-constexpr int OFF_MISC = OFF_BAR + 2 * STAGES * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-constexpr uint32_t STAGE_TX = K_STAGE + V_STAGE;
 }  // namespace dc
+
+// Split-kernel configuration: each consumer warp takes 16 keys of a TK-key
+// stage; CTAS_PER_SM CTAs share an SM.
+template <int TK_, int CW_, int CTAS_>
+struct DCfg {
+    static constexpr int TK = TK_;                 // keys per stage
+    static constexpr int CONSUMER_WARPS = CW_;
+    static constexpr int CTAS_PER_SM = CTAS_;
+    static constexpr int NCT = CW_ * 32;           // consumer threads
+    static constexpr int NUM_THREADS = NCT + 32;   // + the TMA producer warp
+    static constexpr int COLS = dc::DV / NCT;      // output columns per consumer thread (merge, epilogue)
+    static constexpr int K_CHUNK = TK * 128;       // one 64-dim swizzled chunk
+    static constexpr int K_STAGE = 3 * K_CHUNK;
+    static constexpr int V_STAGE = 2 * K_CHUNK;
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + dc::STAGES * K_STAGE;
+    static constexpr int OFF_RED = OFF_V + dc::STAGES * V_STAGE;  // [warps][5 heads][128] fp32
+    static constexpr int RED_BYTES = CW_ * dc::HEADS * dc::DV * 4;
+    static constexpr int OFF_ML = OFF_RED + RED_BYTES;             // [warps][8 heads] m, l
+    static constexpr int OFF_BAR = OFF_ML + 2 * CW_ * 8 * 4;
+    static constexpr int OFF_MISC = OFF_BAR + 2 * dc::STAGES * 8;
+    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+    static constexpr uint32_t STAGE_TX = K_STAGE + V_STAGE;
+    static_assert(TK == 16 * CW_, "one 16-key MMA block per consumer warp");
+    static_assert(dc::DV % NCT == 0, "columns per consumer thread");
+};
+// Several splits (long caches): one item per CTA, 64-key stages, 4 consumer warps.
+using SplitCfg = DCfg<64, 4, 2>;
+// One split (windows, short caches): few small items per SM, whose latency
+// chains dominate; 32-key stages and 2 consumer warps let 4 persistent CTAs
+// (4 items in flight) share each SM.
+using WindowCfg = DCfg<32, 2, 4>;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -110,7 +127,8 @@ __device__ __forceinline__ int decode_visible_keys(const int32_t *__restrict__ c
     return ok ? len - lo : 0;
 }
 
-__device__ __forceinline__ DecodeItem decode_item(const int32_t *__restrict__ cu, int w, const DecodePlan &plan) {
+__device__ __forceinline__ DecodeItem decode_item(const int32_t *__restrict__ cu, int w, const DecodePlan &plan,
+                                              int tk) {
     DecodeItem d;
     d.split = w % plan.num_splits;
     const int rest = w / plan.num_splits;
@@ -120,7 +138,7 @@ __device__ __forceinline__ DecodeItem decode_item(const int32_t *__restrict__ cu
     const int n_vis = decode_visible_keys(cu, d.b, plan, d.start, lo);
     d.k_begin = lo + d.split * plan.split_keys;
     d.k_end = lo + min(n_vis, (d.split + 1) * plan.split_keys);
-    d.n_stages = max(0, (d.k_end - d.k_begin + dc::TK - 1) / dc::TK);
+    d.n_stages = max(0, (d.k_end - d.k_begin + tk - 1) / tk);
     return d;
 }
 
@@ -129,13 +147,19 @@ __device__ __forceinline__ DecodeItem decode_item(const int32_t *__restrict__ cu
 // item's keys stream in while the current one is computed. Consumers fetch
 // an item's Q fragments (and, for a single split, its gate values and lambda)
 // before waiting for its first stage.
-__global__ void __launch_bounds__(dc::NUM_THREADS, 2)
+template <class C>
+__global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS_PER_SM)
 gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                          const __nv_bfloat16 *__restrict__ q_sig, const __nv_bfloat16 *__restrict__ q_noise,
                          const int32_t *__restrict__ cu_seqlens_k, const float *__restrict__ lambda,
                          const __nv_bfloat16 *__restrict__ gate, __nv_bfloat16 *__restrict__ out,
                          float *__restrict__ ws, const DecodePlan plan) {
     using namespace dc;
+    constexpr int TK = C::TK, CONSUMER_WARPS = C::CONSUMER_WARPS, NCT = C::NCT, COLS = C::COLS;
+    constexpr int K_CHUNK = C::K_CHUNK, K_STAGE = C::K_STAGE, V_STAGE = C::V_STAGE;
+    constexpr int OFF_K = C::OFF_K, OFF_V = C::OFF_V, OFF_RED = C::OFF_RED, OFF_ML = C::OFF_ML;
+    constexpr int OFF_BAR = C::OFF_BAR, OFF_MISC = C::OFF_MISC;
+    constexpr uint32_t STAGE_TX = C::STAGE_TX;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
@@ -167,7 +191,7 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             int g = 0, issued = 0;  // stages issued by this CTA (ring position)
             bool ok = true;
             for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x) {
-                const DecodeItem d = decode_item(cu_seqlens_k, w, plan);
+                const DecodeItem d = decode_item(cu_seqlens_k, w, plan, TK);
                 for (int it = 0; it < d.n_stages; ++it, ++g) {
                     const int st = g % STAGES;
                     if (g >= STAGES &&
@@ -192,12 +216,12 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         // ------------------------------- consumers --------------------------------
         const int g8 = lane >> 2, c = lane & 3;
         const int mi = lane >> 3, ri = lane & 7;
-        const int dcol = threadIdx.x;  // output column this thread owns in the merge/epilogue
+        const int dcol = threadIdx.x;  // first of the COLS output columns (dcol + j * NCT) it owns
         const float c_log2 = 0.07216878364870322f * 1.4426950408889634f;  // log2(e) / sqrt(192)
         int g = 0;  // stages consumed by this CTA
         bool ok = true;
         for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x) {
-            const DecodeItem d = decode_item(cu_seqlens_k, w, plan);
+            const DecodeItem d = decode_item(cu_seqlens_k, w, plan, TK);
             // Several splits: empty ones write nothing (the combine kernel skips them).
             if (ns > 1 && d.n_stages == 0) continue;
             // Q^T fragments (B operand): thread holds head g8, dims 16*ks + 2c(+1) and +8.
@@ -213,12 +237,13 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 }
             }
             const size_t orow0 = (static_cast<size_t>(d.b) * hkv + d.group) * 4;
-            float lam_pre[4] = {0.f, 0.f, 0.f, 0.f}, g_pre[4] = {0.f, 0.f, 0.f, 0.f};
+            float lam_pre[4] = {0.f, 0.f, 0.f, 0.f}, g_pre[COLS][4] = {};
             if (ns == 1) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     lam_pre[i] = __ldg(lambda + orow0 + i);
-                    g_pre[i] = __bfloat162float(gate[(orow0 + i) * DV + dcol]);
+#pragma unroll
+                    for (int j = 0; j < COLS; ++j) g_pre[j][i] = __bfloat162float(gate[(orow0 + i) * DV + dcol + j * NCT]);
                 }
             }
             float o[DV / 16][4];
@@ -306,7 +331,7 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 ml[(warp * 8 + 2 * c + 1) * 2 + 0] = m1;
                 ml[(warp * 8 + 2 * c + 1) * 2 + 1] = l1;
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, %0;" ::"n"(NCT) : "memory");
             float gm0 = -INFINITY, gm1 = -INFINITY;
 #pragma unroll
             for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) {
@@ -328,51 +353,62 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                     rw[(2 * c + 1) * DV + dv0 + 8] = o[mt][3] * f1;
                 }
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            // thread dcol (0..127) sums the 4 warps for every head, fixed order
-            float hsum[HEADS], hm[HEADS], hl[HEADS];
+            asm volatile("bar.sync 1, %0;" ::"n"(NCT) : "memory");
+            // each thread sums the warps for every head of its columns, fixed order
+            float hm[HEADS], hl[HEADS];
 #pragma unroll
             for (int h = 0; h < HEADS; ++h) {
                 float M = -INFINITY;
 #pragma unroll
                 for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) M = fmaxf(M, ml[(w4 * 8 + h) * 2]);
-                float Ls = 0.f, Os = 0.f;
+                float Ls = 0.f;
 #pragma unroll
                 for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) {
                     const float mw = ml[(w4 * 8 + h) * 2];
-                    const float f = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
-                    Ls += ml[(w4 * 8 + h) * 2 + 1] * f;
-                    Os += red[(w4 * HEADS + h) * DV + dcol];
+                    Ls += ml[(w4 * 8 + h) * 2 + 1] * ((mw == -INFINITY) ? 0.f : fast_exp2(mw - M));
                 }
                 hm[h] = M;
                 hl[h] = Ls;
-                hsum[h] = Os;
             }
-            if (ns == 1) {
-                // one split holds every key: finish here (gate values fetched at the item start)
-                float hv[HEADS];
 #pragma unroll
-                for (int h = 0; h < HEADS; ++h) hv[h] = (hl[h] > 0.f) ? hsum[h] / hl[h] : 0.f;
+            for (int j = 0; j < COLS; ++j) {
+                const int col = dcol + j * NCT;
+                float hsum[HEADS];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float dd = hv[i] - lam_pre[i] * hv[4];
-                    out[(orow0 + i) * DV + dcol] = __float2bfloat16_rn(__fdividef(dd, 1.f + __expf(-g_pre[i])));
+                for (int h = 0; h < HEADS; ++h) {
+                    float Os = 0.f;
+#pragma unroll
+                    for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) Os += red[(w4 * HEADS + h) * DV + col];
+                    hsum[h] = Os;
                 }
-            } else {
-                const size_t slot = (static_cast<size_t>(d.b) * hkv + d.group) * ns + d.split;
-                float *wo = ws + slot * (HEADS * DV);
-                float *wml = ws + plan.ml_offset_floats + slot * (HEADS * 2);
+                if (ns == 1) {
+                    // one split holds every key: finish here (gate values fetched at the item start)
+                    float hv[HEADS];
 #pragma unroll
-                for (int h = 0; h < HEADS; ++h) wo[h * DV + dcol] = hsum[h];
+                    for (int h = 0; h < HEADS; ++h) hv[h] = (hl[h] > 0.f) ? hsum[h] / hl[h] : 0.f;
 #pragma unroll
-                for (int h = 0; h < HEADS; ++h)
-                    if (dcol == h) {
-                        wml[h * 2 + 0] = hm[h];
-                        wml[h * 2 + 1] = hl[h];
+                    for (int i = 0; i < 4; ++i) {
+                        const float dd = hv[i] - lam_pre[i] * hv[4];
+                        out[(orow0 + i) * DV + col] = __float2bfloat16_rn(__fdividef(dd, 1.f + __expf(-g_pre[j][i])));
                     }
+                } else {
+                    const size_t slot = (static_cast<size_t>(d.b) * hkv + d.group) * ns + d.split;
+                    float *wo = ws + slot * (HEADS * DV);
+#pragma unroll
+                    for (int h = 0; h < HEADS; ++h) wo[h * DV + col] = hsum[h];
+                    if (j == 0) {
+                        float *wml = ws + plan.ml_offset_floats + slot * (HEADS * 2);
+#pragma unroll
+                        for (int h = 0; h < HEADS; ++h)
+                            if (dcol == h) {
+                                wml[h * 2 + 0] = hm[h];
+                                wml[h * 2 + 1] = hl[h];
+                            }
+                    }
+                }
             }
             // every consumer is done with ml/red before the next item writes them
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+            asm volatile("bar.sync 1, %0;" ::"n"(NCT) : "memory");
         }
     }
 }
@@ -432,26 +468,35 @@ gdla_decode_combine_kernel(const float *__restrict__ ws, const int32_t *__restri
                                           threadIdx.x);
 }
 
-int decode_smem_bytes() { return dc::SMEM_BYTES; }
+int decode_smem_bytes() { return SplitCfg::SMEM_BYTES; }
 
-cudaError_t launch_decode(const DecodeLaunch &L, const DecodePlan &plan, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(gdla_decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         dc::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    int dev = 0, num_sms = 0;
-    e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+int decode_key_tile(const DecodePlan &plan) { return plan.num_splits == 1 ? WindowCfg::TK : SplitCfg::TK; }
+
+template <class C>
+static cudaError_t launch_split(const DecodeLaunch &L, const DecodePlan &plan, int num_sms, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(gdla_decode_split_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // One split per sequence (windows, short caches): few small items whose
-    // latency chains dominate, so two persistent CTAs per SM pipeline them.
+    // latency chains dominate, so persistent CTAs (all resident) pipeline them.
     // Several splits: many items of similar size, balanced best by the hardware
     // scheduler with one item per CTA (the same kernel, one loop trip each).
     const long long work = static_cast<long long>(plan.num_splits) * plan.hkv * plan.batch;
-    const long long resident = 2ll * num_sms;  // two CTAs per SM
+    const long long resident = static_cast<long long>(C::CTAS_PER_SM) * num_sms;
     const unsigned grid = static_cast<unsigned>((plan.num_splits == 1 && work > resident) ? resident : work);
-    gdla_decode_split_kernel<<<grid, dc::NUM_THREADS, dc::SMEM_BYTES, stream>>>(
+    gdla_decode_split_kernel<C><<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(
         L.tm_k, L.tm_v, L.q_sig, L.q_noise, L.cu_seqlens_k, L.lambda, L.gate, L.out, L.ws, plan);
-    e = cudaPeekAtLastError();
+    return cudaPeekAtLastError();
+}
+
+cudaError_t launch_decode(const DecodeLaunch &L, const DecodePlan &plan, cudaStream_t stream) {
+    int dev = 0, num_sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    // The K/V tensor maps were encoded with decode_key_tile(plan) rows per box.
+    e = (plan.num_splits == 1) ? launch_split<WindowCfg>(L, plan, num_sms, stream)
+                               : launch_split<SplitCfg>(L, plan, num_sms, stream);
     if (e != cudaSuccess || plan.num_splits == 1) return e;
     dim3 grid2(plan.hkv, plan.batch);
     gdla_decode_combine_kernel<<<grid2, 160, 0, stream>>>(L.ws, L.cu_seqlens_k, L.lambda, L.gate, L.out, plan);

@@ -70,6 +70,16 @@ def test_deterministic():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+def test_single_split_persistent_uneven_items():
+    """Short caches (one split): 700 sequences x 2 KV groups = 1,400 items, more
+    than the resident persistent CTAs, with 1 to 32 key stages each, so each
+    CTA's K/V stage ring runs on across items of different lengths."""
+    rng = np.random.default_rng(57)
+    lengths = tuple(int(x) for x in rng.integers(1, 1001, size=700))
+    _check(lengths, 2, 0, 57, max_len=1000)
+    _check(lengths, 2, 100, 58, max_len=1000)
+
+
 @pytest.mark.parametrize("w", [gi.DECODE_FULL, gi.DECODE_W128], ids=lambda w: w.name)
 def test_decode_B64_H16(w):
     lengths = w.kv_lengths()

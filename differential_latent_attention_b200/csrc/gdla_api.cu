@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
 #include <memory>
 #include <mutex>
 #include <vector>
@@ -47,6 +48,21 @@ bool make_map(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+}  // namespace
+
+int device_sm_count(int dev) {
+    static std::atomic<int> sms[kMaxCachedDevices];
+    int n = 0;
+    if (dev < 0 || dev >= kMaxCachedDevices)
+        return cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess ? n : 0;
+    n = sms[dev].load(std::memory_order_relaxed);
+    if (n == 0 && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+        sms[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+namespace {
 
 bool aligned16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -146,7 +162,7 @@ gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *
     L.gate = static_cast<const __nv_bfloat16 *>(gate_logits);
     L.out = static_cast<__nv_bfloat16 *>(out);
 
-    std::unique_ptr<PrefillPlan> plan(new PrefillPlan());
+    std::unique_ptr<PrefillPlan> plan(new PrefillPlan);  // filled up to n_items / n_seqs, the rest unread
     std::vector<int> local(batch, -1);
     size_t pos = 0;
     while (pos < items.size()) {
@@ -171,6 +187,7 @@ gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *
             ++pos;
         }
         for (int s : used) local[s] = -1;
+        P.n_seqs = n_seq;
         if (launch_prefill(L, P, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDLA_ERR_CUDA;
     }
     return GDLA_OK;

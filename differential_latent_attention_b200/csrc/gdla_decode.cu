@@ -21,6 +21,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "gdla_internal.h"
 #include "gdla_ptx.cuh"
 
@@ -473,10 +475,17 @@ int decode_smem_bytes() { return SplitCfg::SMEM_BYTES; }
 int decode_key_tile(const DecodePlan &plan) { return plan.num_splits == 1 ? WindowCfg::TK : SplitCfg::TK; }
 
 template <class C>
-static cudaError_t launch_split(const DecodeLaunch &L, const DecodePlan &plan, int num_sms, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(gdla_decode_split_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+static cudaError_t launch_split(const DecodeLaunch &L, const DecodePlan &plan, int dev, int num_sms,
+                                cudaStream_t stream) {
+    // shared-memory opt-in once per device
+    static std::atomic<uint64_t> attr_set{0};
+    const uint64_t bit = (dev >= 0 && dev < kMaxCachedDevices) ? (1ull << dev) : 0ull;
+    if (!bit || !(attr_set.load(std::memory_order_relaxed) & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(gdla_decode_split_kernel<C>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set.fetch_or(bit, std::memory_order_relaxed);
+    }
     // One split per sequence (windows, short caches): few small items whose
     // latency chains dominate, so persistent CTAs (all resident) pipeline them.
     // Several splits: many items of similar size, balanced best by the hardware
@@ -490,13 +499,14 @@ static cudaError_t launch_split(const DecodeLaunch &L, const DecodePlan &plan, i
 }
 
 cudaError_t launch_decode(const DecodeLaunch &L, const DecodePlan &plan, cudaStream_t stream) {
-    int dev = 0, num_sms = 0;
+    int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
+    const int num_sms = device_sm_count(dev);
+    if (num_sms <= 0) return cudaErrorInvalidDevice;
     // The K/V tensor maps were encoded with decode_key_tile(plan) rows per box.
-    e = (plan.num_splits == 1) ? launch_split<WindowCfg>(L, plan, num_sms, stream)
-                               : launch_split<SplitCfg>(L, plan, num_sms, stream);
+    e = (plan.num_splits == 1) ? launch_split<WindowCfg>(L, plan, dev, num_sms, stream)
+                               : launch_split<SplitCfg>(L, plan, dev, num_sms, stream);
     if (e != cudaSuccess || plan.num_splits == 1) return e;
     dim3 grid2(plan.hkv, plan.batch);
     gdla_decode_combine_kernel<<<grid2, 160, 0, stream>>>(L.ws, L.cu_seqlens_k, L.lambda, L.gate, L.out, plan);

@@ -23,16 +23,24 @@ constexpr int kPlanMaxItems = 6144;  // q-tiles per launch
 constexpr int kItemSeqShift = 20;
 constexpr uint32_t kItemTileMask = (1u << kItemSeqShift) - 1u;
 
-// Passed by value (constant bank): the q-tiles of one launch, heaviest first.
-struct PrefillPlan {
+// Passed by value (kernel parameters): the q-tiles of one launch, heaviest
+// first. The host builds the largest form and launches the smallest capacity
+// that holds the plan, so a launch carries ~3.3 KB, ~8.7 KB or ~26.6 KB.
+template <int MAX_ITEMS, int MAX_SEQS>
+struct PrefillPlanT {
+    static constexpr int kMaxItems = MAX_ITEMS;
+    static constexpr int kMaxSeqs = MAX_SEQS;
     int n_items;
     int hkv;
     int window;
-    int pad_;
-    int seq_start[kPlanMaxSeqs];  // packed row of each sequence's first token
-    int seq_len[kPlanMaxSeqs];
-    uint32_t items[kPlanMaxItems];  // (local sequence << kItemSeqShift) | CTA block index
+    int n_seqs;
+    int seq_start[MAX_SEQS];  // packed row of each sequence's first token
+    int seq_len[MAX_SEQS];
+    uint32_t items[MAX_ITEMS];  // (local sequence << kItemSeqShift) | CTA block index
 };
+using PrefillPlan = PrefillPlanT<kPlanMaxItems, kPlanMaxSeqs>;
+using PrefillPlanMedium = PrefillPlanT<2048, 64>;
+using PrefillPlanSmall = PrefillPlanT<768, 32>;
 
 struct PrefillLaunch {
     CUtensorMap tm_qs, tm_qn, tm_k, tm_v;
@@ -42,6 +50,10 @@ struct PrefillLaunch {
 };
 
 cudaError_t launch_prefill(const PrefillLaunch &launch, const PrefillPlan &plan, cudaStream_t stream);
+
+// SM count of a device, queried once per device and cached (0 on failure).
+constexpr int kMaxCachedDevices = 64;
+int device_sm_count(int dev);
 
 // Decode: split-KV.
 constexpr int kDecodeMaxSplits = 64;

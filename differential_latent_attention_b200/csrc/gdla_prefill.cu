@@ -44,6 +44,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <cstring>
+
 #include "gdla_internal.h"
 #include "gdla_ptx.cuh"
 
@@ -167,12 +170,12 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&o)[32], float inv_l, 
 }
 }  // namespace pf
 
-template <class C>
+template <class C, class Plan>
 __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_qn,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const float *__restrict__ lambda, const __nv_bfloat16 *__restrict__ gate,
-                    __nv_bfloat16 *__restrict__ out, const __grid_constant__ PrefillPlan plan) {
+                    __nv_bfloat16 *__restrict__ out, const __grid_constant__ Plan plan) {
     using namespace pf;
     constexpr int TILES = C::TILES, BN = C::BN, STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -598,26 +601,61 @@ PrefillGeometry prefill_geometry(int window) {
     return {pf::CausalCfg::CTA_TOK, pf::CausalCfg::BN};
 }
 
-template <class C>
-static cudaError_t launch_cfg(const PrefillLaunch &L, const PrefillPlan &plan, int num_sms, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(gdla_prefill_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+// Each kernel instantiation opts in to its shared memory once per device (a
+// driver call that need not be repeated on every launch).
+template <class C, class Plan>
+static cudaError_t launch_cfg(const PrefillLaunch &L, const Plan &plan, int dev, int num_sms, cudaStream_t stream) {
+    static std::atomic<uint64_t> attr_set{0};  // bit per device
+    const uint64_t bit = (dev >= 0 && dev < kMaxCachedDevices) ? (1ull << dev) : 0ull;
+    if (!bit || !(attr_set.load(std::memory_order_relaxed) & bit)) {
+        cudaError_t e = cudaFuncSetAttribute(gdla_prefill_kernel<C, Plan>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set.fetch_or(bit, std::memory_order_relaxed);
+    }
     const long long work = static_cast<long long>(plan.n_items) * plan.hkv;
     const unsigned grid = static_cast<unsigned>(work < num_sms ? work : num_sms);
-    gdla_prefill_kernel<C><<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(L.tm_qs, L.tm_qn, L.tm_k, L.tm_v,
-                                                                          L.lambda, L.gate, L.out, plan);
+    gdla_prefill_kernel<C, Plan><<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(L.tm_qs, L.tm_qn, L.tm_k, L.tm_v,
+                                                                                L.lambda, L.gate, L.out, plan);
     return cudaPeekAtLastError();
 }
 
+// The plan in the smallest capacity that holds it (kernel parameters are
+// copied with every launch).
+template <class C>
+static cudaError_t launch_sized(const PrefillLaunch &L, const PrefillPlan &plan, int dev, int num_sms,
+                                cudaStream_t stream) {
+    auto shrink = [&](auto &small) {
+        small.n_items = plan.n_items;
+        small.hkv = plan.hkv;
+        small.window = plan.window;
+        small.n_seqs = plan.n_seqs;
+        std::memcpy(small.seq_start, plan.seq_start, sizeof(int) * plan.n_seqs);
+        std::memcpy(small.seq_len, plan.seq_len, sizeof(int) * plan.n_seqs);
+        std::memcpy(small.items, plan.items, sizeof(uint32_t) * plan.n_items);
+    };
+    if (plan.n_items <= PrefillPlanSmall::kMaxItems && plan.n_seqs <= PrefillPlanSmall::kMaxSeqs) {
+        PrefillPlanSmall small;
+        shrink(small);
+        return launch_cfg<C>(L, small, dev, num_sms, stream);
+    }
+    if (plan.n_items <= PrefillPlanMedium::kMaxItems && plan.n_seqs <= PrefillPlanMedium::kMaxSeqs) {
+        PrefillPlanMedium medium;
+        shrink(medium);
+        return launch_cfg<C>(L, medium, dev, num_sms, stream);
+    }
+    return launch_cfg<C>(L, plan, dev, num_sms, stream);
+}
+
 cudaError_t launch_prefill(const PrefillLaunch &L, const PrefillPlan &plan, cudaStream_t stream) {
-    int dev = 0, num_sms = 0;
+    int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
+    const int num_sms = device_sm_count(dev);
+    if (num_sms <= 0) return cudaErrorInvalidDevice;
     if (plan.window > 0 && plan.window <= kPrefillSlidingMaxWindow)
-        return launch_cfg<pf::SlidingCfg>(L, plan, num_sms, stream);
-    return launch_cfg<pf::CausalCfg>(L, plan, num_sms, stream);
+        return launch_sized<pf::SlidingCfg>(L, plan, dev, num_sms, stream);
+    return launch_sized<pf::CausalCfg>(L, plan, dev, num_sms, stream);
 }
 
 }  // namespace gdla

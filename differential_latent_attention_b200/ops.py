@@ -36,6 +36,9 @@ class GDLAError(RuntimeError):
 def library():
     """The loaded libgdla.so (raises if it has not been built)."""
     global _lib
+    lib = _lib
+    if lib is not None:
+        return lib
     with _lock:
         if _lib is None:
             path = _build.LIB_PATH
@@ -62,17 +65,21 @@ def library():
     return _lib
 
 
+# Arguments are passed to the C ABI as plain integers (the argtypes convert them).
 def _ptr(t):
-    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+    return t.data_ptr() if t is not None else 0
 
 
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+    return stream.cuda_stream
 
 
 def _check(t, name, dtype, shape):
+    # common case first: one combined test per call, the detailed ones only to explain a failure
+    if type(t) is torch.Tensor and t.dtype is dtype and t.shape == shape and t.is_cuda and t.is_contiguous():
+        return
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
@@ -94,7 +101,7 @@ def attn_fwd(q_sig, q_noise, k, v, lam, gate, seqlens, window=0, out=None, strea
     bf16 (written into ``out`` when given).
     """
     lens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32).reshape(-1))
-    n = int(lens.astype(np.int64).sum())
+    n = int(lens.sum(dtype=np.int64))
     hkv = q_noise.shape[1] if q_noise.dim() == 3 else -1
     hs = GROUP * hkv
     _check(q_sig, "q_sig", torch.bfloat16, (n, hs, DQK))
@@ -107,7 +114,7 @@ def attn_fwd(q_sig, q_noise, k, v, lam, gate, seqlens, window=0, out=None, strea
         out = torch.empty((n, hs, DV), dtype=torch.bfloat16, device=q_sig.device)
     _check(out, "out", torch.bfloat16, (n, hs, DV))
     st = library().gdla_attn_fwd(_ptr(q_sig), _ptr(q_noise), _ptr(k), _ptr(v), _ptr(lam), _ptr(gate), _ptr(out),
-                                 int(lens.shape[0]), lens.ctypes.data_as(ctypes.c_void_p), hkv, int(window),
+                                 int(lens.shape[0]), lens.__array_interface__["data"][0], hkv, int(window),
                                  _stream(stream))
     if st != 0:
         raise GDLAError(st, "gdla_attn_fwd")

@@ -26,8 +26,9 @@
  *    comment says HOST. Tensor base pointers must be 16-byte aligned.
  *  - bf16 is IEEE bfloat16 (1-8-7); lambda is fp32.
  *  - The library allocates no memory, keeps no state between calls (apart
- *    from the device-side failure word, see gdla_device_error) and may be
- *    called from several host threads at once.
+ *    from the device-side failure word, see gdla_device_error, and per-device
+ *    launch facts cached on the host: SM count, kernel attribute opt-ins) and
+ *    may be called from several host threads at once.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
  *    default stream). GDLA_OK means every kernel was enqueued; a CUDA launch
  *    failure is reported as GDLA_ERR_CUDA.

@@ -21,7 +21,8 @@ MAX_KV_HEADS = 64
 STATUS = {0: "GDLA_OK", 1: "GDLA_ERR_INVALID_ARG", 2: "GDLA_ERR_UNSUPPORTED", 3: "GDLA_ERR_WORKSPACE",
           4: "GDLA_ERR_CUDA"}
 EXPORTED = ("gdla_attn_fwd", "gdla_decode_workspace_bytes", "gdla_attn_decode", "gdla_attn_decode_noalloc",
-            "gdla_device_error", "gdla_status_string", "gdla_version")
+            "gdla_device_error", "gdla_selftest_wait_timeout", "gdla_status_string", "gdla_version")
+SELFTEST_SITE = 0x30001  # GDLA_SELFTEST_SITE
 
 _lib = None
 _lock = threading.Lock()
@@ -57,6 +58,8 @@ def library():
             lib.gdla_attn_decode_noalloc.restype = i
             lib.gdla_device_error.argtypes = [i]
             lib.gdla_device_error.restype = i
+            lib.gdla_selftest_wait_timeout.argtypes = [p]
+            lib.gdla_selftest_wait_timeout.restype = i
             lib.gdla_status_string.argtypes = [i]
             lib.gdla_status_string.restype = ctypes.c_char_p
             lib.gdla_version.argtypes = []
@@ -164,3 +167,11 @@ def attn_decode(q_sig, q_noise, k_cache, v_cache, cu_seqlens_k, max_seqlen_k, la
 def device_error(clear=True) -> int:
     """Code recorded by a kernel whose bounded wait ran out (0 = none); synchronises."""
     return int(library().gdla_device_error(1 if clear else 0))
+
+
+def selftest_wait_timeout(stream=None):
+    """Enqueue the failure-path self-test (a bounded wait that runs out after about a
+    second and records SELFTEST_SITE in the device failure word)."""
+    st = library().gdla_selftest_wait_timeout(_stream(stream))
+    if st != 0:
+        raise GDLAError(st, "gdla_selftest_wait_timeout")

@@ -182,6 +182,17 @@ GDLA_API gdla_status_t gdla_attn_decode_noalloc(const void *q_sig, const void *q
  */
 GDLA_API int gdla_device_error(int clear);
 
+/*
+ * Self-test of that failure path: launches one CTA (on `stream`) whose thread
+ * waits, with the kernels' own bounded wait, on an mbarrier that nothing ever
+ * arrives on. After the wait limit (about one second) it records
+ * GDLA_SELFTEST_SITE in the device failure word and the kernel returns; the
+ * context stays usable. No tensor is touched. Returns GDLA_OK once the kernel
+ * is enqueued, GDLA_ERR_CUDA if the launch fails.
+ */
+#define GDLA_SELFTEST_SITE 0x30001
+GDLA_API gdla_status_t gdla_selftest_wait_timeout(void *stream);
+
 /* Static, human-readable name of a status code. */
 GDLA_API const char *gdla_status_string(gdla_status_t status);
 

@@ -272,11 +272,7 @@ def run_gdla(args):
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 6), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "batch": len(w.seqlens), "seq_len": w.seqlens[0], "q_heads": 80,
-                   "signal_heads": 64, "noise_heads": 16, "kv_heads": 16, "dqk": 192, "dv": 128,
-                   "window": "full causal", "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed (512 MiB write) before every timed step, outside the events",
-                   "algorithmic_flops_per_step": flops},
+        "config": headline_config(w, world),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "peak_source": f"bf16_tflops (burst) of {peak_src}",
                      "kernel": PREFILL_KERNEL, "traffic": profiled_traffic(PREFILL_KERNEL, w.name)},
@@ -294,6 +290,15 @@ def run_gdla(args):
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
+
+
+def headline_config(w, world):
+    """The headline workload's config object, the same in both arms' JSON lines."""
+    return {"workload": w.name, "batch": len(w.seqlens), "seq_len": w.seqlens[0], "q_heads": 80,
+            "signal_heads": 64, "noise_heads": 16, "kv_heads": 16, "dqk": 192, "dv": 128,
+            "window": "full causal", "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed (512 MiB write) before every timed step, outside the events",
+            "algorithmic_flops_per_step": prefill_flops(w)}
 
 
 def extra_workloads(gdla, dev, flush, args, world, rank, peaks):
@@ -401,8 +406,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3 / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "batch": 1, "seq_len": 4096, "q_heads": 80, "kv_heads": 16, "dqk": 192,
-                   "dv": 128, "window": "full causal"},
+        "config": headline_config(w, world),
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

@@ -112,13 +112,21 @@ KERNEL_SOURCES = {
 }
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source text without comments, trailing spaces or blank lines: an
+    edit to comments does not change the kernel a profile was taken of."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of the sources a kernel is compiled from (its .cu file and the shared headers)."""
+    """Hash of the code a kernel is compiled from (its .cu file and the shared headers, comments excluded)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "differential_latent_attention_b200", "csrc")
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + b"\0" + f.read())
+        with open(os.path.join(csrc, name)) as f:
+            h.update(name.encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

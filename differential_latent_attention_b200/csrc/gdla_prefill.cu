@@ -18,7 +18,9 @@
 //       rows 32w + 30, 31    unused (zero queries)
 // Each BN-key K/V tile is staged once in shared memory (TMA) and consumed by
 // every tile and all five heads. Per key tile k and q tile x:
-//     S_x = Q_x K^T   tcgen05 M=128 N=BN K=192, smem operands, fp32 in TMEM
+//     S_x = Q_x K^T   tcgen05 M=128 N=BN K=192, fp32 in TMEM; K from shared
+//                     memory, Q from TMEM (one q tile, copied there per item) or
+//                     from shared memory (two q tiles)
 //     softmax_x       one warpgroup per tile, one TMEM lane per row: online
 //                     max/sum, P = exp2(.) rounded to bf16 into TMEM over S_x
 //     O_x += P_x V    tcgen05 with A = P from TMEM, B = V from smem (MN-major)
@@ -26,7 +28,8 @@
 // softmax of tile k runs; with two q tiles the softmax warpgroups alternate
 // (ping-pong). Epilogue: every warp finalises its rows (O/l), passes each
 // token's noise row to its four signal rows with warp shuffles, and writes
-// sigmoid(g)(H_S - lambda H_N) as bf16. Meanwhile the tensor core already
+// sigmoid(g)(H_S - lambda H_N) as bf16 (32-byte gate loads and output stores
+// when the buffers allow). Meanwhile the tensor core already
 // computes QK^T of the next item (its Q was loaded as soon as the last QK^T
 // of the current item finished).
 //
@@ -38,7 +41,8 @@
 //           is bound by HBM and 48-token items halve the per-token overheads.
 // Warps: 4 per q tile (softmax + epilogue), then the TMA producer warp (which
 // also zero-fills the unused Q rows once) and the MMA warp (TMEM allocation,
-// MMA issue by one elected lane of a converged warp).
+// MMA issue by one elected lane of a converged warp). The plan of a launch (its
+// items) travels in the kernel parameters, in one of three capacities.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>

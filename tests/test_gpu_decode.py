@@ -84,3 +84,9 @@ def test_single_split_persistent_uneven_items():
 def test_decode_B64_H16(w):
     lengths = w.kv_lengths()
     _check(tuple(int(x) for x in lengths), w.num_kv_heads, w.window, w.seed, max_len=32768)
+
+
+@pytest.mark.parametrize("window", [0, 128])
+def test_largest_kv_head_count(window):
+    """GDLA_MAX_KV_HEADS = 64 KV heads."""
+    _check((300, 2000, 1), 64, window, 56)

@@ -146,3 +146,16 @@ def test_more_blocks_than_one_launch_holds():
     seqlens = (800,) * 200
     rows = gi.sample_rows(seqlens, 3, seed=16, must_include=(0, 799))
     check_prefill(seqlens, 1, 0, 16, rows=rows)
+
+
+@pytest.mark.parametrize("window", [0, 128])
+def test_largest_kv_head_count(window):
+    """GDLA_MAX_KV_HEADS = 64 KV heads (256 signal + 64 noise query heads)."""
+    check_prefill((130, 31), 64, window, 20)
+
+
+@pytest.mark.parametrize("window", [257, 300, 1000])
+def test_windows_in_the_causal_configuration(window):
+    """Windows over 256 run the one-tile configuration with window masks and key-tile
+    skipping; the sequences are longer than the window, so both take effect."""
+    check_prefill((1500, 700), 2, window, 21)

@@ -52,21 +52,27 @@ PINS = [
 ]
 
 
-def _build_mutant(tmp_path, name, old, new):
+# Mutant builds stay inside the repository, in its (git-ignored) build folder.
+MUTANT_DIR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "_build", "oracle_mutants")
+
+
+def _build_mutant(name, old, new):
     src = open(SRC).read()
     assert src.count(old) >= 1, f"mutation site for {name} not found"
-    path = tmp_path / f"{name}.c"
-    path.write_text(src.replace(old, new, 1))   # first site: the prefill path
-    lib = tmp_path / f"lib{name}.so"
+    os.makedirs(MUTANT_DIR, exist_ok=True)
+    path = os.path.join(MUTANT_DIR, f"{name}.c")
+    with open(path, "w") as f:
+        f.write(src.replace(old, new, 1))   # first site: the prefill path
+    lib = os.path.join(MUTANT_DIR, f"lib{name}.so")
     subprocess.check_call(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-pthread", "-o", str(lib),
                            str(path), "-lm"])
     return str(lib)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_mutant_is_caught(name, tmp_path, monkeypatch):
+def test_mutant_is_caught(name, monkeypatch):
     old, new = MUTANTS[name]
-    path = _build_mutant(tmp_path, name, old, new)
+    path = _build_mutant(name, old, new)
     real = oracle._load()
     lib = ctypes.CDLL(path)
     for fn in ("gdla_oracle_prefill", "gdla_oracle_decode"):

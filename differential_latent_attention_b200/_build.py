@@ -51,7 +51,10 @@ def build(force: bool = False, verbose: bool = False) -> str:
            os.path.join(CSRC, "gdla_lib.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
-    subprocess.check_call(cmd)
+    # the compiler's intermediate files stay inside the repository
+    scratch = os.path.join(os.path.dirname(PKG), "_build", "tmp")
+    os.makedirs(scratch, exist_ok=True)
+    subprocess.check_call(cmd, env={**os.environ, "TMPDIR": scratch})
     os.replace(tmp, LIB_PATH)
     return LIB_PATH
 

@@ -41,8 +41,11 @@ def build(force: bool = False) -> str:
     """Compile gdla_oracle.c into libgdla_oracle.so (gcc, -O2, pthreads)."""
     if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
         tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        # the compiler's intermediate files stay inside the repository
+        scratch = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "_build", "tmp")
+        os.makedirs(scratch, exist_ok=True)
         subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
-                               "-o", tmp, _SRC, "-lm"])
+                               "-o", tmp, _SRC, "-lm"], env={**os.environ, "TMPDIR": scratch})
         os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
 

@@ -65,7 +65,7 @@ def _build_mutant(name, old, new):
         f.write(src.replace(old, new, 1))   # first site: the prefill path
     lib = os.path.join(MUTANT_DIR, f"lib{name}.so")
     subprocess.check_call(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-pthread", "-o", str(lib),
-                           str(path), "-lm"])
+                           str(path), "-lm"], env={**os.environ, "TMPDIR": MUTANT_DIR})
     return str(lib)
 
 

@@ -35,6 +35,9 @@ _lock = threading.Lock()
 GROUP = 4
 DQK = 192
 DV = 128
+DC = 512          # KV low-rank (latent) dim
+DR = 64           # shared rotary key dim
+DL = DC + DR      # width of a latent cache row and of an absorbed query
 
 
 def build(force: bool = False) -> str:
@@ -63,6 +66,9 @@ def _load():
             lib.gdla_oracle_decode.argtypes = [p, p, p, p, p, p, p, ctypes.c_int, ctypes.c_int,
                                                ctypes.c_int, p, ctypes.c_int]
             lib.gdla_oracle_decode.restype = ctypes.c_int
+            lib.gdla_oracle_decode_latent.argtypes = [p, p, p, p, p, p, p, ctypes.c_int, ctypes.c_int,
+                                                      ctypes.c_int, p, ctypes.c_int]
+            lib.gdla_oracle_decode_latent.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -151,4 +157,37 @@ def decode(q_sig, q_noise, k_cache, v_cache, cu_seqlens_k, lam, gate, window, nu
                                     _ptr(lam), _ptr(gate), b, hkv, int(window), _ptr(out), nt)
     if rc != 0:
         raise ValueError("gdla_oracle_decode rejected its arguments")
+    return out
+
+
+def decode_latent(q_abs_sig, q_abs_noise, ckv, cu_seqlens_k, w_uv, lam, gate, window, num_threads=None):
+    """GDLA decode over the compressed KV cache with the projections absorbed, in fp64.
+
+    q_abs_sig [B, 4H, 576] and q_abs_noise [B, H, 576]: queries as
+    [W^UK_j^T q_nope (512) | q_rope (64)]; ckv [Nk, 576]: per token [c (512) | kr (64)],
+    packed by cu_seqlens_k [B+1]; w_uv [H, 128, 512]; lam [B, 4H]; gate [B, 4H, 128].
+    All bf16 inputs as uint16 bit patterns. Returns float64 [B, 4H, 128].
+    """
+    hkv = q_abs_noise.shape[1]
+    hs = GROUP * hkv
+    q_abs_sig = _bits(q_abs_sig, (hs, DL), "q_abs_sig")
+    q_abs_noise = _bits(q_abs_noise, (hkv, DL), "q_abs_noise")
+    ckv = _bits(ckv, (DL,), "ckv")
+    w_uv = _bits(w_uv, (DV, DC), "w_uv")
+    gate = _bits(gate, (hs, DV), "gate")
+    lam = np.ascontiguousarray(lam, dtype=np.float32)
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens_k, dtype=np.int64))
+    b = cu.shape[0] - 1
+    if q_abs_sig.shape[0] != b or q_abs_noise.shape[0] != b or gate.shape[0] != b or lam.shape != (b, hs):
+        raise ValueError("decode_latent: per-sequence inputs must have leading dim B = len(cu_seqlens_k) - 1")
+    if w_uv.shape[0] != hkv:
+        raise ValueError("decode_latent: w_uv needs one [128, 512] matrix per KV head")
+    if cu[-1] > ckv.shape[0]:
+        raise ValueError("decode_latent: cache shorter than cu_seqlens_k[-1]")
+    out = np.zeros((b, hs, DV), dtype=np.float64)
+    nt = int(num_threads or default_threads())
+    rc = _load().gdla_oracle_decode_latent(_ptr(q_abs_sig), _ptr(q_abs_noise), _ptr(ckv), _ptr(cu), _ptr(w_uv),
+                                           _ptr(lam), _ptr(gate), b, hkv, int(window), _ptr(out), nt)
+    if rc != 0:
+        raise ValueError("gdla_oracle_decode_latent rejected its arguments")
     return out

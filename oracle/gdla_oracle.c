@@ -295,3 +295,135 @@ int gdla_oracle_decode(const uint16_t *q_sig, const uint16_t *q_noise, const uin
     free(jobs);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Decode over the compressed (latent) KV cache, with the projections        */
+/* absorbed                                                                  */
+/* ------------------------------------------------------------------------ */
+/*
+ * What it follows ([A], head-configuration paragraph): the KV path keeps one
+ * compressed KV row per token (KV low-rank dimension 512) and one rotary key
+ * (64) shared by every KV head; the 16 KV heads are an up-projection of the
+ * compressed row. Readings: the 192 query-key dims are 128 non-rotary then 64
+ * rotary; per KV head j,
+ *     K_j,u = [ W^UK_j c_u (128) | kr_u (64) ],   V_j,u = W^UV_j c_u (128),
+ * with W^UK_j and W^UV_j of shape [128 x 512]. A query of group j with its
+ * non-rotary part absorbed, q_abs = [ W^UK_j^T q_nope (512) | q_rope (64) ],
+ * gives q . K_j,u = q_abs . [c_u | kr_u], and sum_u p_u V_j,u = W^UV_j sum_u p_u c_u.
+ * So every head attends over the shared 576-wide rows [c_u | kr_u] (same
+ * 1/sqrt(192) scale) and its 512-wide latent output is projected by W^UV_j.
+ */
+#define DC 512      /* KV low-rank (latent) dim */
+#define DR 64       /* shared rotary key dim */
+#define DL (DC + DR)
+
+/* One head over the latent rows: the 512-wide softmax-weighted latent average. */
+static void attend_latent(const uint16_t *q, const uint16_t *rows, long nkeys, double *scores, double *o) {
+    double qd[DL];
+    for (int e = 0; e < DL; ++e) qd[e] = bf16_to_double(q[e]);
+    const double root = sqrt((double)DQK);
+    double smax = -INFINITY;
+    for (long u = 0; u < nkeys; ++u) {
+        const uint16_t *r = rows + u * DL;
+        double s = 0.0;
+        for (int e = 0; e < DL; ++e) s += qd[e] * bf16_to_double(r[e]);
+        s = s / root;
+        scores[u] = s;
+        if (s > smax) smax = s;
+    }
+    double den = 0.0;
+    for (int e = 0; e < DC; ++e) o[e] = 0.0;
+    for (long u = 0; u < nkeys; ++u) {
+        const uint16_t *r = rows + u * DL;
+        const double w = exp(scores[u] - smax);
+        den += w;
+        for (int e = 0; e < DC; ++e) o[e] += w * bf16_to_double(r[e]);
+    }
+    for (int e = 0; e < DC; ++e) o[e] /= den;
+}
+
+/* H = W^UV_j o: [128 x 512] times a 512-vector. */
+static void up_project(const uint16_t *w_uv_j, const double *o, double *h) {
+    for (int d = 0; d < DV; ++d) {
+        double acc = 0.0;
+        for (int e = 0; e < DC; ++e) acc += bf16_to_double(w_uv_j[(long)d * DC + e]) * o[e];
+        h[d] = acc;
+    }
+}
+
+typedef struct {
+    const uint16_t *q_sig, *q_noise, *ckv, *w_uv, *gate;
+    const float *lambda;
+    const int64_t *cu;
+    int batch, hkv, window;
+    double *out;
+    long max_keys;
+    int nthreads, tid;
+} latent_job_t;
+
+static void *latent_worker(void *arg) {
+    latent_job_t *J = (latent_job_t *)arg;
+    const int hs = GROUP * J->hkv;
+    double *scores = (double *)malloc(sizeof(double) * (size_t)(J->max_keys > 0 ? J->max_keys : 1));
+    if (!scores) return (void *)1;
+    const int64_t ntasks = (int64_t)J->batch * J->hkv;
+    for (int64_t task = J->tid; task < ntasks; task += J->nthreads) {
+        const int64_t b = task / J->hkv;
+        const int j = (int)(task % J->hkv);
+        const int64_t s0 = J->cu[b];
+        const int64_t t = J->cu[b + 1] - s0 - 1;   /* the query's own position */
+        int64_t lo = 0;
+        if (J->window > 0 && t - J->window + 1 > 0) lo = t - J->window + 1;
+        const long nkeys = (long)(t - lo + 1);
+        const uint16_t *rows = J->ckv + (s0 + lo) * DL;
+        const uint16_t *w_uv_j = J->w_uv + (long)j * DV * DC;
+        double o[DC], hn[DV], hsig[DV];
+        attend_latent(J->q_noise + (b * J->hkv + j) * DL, rows, nkeys, scores, o);
+        up_project(w_uv_j, o, hn);
+        for (int i = 0; i < GROUP; ++i) {
+            const int64_t head = b * hs + (long)GROUP * j + i;
+            attend_latent(J->q_sig + head * DL, rows, nkeys, scores, o);
+            up_project(w_uv_j, o, hsig);
+            const double l = (double)J->lambda[head];
+            for (int d = 0; d < DV; ++d) {
+                const double dd = hsig[d] - l * hn[d];
+                const double g = bf16_to_double(J->gate[head * DV + d]);
+                J->out[head * DV + d] = dd / (1.0 + exp(-g));
+            }
+        }
+    }
+    free(scores);
+    return NULL;
+}
+
+/*
+ * Varlen decode over the latent cache: one query per sequence at position
+ * L_b - 1, queries already absorbed.
+ *   q_abs_sig [B, 4*hkv, 576], q_abs_noise [B, hkv, 576] bf16 bits,
+ *   ckv [Nk, 576] = [c (512) | kr (64)] bf16 bits (sequence b owns rows
+ *   cu[b]..cu[b+1]-1), w_uv [hkv, 128, 512] bf16 bits, lambda [B, 4*hkv] fp32,
+ *   gate [B, 4*hkv, 128]; out [B, 4*hkv, 128] doubles.
+ * Every L_b must be >= 1. Returns 0, or -1 on a bad argument.
+ */
+int gdla_oracle_decode_latent(const uint16_t *q_abs_sig, const uint16_t *q_abs_noise, const uint16_t *ckv,
+                              const int64_t *cu_seqlens_k, const uint16_t *w_uv, const float *lambda,
+                              const uint16_t *gate, int batch, int hkv, int window, double *out,
+                              int nthreads) {
+    if (hkv < 1 || batch < 0 || nthreads < 1) return -1;
+    long max_len = 0;
+    for (int b = 0; b < batch; ++b) {
+        const int64_t len = cu_seqlens_k[b + 1] - cu_seqlens_k[b];
+        if (len < 1) return -1;
+        if (len > max_len) max_len = (long)len;
+    }
+    latent_job_t *jobs = (latent_job_t *)malloc(sizeof(latent_job_t) * (size_t)nthreads);
+    if (!jobs) return -1;
+    for (int i = 0; i < nthreads; ++i) {
+        latent_job_t J = {q_abs_sig, q_abs_noise, ckv, w_uv, gate, lambda, cu_seqlens_k,
+                          batch, hkv, window, out, max_len, nthreads, i};
+        jobs[i] = J;
+    }
+    int rc = run_threads(latent_worker, jobs, sizeof(latent_job_t), nthreads);
+    free(jobs);
+    return rc;
+}

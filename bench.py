@@ -38,6 +38,11 @@ import gdla_inputs as gi  # noqa: E402
 
 METRIC = "GDLA fwd TFLOP/s (full causal) & tokens/s (SWA-128, decode) vs B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Datasheet figures, reported beside the measured-peak fractions. The measured HBM
+# figure is a copy (read + write) rate, not a ceiling for a kernel that only reads.
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+L2_BYTES = 126 << 20
+EXTRA_STEPS_MIN = 20  # timed steps of each extra workload (the median is reported)
 L2_FLUSH_BYTES = 512 << 20
 FLOPS_PER_PAIR_HEAD = 2 * 192 + 2 * 128
 PREFILL_KERNEL = "gdla_prefill_kernel"
@@ -219,6 +224,54 @@ def time_steps(fn, steps, warmup, flush, world):
     return [s.elapsed_time(e) for s, e in ev]
 
 
+def time_rotating(fns, steps, warmup, world):
+    """Per-step device time (ms) with CUDA events, step i running fns[i % len(fns)]
+    and no L2 flush: the sets' inputs together exceed twice the L2, so each step's
+    inputs have been evicted since their previous use and no dirty flush lines are
+    written back inside the timed region."""
+    for i in range(warmup):
+        fns[i % len(fns)]()
+    torch.cuda.synchronize()
+    barrier(world)
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i, (s, e) in enumerate(ev):
+        s.record(stream)
+        fns[(warmup + i) % len(fns)]()
+        e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return [s.elapsed_time(e) for s, e in ev]
+
+
+def hbm_roofline(nbytes, ms, peak):
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s", "frac": round(gbs / peak, 4),
+            "frac_nominal": round(gbs / NOMINAL_PEAKS["hbm_gbs"], 4)}
+
+
+def decode_rotation_sets(wd, lengths, n_sets, shift, dev, rank):
+    """``n_sets`` decode problems sharing one packed cache: set r places every
+    sequence ``r * shift`` rows further along it (so with ``shift`` >= the window
+    the sets read disjoint cache rows) and has its own queries, lambda, gate and
+    output."""
+    lengths = np.asarray(lengths, dtype=np.int64)
+    ext = lengths.copy()
+    ext[-1] += (n_sets - 1) * shift
+    base = gi.make_decode_inputs(ext, wd.num_kv_heads, wd.seed + 1000 * rank, device=dev)
+    cu0 = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    sets = []
+    for r in range(n_sets):
+        small = gi.make_decode_inputs(np.ones(len(lengths), dtype=np.int64), wd.num_kv_heads,
+                                      wd.seed + 1000 * rank + 7919 * (r + 1), device=dev)
+        sets.append({"q_sig": small["q_sig"], "q_noise": small["q_noise"], "lam": small["lam"],
+                     "gate": small["gate"], "k_cache": base["k_cache"], "v_cache": base["v_cache"],
+                     "cu_seqlens_k": torch.as_tensor((cu0 + r * shift).astype(np.int32), device=dev),
+                     "out": torch.empty((len(lengths), 4 * wd.num_kv_heads, 128), dtype=torch.bfloat16,
+                                        device=dev)})
+    return sets
+
+
 def e2e_pipelined(gdla, w, host, bufs, outs, out_h, steps, world):
     """Mean ms per step of copy-in -> attn_fwd -> read-back with consecutive steps
     overlapped: step i uses device set i % 2; its inputs are copied on one stream
@@ -340,6 +393,7 @@ def run_gdla(args):
         "config": headline_config(w, world),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 3), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "peak_source": f"bf16_tflops (burst) of {peak_src}",
+                     "frac_nominal": round(achieved / NOMINAL_PEAKS["bf16_tflops"], 4),
                      "kernel": PREFILL_KERNEL, "traffic": profiled_traffic(PREFILL_KERNEL, w.name)},
         "e2e": {"value": round(e2e_value, 4), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
@@ -369,58 +423,151 @@ def headline_config(w, world):
 
 
 def extra_workloads(gdla, dev, flush, args, world, rank, peaks):
+    """The other workloads: SWA-128 prefill, the hybrid 1 full + 3 window-128
+    schedule at T = 65536, and varlen decode (full context and window 128). Each
+    is timed over at least EXTRA_STEPS_MIN steps and reported as the median.
+    On one GPU (rank 0) each also gets the fp64 oracle timed on the same inputs
+    (all rows, or a labelled sample for the T = 65536 full-causal layer)."""
+    cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
     res = []
-    steps = max(3, min(args.steps, 20))
+    steps = max(EXTRA_STEPS_MIN, args.steps)
     hbm = peaks["hbm_gbs"]
+    # tiny: T = 256, one KV group (a parity case; launch-latency bound, 1.2 MB fits in L2)
+    w = gi.TINY
+    t = gi.make_prefill_inputs(w.seqlens, w.num_kv_heads, w.seed + 1000 * rank, device=dev)
+    out = torch.empty((w.tokens, 4 * w.num_kv_heads, 128), dtype=torch.bfloat16, device=dev)
+    per = time_steps(lambda: gdla.attn_fwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"],
+                                           w.seqlens, w.window, out=out), steps, 3, lambda: None, world)
+    ms = reduce_max(statistics.median(per), world, dev)
+    res.append({"workload": w.name, "metric": "tokens/s", "value": w.tokens * world / (ms * 1e-3),
+                "ms": round(ms, 5), "steps": steps, "stat": "median",
+                "l2": "not flushed (inputs resident; the call is launch-latency bound)",
+                "tflops": prefill_flops(w) / (ms * 1e-3) / 1e12})
+    if cpu:
+        res[-1]["cpu_baseline"] = oracle_prefill_rows(t, w, None, "tokens/s")
+    del t, out
     # sliding window 128 prefill, B = 2 x 32768
     w = gi.SWA
     t = gi.make_prefill_inputs(w.seqlens, w.num_kv_heads, w.seed + 1000 * rank, device=dev)
     out = torch.empty((w.tokens, 64, 128), dtype=torch.bfloat16, device=dev)
     per = time_steps(lambda: gdla.attn_fwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"],
                                            w.seqlens, w.window, out=out), steps, 3, flush, world)
-    ms = reduce_max(statistics.mean(per), world, dev)
-    gbs = prefill_bytes(w) / (ms * 1e-3) / 1e9
+    ms = reduce_max(statistics.median(per), world, dev)
     res.append({"workload": w.name, "metric": "tokens/s", "value": w.tokens * world / (ms * 1e-3),
-                "ms": round(ms, 5), "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
-                                                 "unit": "GB/s", "frac": round(gbs / hbm, 4)},
+                "ms": round(ms, 5), "steps": steps, "stat": "median",
+                "roofline": hbm_roofline(prefill_bytes(w), ms, hbm),
                 "tflops": prefill_flops(w) / (ms * 1e-3) / 1e12})
+    if cpu:
+        res[-1]["cpu_baseline"] = oracle_prefill_rows(t, w, None, "tokens/s")
     del t, out
     # the pages' hybrid schedule: one full-causal layer then three window-128 layers, T = 65536
-    hyb_ms, hyb_flops, hyb_bytes = 0.0, 0.0, 0.0
     layer_ms = []
-    for wl in gi.HYBRID_LAYERS:
+    hyb_flops, hyb_bytes = 0.0, 0.0
+    hyb_cpu = {}
+    for li, wl in enumerate(gi.HYBRID_LAYERS):
         t = gi.make_prefill_inputs(wl.seqlens, wl.num_kv_heads, wl.seed + 1000 * rank, device=dev)
         out = torch.empty((wl.tokens, 64, 128), dtype=torch.bfloat16, device=dev)
         per = time_steps(lambda: gdla.attn_fwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"],
-                                               wl.seqlens, wl.window, out=out), 3, 3, flush, world)
-        ms = reduce_max(statistics.mean(per), world, dev)
-        layer_ms.append(round(ms, 4))
-        hyb_ms += ms
+                                               wl.seqlens, wl.window, out=out), steps, 3, flush, world)
+        layer_ms.append(reduce_max(statistics.median(per), world, dev))
         hyb_flops += prefill_flops(wl)
         hyb_bytes += prefill_bytes(wl) if wl.window > 0 else 0.0
+        if cpu and li == 0:
+            rows = gi.sample_rows(wl.seqlens, 512, seed=40, must_include=(0, 1, 127, 128, 65535))
+            hyb_cpu["full_layer"] = oracle_prefill_rows(t, wl, rows, "rows/s")
+        elif cpu and li == 1:
+            hyb_cpu["window_layer"] = oracle_prefill_rows(t, wl, None, "tokens/s")
         del t, out
+    hyb_ms = sum(layer_ms)
+    full_tflops = prefill_flops(gi.HYBRID_LAYERS[0]) / (layer_ms[0] * 1e-3) / 1e12
+    swa_gbs = hyb_bytes / (sum(layer_ms[1:]) * 1e-3) / 1e9
     res.append({"workload": "hybrid_T65536_H16_1full_3w128", "metric": "tokens/s (4 layers)",
                 "value": gi.HYBRID_LAYERS[0].tokens * 4 * world / (hyb_ms * 1e-3), "ms": round(hyb_ms, 4),
-                "layer_ms": layer_ms,
-                "full_layer_tflops": round(prefill_flops(gi.HYBRID_LAYERS[0]) / (layer_ms[0] * 1e-3) / 1e12, 2),
-                "swa_layers_gbs": round(hyb_bytes / (sum(layer_ms[1:]) * 1e-3) / 1e9, 1)})
-    # varlen decode, 64 sequences, full context and window 128
+                "steps": steps, "stat": "median per layer", "layer_ms": [round(x, 4) for x in layer_ms],
+                "full_layer_tflops": round(full_tflops, 2),
+                "full_layer_frac": round(full_tflops / peaks["bf16_tflops"], 4),
+                "swa_layers_gbs": round(swa_gbs, 1), "swa_layers_frac": round(swa_gbs / hbm, 4)})
+    if hyb_cpu:
+        full_s = hyb_cpu["full_layer"]["extrapolated_full_s"]
+        win_s = hyb_cpu["window_layer"]["seconds"]
+        hyb_cpu.update({"value": round(gi.HYBRID_LAYERS[0].tokens * 4 / (full_s + 3 * win_s), 3),
+                        "unit": "tokens/s (4 layers)", "cores": hyb_cpu["window_layer"]["cores"], "kind": "oracle",
+                        "sample": "full-causal layer: 512 sampled rows, extrapolated to all 65,536 rows by flops; "
+                                  "window-128 layer: all rows (layers 2 and 3 have the same shape)",
+                        "extrapolated": True})
+        res[-1]["cpu_baseline"] = hyb_cpu
+    # varlen decode, 64 sequences: full context (L2 flushed; 11 GB of cache), and
+    # window 128 (88 MB, under L2: 4 rotating input sets, flushed figure beside it)
     for wd in (gi.DECODE_FULL, gi.DECODE_W128):
         lengths = wd.kv_lengths()
-        d = gi.make_decode_inputs(lengths, wd.num_kv_heads, wd.seed + 1000 * rank, device=dev)
-        o = torch.empty((wd.batch, 64, 128), dtype=torch.bfloat16, device=dev)
         ws_bytes = gdla.decode_workspace_bytes(wd.batch, wd.num_kv_heads, 32768, wd.window)
         ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
-        per = time_steps(lambda: gdla.attn_decode(d["q_sig"], d["q_noise"], d["k_cache"], d["v_cache"],
-                                                  d["cu_seqlens_k"], 32768, d["lam"], d["gate"], wd.window,
-                                                  out=o, workspace=ws), steps, 3, flush, world)
-        ms = reduce_max(statistics.mean(per), world, dev)
-        gbs = decode_bytes(lengths, wd.num_kv_heads, wd.window) / (ms * 1e-3) / 1e9
-        res.append({"workload": wd.name, "metric": "query tokens/s", "value": wd.batch * world / (ms * 1e-3),
-                    "ms": round(ms, 5), "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm,
-                                                     "unit": "GB/s", "frac": round(gbs / hbm, 4)}})
-        del d, o, ws
+        nbytes = decode_bytes(lengths, wd.num_kv_heads, wd.window)
+
+        def call(d):
+            gdla.attn_decode(d["q_sig"], d["q_noise"], d["k_cache"], d["v_cache"], d["cu_seqlens_k"], 32768,
+                             d["lam"], d["gate"], wd.window, out=d["out"], workspace=ws)
+
+        n_sets = 1 if wd.window <= 0 else max(3, int(math.ceil(2 * L2_BYTES / nbytes)) + 1)
+        sets = decode_rotation_sets(wd, lengths, n_sets, max(wd.window, 0), dev, rank)
+        flushed = time_steps(lambda: call(sets[0]), steps, 3, flush, world)
+        ms_flushed = reduce_max(statistics.median(flushed), world, dev)
+        entry = {"workload": wd.name, "metric": "query tokens/s", "steps": steps, "stat": "median"}
+        if n_sets > 1:
+            rot = time_rotating([lambda d=d: call(d) for d in sets], steps, 3 * n_sets, world)
+            ms = reduce_max(statistics.median(rot), world, dev)
+            entry["l2"] = (f"{n_sets} rotating input sets ({n_sets * nbytes / 1e6:.0f} MB of visible K/V and "
+                           f"per-query tensors, > 2x L2), no flush")
+            entry["flushed"] = {"ms": round(ms_flushed, 5), "roofline": hbm_roofline(nbytes, ms_flushed, hbm),
+                                "l2": "flushed (512 MiB write) before every timed step"}
+        else:
+            ms = ms_flushed
+            entry["l2"] = "flushed (512 MiB write) before every timed step"
+        entry.update({"value": wd.batch * world / (ms * 1e-3), "ms": round(ms, 5),
+                      "roofline": hbm_roofline(nbytes, ms, hbm)})
+        if cpu:
+            entry["cpu_baseline"] = oracle_decode_all(sets[0], wd)
+        res.append(entry)
+        del sets, ws
     return res
+
+
+def oracle_prefill_rows(t, w, rows, unit):
+    """The fp64 oracle, as it stands, on the same prefill inputs: all rows (rows is
+    None; value in tokens/s) or the given rows (value in rows/s, with the
+    full-workload time extrapolated by flops and labelled as such)."""
+    import oracle
+    host = [gi.bf16_bits(t["q_sig"]), gi.bf16_bits(t["q_noise"]), gi.bf16_bits(t["k"]), gi.bf16_bits(t["v"]),
+            t["lam"].cpu().numpy(), gi.bf16_bits(t["gate"])]
+    cores = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.prefill(*host, w.seqlens, w.window, rows=rows, num_threads=cores)
+    dt = time.perf_counter() - t0
+    if rows is None:
+        return {"value": round(w.tokens / dt, 3), "unit": unit, "cores": cores, "kind": "oracle",
+                "sample": f"all {w.tokens} query rows (all heads) of {w.name}", "seconds": round(dt, 2)}
+    # visible keys of the sampled rows (one sequence: row r sees min(r + 1, window) keys)
+    rows = np.asarray(rows, dtype=np.int64)
+    keys = np.minimum(rows + 1, w.window) if w.window > 0 else rows + 1
+    sample_flops = float(keys.sum()) * 5 * w.num_kv_heads * FLOPS_PER_PAIR_HEAD
+    full_s = prefill_flops(w) / (sample_flops / dt)
+    return {"value": round(len(rows) / dt, 3), "unit": unit, "cores": cores, "kind": "oracle",
+            "sample": f"{len(rows)} sampled query rows (all heads) of {w.name}", "seconds": round(dt, 2),
+            "extrapolated_full_s": round(full_s, 1), "extrapolated": True}
+
+
+def oracle_decode_all(d, wd):
+    """The fp64 oracle on every sequence of a decode workload (same inputs)."""
+    import oracle
+    args = [gi.bf16_bits(d["q_sig"]), gi.bf16_bits(d["q_noise"]), gi.bf16_bits(d["k_cache"]),
+            gi.bf16_bits(d["v_cache"]), d["cu_seqlens_k"].cpu().numpy().astype(np.int64), d["lam"].cpu().numpy(),
+            gi.bf16_bits(d["gate"])]
+    cores = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.decode(*args, wd.window, num_threads=cores)
+    dt = time.perf_counter() - t0
+    return {"value": round(wd.batch / dt, 3), "unit": "query tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"all {wd.batch} sequences of {wd.name}", "seconds": round(dt, 3)}
 
 
 def cpu_baseline(t, w, target_s: float = 12.0):
@@ -485,7 +632,8 @@ PROFILE_CASES = ("prefill_T4096_full", "swa128_B2_T8192", "decode_B64_L1024_4096
 
 def run_profile_case(args):
     """A few launches of one workload, small enough for a full ncu capture
-    (ncu -k <kernel> -s <skip> -c <count> python bench.py --profile-case NAME)."""
+    (ncu --clock-control none -k <kernel> -s <skip> -c <count> python bench.py --profile-case NAME;
+    never omit --clock-control none: without it ncu locks the GPU clocks)."""
     import differential_latent_attention_b200 as gdla
     dev = torch.device("cuda", 0)
     name = args.profile_case

@@ -179,6 +179,13 @@ GDLA_API gdla_status_t gdla_attn_decode_noalloc(const void *q_sig, const void *q
  * records a nonzero code here instead of hanging the GPU. This call
  * synchronises the current device, returns the recorded code (0 = none) and,
  * if `clear` is nonzero, resets it. Returns -1 if the device cannot be read.
+ *
+ * A nonzero code means that at least one CTA of some call since the word was
+ * last cleared stopped early: output rows that CTA owned were NOT written
+ * (they keep whatever the buffer held before), so the outputs of every call
+ * enqueued since the last clear must be treated as invalid. Callers that
+ * cannot rule out such a stall (e.g. a GPU shared with other heavy work)
+ * should check this word before trusting a result.
  */
 GDLA_API int gdla_device_error(int clear);
 

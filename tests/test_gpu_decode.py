@@ -90,3 +90,49 @@ def test_decode_B64_H16(w):
 def test_largest_kv_head_count(window):
     """GDLA_MAX_KV_HEADS = 64 KV heads."""
     _check((300, 2000, 1), 64, window, 56)
+
+
+def test_64_splits_of_more_than_1024_keys():
+    """max_seqlen_k = 81,920: the split plan reaches its cap of 64 splits, each of
+    1,280 keys (more than the 1,024-key minimum), so the combine kernel merges a
+    full 64-entry split row; lengths fill the last split fully, partly, or leave
+    most splits empty."""
+    from differential_latent_attention_b200 import ops
+    assert ops.decode_workspace_bytes(4, 1, 81920, 0) == 4 * 1 * 64 * 5 * 130 * 4
+    _check((81920, 70001, 5, 40000), 1, 0, 59, max_len=81920)
+
+
+def _permute_groups(d, perm):
+    """The same decode problem with its KV groups reordered by perm (query, lambda,
+    gate and cache heads moved together)."""
+    perm = torch.as_tensor(perm, device="cuda")
+    sig = torch.stack([perm * 4 + i for i in range(4)], dim=1).reshape(-1)
+    return {"q_sig": d["q_sig"][:, sig].contiguous(), "q_noise": d["q_noise"][:, perm].contiguous(),
+            "k_cache": d["k_cache"][:, perm].contiguous(), "v_cache": d["v_cache"][:, perm].contiguous(),
+            "cu_seqlens_k": d["cu_seqlens_k"], "lam": d["lam"][:, sig].contiguous(),
+            "gate": d["gate"][:, sig].contiguous()}, sig
+
+
+@pytest.mark.parametrize("window", [0, 128])
+def test_group_permutation_equivariant_bitwise(window):
+    """Reordering the KV groups (with their signal and noise heads) reorders the
+    output the same way, bit for bit: groups are computed independently."""
+    d = gi.make_decode_inputs((3000, 77, 1500), 3, 64, device="cuda")
+    perm = [2, 0, 1]
+    a = gpu_decode(d, 3000, window)
+    dp, sig = _permute_groups(d, perm)
+    b = gpu_decode(dp, 3000, window)
+    torch.cuda.synchronize()
+    assert torch.equal(a[:, sig].view(torch.int16), b.view(torch.int16))
+
+
+def test_window_at_least_length_equals_full_bitwise():
+    """A window no shorter than every sequence sees exactly the full context: the
+    output is bit-identical to window 0 (both take the several-split path)."""
+    d = gi.make_decode_inputs((2500, 3000, 17), 2, 65, device="cuda")
+    a = gpu_decode(d, 3000, 0)
+    b = gpu_decode(d, 3000, 3000)
+    c = gpu_decode(d, 3000, 100000)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(a.view(torch.int16), c.view(torch.int16))

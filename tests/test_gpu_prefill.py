@@ -159,3 +159,42 @@ def test_windows_in_the_causal_configuration(window):
     """Windows over 256 run the one-tile configuration with window masks and key-tile
     skipping; the sequences are longer than the window, so both take effect."""
     check_prefill((1500, 700), 2, window, 21)
+
+
+def _permute_prefill_groups(t, perm):
+    perm = torch.as_tensor(perm, device="cuda")
+    sig = torch.stack([perm * 4 + i for i in range(4)], dim=1).reshape(-1)
+    return {"q_sig": t["q_sig"][:, sig].contiguous(), "q_noise": t["q_noise"][:, perm].contiguous(),
+            "k": t["k"][:, perm].contiguous(), "v": t["v"][:, perm].contiguous(),
+            "lam": t["lam"][:, sig].contiguous(), "gate": t["gate"][:, sig].contiguous()}, sig
+
+
+@pytest.mark.parametrize("window", [0, 128, 1000])
+def test_group_permutation_equivariant_bitwise(window):
+    """Reordering the KV groups (with their signal and noise query heads, lambda
+    and gate) reorders the output the same way, bit for bit."""
+    seqlens = (1300, 77, 300)
+    t = gi.make_prefill_inputs(seqlens, 3, 22, device="cuda")
+    a = gpu_prefill(t, seqlens, window)
+    tp, sig = _permute_prefill_groups(t, [1, 2, 0])
+    b = gpu_prefill(tp, seqlens, window)
+    torch.cuda.synchronize()
+    assert torch.equal(a[:, sig].view(torch.int16), b.view(torch.int16))
+
+
+def test_window_at_least_length_equals_full_bitwise():
+    """Windows no shorter than the sequence see the full causal context: bit-identical
+    outputs (one-tile configuration: window 4096 vs full causal; sliding
+    configuration: windows 255 and 256 over sequences of at most 200 tokens)."""
+    seqlens = (1000, 129, 1)
+    t = gi.make_prefill_inputs(seqlens, 2, 23, device="cuda")
+    a = gpu_prefill(t, seqlens, 0)
+    b = gpu_prefill(t, seqlens, 4096)
+    short = (200, 48, 1, 97)
+    ts = gi.make_prefill_inputs(short, 2, 24, device="cuda")
+    c = gpu_prefill(ts, short, 255)
+    d = gpu_prefill(ts, short, 256)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert torch.equal(c.view(torch.int16), d.view(torch.int16))
+    check_prefill(short, 2, 256, 24, t=ts)

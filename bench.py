@@ -66,6 +66,21 @@ def decode_bytes(lengths, hkv, window) -> float:
     return float(keys) * hkv * (192 + 128) * 2 + len(lengths) * per_query
 
 
+def latent_bytes(lengths, hkv, window) -> float:
+    """Decode over the latent cache: 1,152 B per visible key (one 576-wide bf16
+    row shared by every head), the absorbed queries, lambda, gate and output of
+    each sequence, and W^UV once."""
+    hs = 4 * hkv
+    keys = sum(min(int(l), window) if window > 0 else int(l) for l in lengths)
+    per_query = 2 * (5 * hkv * 576 + hs * 128 + hs * 128) + 4 * hs
+    return float(keys) * 576 * 2 + len(lengths) * per_query + hkv * 128 * 512 * 2
+
+
+def latent_flops(lengths, hkv, window) -> float:
+    keys = sum(min(int(l), window) if window > 0 else int(l) for l in lengths)
+    return float(keys) * 5 * hkv * (576 + 512) * 2 + len(lengths) * 5 * hkv * 128 * 512 * 2
+
+
 def decode_flops(lengths, hkv, window) -> float:
     keys = sum(min(int(l), window) if window > 0 else int(l) for l in lengths)
     return float(keys) * 5 * hkv * FLOPS_PER_PAIR_HEAD
@@ -529,7 +544,84 @@ def extra_workloads(gdla, dev, flush, args, world, rank, peaks):
             entry["cpu_baseline"] = oracle_decode_all(sets[0], wd)
         res.append(entry)
         del sets, ws
+    res.extend(latent_workloads(gdla, dev, flush, steps, world, rank, peaks, cpu))
     return res
+
+
+def latent_rotation_sets(wd, lengths, n_sets, shift, dev, rank):
+    """Like decode_rotation_sets, for the latent-cache decode."""
+    lengths = np.asarray(lengths, dtype=np.int64)
+    ext = lengths.copy()
+    ext[-1] += (n_sets - 1) * shift
+    base = gi.make_latent_decode_inputs(ext, wd.num_kv_heads, wd.seed + 1000 * rank, device=dev)
+    cu0 = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    sets = []
+    for r in range(n_sets):
+        small = gi.make_latent_decode_inputs(np.ones(len(lengths), dtype=np.int64), wd.num_kv_heads,
+                                             wd.seed + 1000 * rank + 7919 * (r + 1), device=dev)
+        sets.append({"q_abs_sig": small["q_abs_sig"], "q_abs_noise": small["q_abs_noise"], "lam": small["lam"],
+                     "gate": small["gate"], "w_uv": base["w_uv"], "ckv": base["ckv"],
+                     "cu_seqlens_k": torch.as_tensor((cu0 + r * shift).astype(np.int32), device=dev),
+                     "out": torch.empty((len(lengths), 4 * wd.num_kv_heads, 128), dtype=torch.bfloat16,
+                                        device=dev)})
+    return sets
+
+
+def latent_workloads(gdla, dev, flush, steps, world, rank, peaks, cpu):
+    """The 64-sequence decode batch over the compressed latent cache (1,152 B per
+    key instead of 10,240), full context (L2 flushed) and window 128 (rotating
+    input sets, flushed figure beside it)."""
+    res = []
+    hbm = peaks["hbm_gbs"]
+    for wd in (gi.LATENT_FULL, gi.LATENT_W128):
+        lengths = wd.kv_lengths()
+        ws = torch.empty(max(gdla.decode_latent_workspace_bytes(wd.batch, wd.num_kv_heads, 32768, wd.window), 1),
+                         dtype=torch.uint8, device=dev)
+        nbytes = latent_bytes(lengths, wd.num_kv_heads, wd.window)
+        flops = latent_flops(lengths, wd.num_kv_heads, wd.window)
+
+        def call(d):
+            gdla.attn_decode_latent(d["q_abs_sig"], d["q_abs_noise"], d["ckv"], d["cu_seqlens_k"], 32768,
+                                    d["w_uv"], d["lam"], d["gate"], wd.window, out=d["out"], workspace=ws)
+
+        n_sets = 1 if wd.window <= 0 else max(3, int(math.ceil(2 * L2_BYTES / nbytes)) + 1)
+        sets = latent_rotation_sets(wd, lengths, n_sets, max(wd.window, 0), dev, rank)
+        flushed = time_steps(lambda: call(sets[0]), steps, 3, flush, world)
+        ms_flushed = reduce_max(statistics.median(flushed), world, dev)
+        entry = {"workload": wd.name, "metric": "query tokens/s", "steps": steps, "stat": "median"}
+        if n_sets > 1:
+            rot = time_rotating([lambda d=d: call(d) for d in sets], steps, 3 * n_sets, world)
+            ms = reduce_max(statistics.median(rot), world, dev)
+            entry["l2"] = (f"{n_sets} rotating input sets ({n_sets * nbytes / 1e6:.0f} MB of visible cache rows "
+                           f"and per-query tensors, > 2x L2), no flush")
+            entry["flushed"] = {"ms": round(ms_flushed, 5), "roofline": hbm_roofline(nbytes, ms_flushed, hbm),
+                                "l2": "flushed (512 MiB write) before every timed step"}
+        else:
+            ms = ms_flushed
+            entry["l2"] = "flushed (512 MiB write) before every timed step"
+        entry.update({"value": wd.batch * world / (ms * 1e-3), "ms": round(ms, 5),
+                      "roofline": hbm_roofline(nbytes, ms, hbm),
+                      "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+                      "tensor_frac": round(flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)})
+        if cpu:
+            entry["cpu_baseline"] = oracle_latent_all(sets[0], wd)
+        res.append(entry)
+        del sets, ws
+    return res
+
+
+def oracle_latent_all(d, wd):
+    """The fp64 latent-cache decode oracle on every sequence (same inputs)."""
+    import oracle
+    args = [gi.bf16_bits(d["q_abs_sig"]), gi.bf16_bits(d["q_abs_noise"]), gi.bf16_bits(d["ckv"]),
+            d["cu_seqlens_k"].cpu().numpy().astype(np.int64), gi.bf16_bits(d["w_uv"]), d["lam"].cpu().numpy(),
+            gi.bf16_bits(d["gate"])]
+    cores = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.decode_latent(*args, wd.window, num_threads=cores)
+    dt = time.perf_counter() - t0
+    return {"value": round(wd.batch / dt, 3), "unit": "query tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"all {wd.batch} sequences of {wd.name}", "seconds": round(dt, 3)}
 
 
 def oracle_prefill_rows(t, w, rows, unit):
@@ -627,7 +719,8 @@ def run_reference(args):
     }), flush=True)
 
 
-PROFILE_CASES = ("prefill_T4096_full", "swa128_B2_T8192", "decode_B64_L1024_4096", "decode_B64_L1024_4096_w128")
+PROFILE_CASES = ("prefill_T4096_full", "swa128_B2_T8192", "decode_B64_L1024_4096", "decode_B64_L1024_4096_w128",
+                 "latent_decode_B64_L1024_4096", "latent_decode_B64_L1024_4096_w128")
 
 
 def run_profile_case(args):
@@ -637,7 +730,13 @@ def run_profile_case(args):
     import differential_latent_attention_b200 as gdla
     dev = torch.device("cuda", 0)
     name = args.profile_case
-    if name.startswith("decode"):
+    if name.startswith("latent"):
+        wd = gi.DecodeWorkload(name, 64, 16, 128 if name.endswith("w128") else 0, 4, 1024, 4096)
+        lengths = wd.kv_lengths()
+        d = gi.make_latent_decode_inputs(lengths, 16, wd.seed, device=dev)
+        fn = lambda: gdla.attn_decode_latent(d["q_abs_sig"], d["q_abs_noise"], d["ckv"], d["cu_seqlens_k"], 4096,
+                                             d["w_uv"], d["lam"], d["gate"], wd.window)
+    elif name.startswith("decode"):
         wd = gi.DecodeWorkload(name, 64, 16, 128 if name.endswith("w128") else 0, 4, 1024, 4096)
         lengths = wd.kv_lengths()
         d = gi.make_decode_inputs(lengths, 16, wd.seed, device=dev)

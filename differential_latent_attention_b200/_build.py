@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "libgdla.so")
 SOURCES = ["gdla_lib.cu", "gdla_api.cu", "gdla_prefill.cu", "gdla_decode.cu", "gdla_decode_noalloc.cu",
-           "gdla_selftest.cu", "gdla_internal.h", "gdla_ptx.cuh"]
+           "gdla_decode_latent.cu", "gdla_selftest.cu", "gdla_internal.h", "gdla_ptx.cuh"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

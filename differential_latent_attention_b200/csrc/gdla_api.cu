@@ -49,7 +49,44 @@ bool make_map(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D fp32 tensor [d1][d0] (d0 contiguous), unswizzled boxes.
+bool make_map_f32_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint32_t b0, uint32_t b1) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {d0, d1};
+    cuuint64_t strides[1] = {d0 * 4};
+    cuuint32_t box[2] = {b0, b1};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
+
+unsigned long long current_context_id() {
+    typedef CUresult (*GetCurrentFn)(CUcontext *);
+    typedef CUresult (*GetIdFn)(CUcontext, unsigned long long *);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    if (get_current == nullptr || get_id == nullptr) return 0;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    unsigned long long id = 0;
+    return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
 
 int device_sm_count(int dev) {
     static std::atomic<int> sms[kMaxCachedDevices];
@@ -156,7 +193,14 @@ gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *
     if (!make_map(&L.tm_qs, q_sig, 192, 4 * hkv, N, 64, 4, TQ) ||
         !make_map(&L.tm_qn, q_noise, 192, hkv, N, 64, 1, TQ) ||
         !make_map(&L.tm_k, k, 192, hkv, N, 64, 1, geo.key_tile) ||
-        !make_map(&L.tm_v, v, 128, hkv, N, 64, 1, geo.key_tile))
+        !make_map(&L.tm_v, v, 128, hkv, N, 64, 1, geo.v_box))
+        return GDLA_ERR_CUDA;
+    // The asynchronous epilogue (short windows) moves the gate logits and lambda
+    // of a 24-token tile's 4 signal heads in, and each warp's 6 output tokens out.
+    if (geo.async_epilogue &&
+        (!make_map(&L.tm_gate, gate_logits, 128, 4 * hkv, N, 64, 4, kPrefillTileTokens) ||
+         !make_map_f32_2d(&L.tm_lam, lambda, 4 * hkv, N, 4, kPrefillTileTokens) ||
+         !make_map(&L.tm_out, out, 128, 4 * hkv, N, 64, 4, TQ)))
         return GDLA_ERR_CUDA;
     L.lambda = lambda;
     L.gate = static_cast<const __nv_bfloat16 *>(gate_logits);
@@ -227,6 +271,44 @@ gdla_status_t gdla_attn_decode(const void *q_sig, const void *q_noise, const voi
     L.out = static_cast<__nv_bfloat16 *>(out);
     L.ws = static_cast<float *>(workspace);
     if (launch_decode(L, plan, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDLA_ERR_CUDA;
+    return GDLA_OK;
+}
+
+size_t gdla_decode_latent_workspace_bytes(int batch, int num_kv_heads, int max_seqlen_k, int window) {
+    if (batch < 1 || num_kv_heads < 1 || num_kv_heads > GDLA_LATENT_MAX_KV_HEADS || max_seqlen_k < 1) return 0;
+    return latent_workspace_bytes(make_latent_plan(batch, num_kv_heads, max_seqlen_k, window, 1));
+}
+
+gdla_status_t gdla_attn_decode_latent(const void *q_abs_sig, const void *q_abs_noise, const void *ckv,
+                                      const int32_t *cu_seqlens_k, int num_cache_rows, int max_seqlen_k,
+                                      const void *w_uv, const float *lambda, const void *gate_logits, void *out,
+                                      int batch, int num_kv_heads, int window, void *workspace,
+                                      size_t workspace_bytes, void *stream) {
+    if (batch < 1 || num_cache_rows < 1 || max_seqlen_k < 1) return GDLA_ERR_INVALID_ARG;
+    if (num_kv_heads < 1 || num_kv_heads > GDLA_LATENT_MAX_KV_HEADS) return GDLA_ERR_UNSUPPORTED;
+    if (!aligned16(q_abs_sig) || !aligned16(q_abs_noise) || !aligned16(ckv) || !aligned16(w_uv) ||
+        !aligned16(lambda) || !aligned16(gate_logits) || !aligned16(out) || cu_seqlens_k == nullptr ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u) != 0)
+        return GDLA_ERR_INVALID_ARG;
+    const LatentPlan plan = make_latent_plan(batch, num_kv_heads, max_seqlen_k, window, num_cache_rows);
+    const size_t need = latent_workspace_bytes(plan);
+    if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return GDLA_ERR_WORKSPACE;
+    LatentLaunch L{};
+    const int hkv = num_kv_heads;
+    // Q boxes: one sequence's 4H signal rows and H noise rows, 64 dims at a time;
+    // latent cache: 48 rows x 64 dims.
+    if (!make_map(&L.tm_qs, q_abs_sig, 576, 4 * hkv, static_cast<uint64_t>(batch), 64, 4 * hkv, 1) ||
+        !make_map(&L.tm_qn, q_abs_noise, 576, hkv, static_cast<uint64_t>(batch), 64, hkv, 1) ||
+        !make_map(&L.tm_c, ckv, 576, 1, static_cast<uint64_t>(num_cache_rows), 64, 1, 48))
+        return GDLA_ERR_CUDA;
+    L.cu_seqlens_k = cu_seqlens_k;
+    L.w_uv = static_cast<const __nv_bfloat16 *>(w_uv);
+    L.lambda = lambda;
+    L.gate = static_cast<const __nv_bfloat16 *>(gate_logits);
+    L.out = static_cast<__nv_bfloat16 *>(out);
+    L.ws = static_cast<float *>(workspace);
+    if (launch_decode_latent(L, plan, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDLA_ERR_CUDA;
     return GDLA_OK;
 }
 

@@ -31,6 +31,19 @@ namespace gdla {
 namespace dc {
 constexpr int DQK = 192, DV = 128, HEADS = 5;
 constexpr int STAGES = 2;
+// Per-stage auxiliary area. The producer writes the item's key range into
+// every stage it issues and, with an item's first stage, bulk-copies the
+// item's queries (and, when one split holds every key, its gate logits and
+// lambda) there, so the consumers never wait on global loads of their own.
+constexpr int Q_ROW = DQK * 2;                      // 384 bytes per query row
+constexpr int Q_ROW_STRIDE = Q_ROW + 16;            // padded: ldmatrix rows fall in distinct banks
+constexpr int AUX_DESC = 0;                         // int[4]: first cache row, k_begin, k_end, n_stages
+constexpr int AUX_LAM = 16;                         // fp32[4]
+constexpr int AUX_Q = 128;                          // bf16 [8 rows: 4 signal, noise, 3 zero][Q_ROW_STRIDE]
+constexpr int AUX_GATE = AUX_Q + 8 * Q_ROW_STRIDE;  // bf16 [4][128]
+constexpr int AUX_BYTES = AUX_GATE + 4 * DV * 2;
+constexpr uint32_t Q_TX = HEADS * Q_ROW;
+constexpr uint32_t EPI_TX = 4 * DV * 2 + 16;        // gate rows + lambda
 }  // namespace dc
 
 // Split-kernel configuration: each consumer warp takes 16 keys of a TK-key
@@ -42,13 +55,16 @@ struct DCfg {
     static constexpr int CTAS_PER_SM = CTAS_;
     static constexpr int NCT = CW_ * 32;           // consumer threads
     static constexpr int NUM_THREADS = NCT + 32;   // + the TMA producer warp
-    static constexpr int COLS = dc::DV / NCT;      // output columns per consumer thread (merge, epilogue)
+    // merge and epilogue: MT threads, COLS output columns each
+    static constexpr int MT = NCT < dc::DV ? NCT : dc::DV;
+    static constexpr int COLS = dc::DV / MT;
     static constexpr int K_CHUNK = TK * 128;       // one 64-dim swizzled chunk
     static constexpr int K_STAGE = 3 * K_CHUNK;
     static constexpr int V_STAGE = 2 * K_CHUNK;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + dc::STAGES * K_STAGE;
-    static constexpr int OFF_RED = OFF_V + dc::STAGES * V_STAGE;  // [warps][5 heads][128] fp32
+    static constexpr int OFF_AUX = OFF_V + dc::STAGES * V_STAGE;
+    static constexpr int OFF_RED = OFF_AUX + dc::STAGES * dc::AUX_BYTES;  // [warps][5 heads][128] fp32
     static constexpr int RED_BYTES = CW_ * dc::HEADS * dc::DV * 4;
     static constexpr int OFF_ML = OFF_RED + RED_BYTES;             // [warps][8 heads] m, l
     static constexpr int OFF_BAR = OFF_ML + 2 * CW_ * 8 * 4;
@@ -56,7 +72,9 @@ struct DCfg {
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
     static constexpr uint32_t STAGE_TX = K_STAGE + V_STAGE;
     static_assert(TK == 16 * CW_, "one 16-key MMA block per consumer warp");
-    static_assert(dc::DV % NCT == 0, "columns per consumer thread");
+    static_assert(dc::DV % MT == 0, "columns per merge thread");
+    static_assert(TK <= 256, "TMA box height");
+    static_assert(SMEM_BYTES * CTAS_ <= 232448, "shared memory per SM");
 };
 // Several splits (long caches): one item per CTA, 64-key stages, 4 consumer warps.
 using SplitCfg = DCfg<64, 4, 2>;
@@ -145,10 +163,11 @@ __device__ __forceinline__ DecodeItem decode_item(const int32_t *__restrict__ cu
 }
 
 // Persistent split kernel: every CTA loops over (split, group, sequence)
-// items; the producer's K/V stage ring runs on across items, so the next
-// item's keys stream in while the current one is computed. Consumers fetch
-// an item's Q fragments (and, for a single split, its gate values and lambda)
-// before waiting for its first stage.
+// items; the producer's stage ring runs on across items, so the next item's
+// keys stream in while the current one is computed. The producer alone reads
+// the sequence bounds and the item's queries, gate logits and lambda: it puts
+// the item's key range into every stage it issues (an empty item gets one
+// stage carrying only that) and copies the rest into the item's first stage.
 template <class C>
 __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS_PER_SM)
 gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -157,10 +176,10 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                          const __nv_bfloat16 *__restrict__ gate, __nv_bfloat16 *__restrict__ out,
                          float *__restrict__ ws, const DecodePlan plan) {
     using namespace dc;
-    constexpr int TK = C::TK, CONSUMER_WARPS = C::CONSUMER_WARPS, NCT = C::NCT, COLS = C::COLS;
+    constexpr int TK = C::TK, CONSUMER_WARPS = C::CONSUMER_WARPS, NCT = C::NCT, MT = C::MT, COLS = C::COLS;
     constexpr int K_CHUNK = C::K_CHUNK, K_STAGE = C::K_STAGE, V_STAGE = C::V_STAGE;
-    constexpr int OFF_K = C::OFF_K, OFF_V = C::OFF_V, OFF_RED = C::OFF_RED, OFF_ML = C::OFF_ML;
-    constexpr int OFF_BAR = C::OFF_BAR, OFF_MISC = C::OFF_MISC;
+    constexpr int OFF_K = C::OFF_K, OFF_V = C::OFF_V, OFF_AUX = C::OFF_AUX, OFF_RED = C::OFF_RED;
+    constexpr int OFF_ML = C::OFF_ML, OFF_BAR = C::OFF_BAR, OFF_MISC = C::OFF_MISC;
     constexpr uint32_t STAGE_TX = C::STAGE_TX;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -183,6 +202,12 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         *abort_flag = 0;
         fence_mbar_init();
     }
+    // Query rows 5..7 of every stage (the unused MMA columns) stay zero; the
+    // producer's copies never touch them.
+    for (int i = threadIdx.x; i < STAGES * 3 * (Q_ROW_STRIDE / 4); i += C::NUM_THREADS) {
+        const int st = i / (3 * (Q_ROW_STRIDE / 4)), r = i % (3 * (Q_ROW_STRIDE / 4));
+        reinterpret_cast<uint32_t *>(smem + OFF_AUX + st * AUX_BYTES + AUX_Q + 5 * Q_ROW_STRIDE)[r] = 0u;
+    }
     __syncthreads();
 
     if (warp == CONSUMER_WARPS) {
@@ -194,20 +219,39 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             bool ok = true;
             for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x) {
                 const DecodeItem d = decode_item(cu_seqlens_k, w, plan, TK);
-                for (int it = 0; it < d.n_stages; ++it, ++g) {
+                const int n_issue = max(1, d.n_stages);
+                for (int it = 0; it < n_issue; ++it, ++g) {
                     const int st = g % STAGES;
                     if (g >= STAGES &&
                         !mbar_wait(empty + st, ((g / STAGES) + 1) & 1, abort_flag, ERR_SITE_DECODE | 1)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(full + st, STAGE_TX);
+                    uint8_t *aux = smem + OFF_AUX + st * AUX_BYTES;
+                    *reinterpret_cast<int4 *>(aux + AUX_DESC) = make_int4(d.start, d.k_begin, d.k_end, d.n_stages);
+                    issued = g + 1;
+                    if (d.n_stages == 0) {
+                        mbar_arrive(full + st);  // the key range only (release orders the write above)
+                        continue;
+                    }
+                    const bool first = (it == 0);
+                    mbar_arrive_expect_tx(full + st, STAGE_TX + (first ? Q_TX + (ns == 1 ? EPI_TX : 0u) : 0u));
+                    if (first) {
+                        const size_t srow = static_cast<size_t>(d.b) * 4 * hkv + 4 * d.group;  // first signal head
+                        for (int i = 0; i < 4; ++i)
+                            bulk_load(aux + AUX_Q + i * Q_ROW_STRIDE, q_sig + (srow + i) * DQK, Q_ROW, full + st);
+                        bulk_load(aux + AUX_Q + 4 * Q_ROW_STRIDE,
+                                  q_noise + (static_cast<size_t>(d.b) * hkv + d.group) * DQK, Q_ROW, full + st);
+                        if (ns == 1) {
+                            bulk_load(aux + AUX_GATE, gate + srow * DV, 4 * DV * 2, full + st);
+                            bulk_load(aux + AUX_LAM, lambda + srow, 16, full + st);
+                        }
+                    }
                     const int row = d.start + d.k_begin + it * TK;
                     for (int c = 0; c < 3; ++c)
                         tma_load_3d(smem + OFF_K + st * K_STAGE + c * K_CHUNK, &tm_k, full + st, c * 64, d.group, row);
                     for (int c = 0; c < 2; ++c)
                         tma_load_3d(smem + OFF_V + st * V_STAGE + c * K_CHUNK, &tm_v, full + st, c * 64, d.group, row);
-                    issued = g + 1;
                 }
             }
             if (*abort_flag)
@@ -218,34 +262,54 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
         // ------------------------------- consumers --------------------------------
         const int g8 = lane >> 2, c = lane & 3;
         const int mi = lane >> 3, ri = lane & 7;
-        const int dcol = threadIdx.x;  // first of the COLS output columns (dcol + j * NCT) it owns
+        const int tid = threadIdx.x;     // merge/epilogue: threads < MT own columns tid + j * MT
+        const bool merger = tid < MT;
         const float c_log2 = 0.07216878364870322f * 1.4426950408889634f;  // log2(e) / sqrt(192)
         int g = 0;  // stages consumed by this CTA
         bool ok = true;
         for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x) {
-            const DecodeItem d = decode_item(cu_seqlens_k, w, plan, TK);
-            // Several splits: empty ones write nothing (the combine kernel skips them).
-            if (ns > 1 && d.n_stages == 0) continue;
-            // Q^T fragments (B operand): thread holds head g8, dims 16*ks + 2c(+1) and +8.
+            // The item's first stage carries its key range (and its queries).
+            int st = g % STAGES;
+            if (!__all_sync(0xffffffffu, mbar_wait(full + st, (g / STAGES) & 1, abort_flag, ERR_SITE_DECODE | 2))) {
+                ok = false;
+                break;
+            }
+            const uint8_t *aux = smem + OFF_AUX + st * AUX_BYTES;
+            const int4 desc = *reinterpret_cast<const int4 *>(aux + AUX_DESC);
+            const int k_begin = desc.y, k_end = desc.z, n_stages = desc.w;
+            const size_t orow0 = static_cast<size_t>(w / ns) * 4;  // (b * hkv + group) * 4: first signal row
+            if (n_stages == 0) {
+                // No visible key. Several splits: the combine kernel skips this
+                // split. One split: the sequence's output is zero.
+                if (ns == 1 && merger) {
+#pragma unroll
+                    for (int j = 0; j < COLS; ++j)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) out[(orow0 + i) * DV + tid + j * MT] = __float2bfloat16_rn(0.f);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty + st);
+                ++g;
+                continue;
+            }
+            // Q^T fragments (B operand): thread holds head g8, dims 16*ks + 2c(+1) and +8;
+            // one ldmatrix.x4 gives two 16-dim steps (rows 5..7 are the zero heads).
             uint32_t qf[DQK / 16][2];
             {
-                const __nv_bfloat16 *qrow = nullptr;
-                if (g8 < 4) qrow = q_sig + (static_cast<size_t>(d.b) * 4 * hkv + 4 * d.group + g8) * DQK;
-                else if (g8 == 4) qrow = q_noise + (static_cast<size_t>(d.b) * hkv + d.group) * DQK;
+                const uint32_t qb = smem_u32(aux + AUX_Q) + ri * Q_ROW_STRIDE + (mi & 1) * 16 + (mi >> 1) * 32;
 #pragma unroll
-                for (int ks = 0; ks < DQK / 16; ++ks) {
-                    qf[ks][0] = qrow ? __ldg(reinterpret_cast<const uint32_t *>(qrow + ks * 16 + 2 * c)) : 0u;
-                    qf[ks][1] = qrow ? __ldg(reinterpret_cast<const uint32_t *>(qrow + ks * 16 + 8 + 2 * c)) : 0u;
-                }
+                for (int ks2 = 0; ks2 < DQK / 32; ++ks2)
+                    ldsm_x4(qb + ks2 * 64, qf[2 * ks2][0], qf[2 * ks2][1], qf[2 * ks2 + 1][0], qf[2 * ks2 + 1][1]);
             }
-            const size_t orow0 = (static_cast<size_t>(d.b) * hkv + d.group) * 4;
             float lam_pre[4] = {0.f, 0.f, 0.f, 0.f}, g_pre[COLS][4] = {};
-            if (ns == 1) {
+            if (ns == 1 && merger) {
+                const float *lam_s = reinterpret_cast<const float *>(aux + AUX_LAM);
+                const __nv_bfloat16 *gate_s = reinterpret_cast<const __nv_bfloat16 *>(aux + AUX_GATE);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    lam_pre[i] = __ldg(lambda + orow0 + i);
+                    lam_pre[i] = lam_s[i];
 #pragma unroll
-                    for (int j = 0; j < COLS; ++j) g_pre[j][i] = __bfloat162float(gate[(orow0 + i) * DV + dcol + j * NCT]);
+                    for (int j = 0; j < COLS; ++j) g_pre[j][i] = __bfloat162float(gate_s[i * DV + tid + j * MT]);
                 }
             }
             float o[DV / 16][4];
@@ -254,9 +318,10 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             float m0 = -INFINITY, m1 = -INFINITY;  // running max (log2 units) of heads 2c, 2c+1
             float l0 = 0.f, l1 = 0.f;              // this thread's partial sums
 
-            for (int it = 0; it < d.n_stages; ++it, ++g) {
-                const int st = g % STAGES;
-                if (!__all_sync(0xffffffffu, mbar_wait(full + st, (g / STAGES) & 1, abort_flag, ERR_SITE_DECODE | 2))) {
+            for (int it = 0; it < n_stages; ++it, ++g) {
+                st = g % STAGES;
+                if (it > 0 &&
+                    !__all_sync(0xffffffffu, mbar_wait(full + st, (g / STAGES) & 1, abort_flag, ERR_SITE_DECODE | 2))) {
                     ok = false;
                     break;
                 }
@@ -276,9 +341,9 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                     }
                 }
                 // mask keys past the split end (and the cache rows of other sequences)
-                const int ubase = d.k_begin + it * TK + key0;
-                if (ubase + g8 >= d.k_end) { sacc[0] = -INFINITY; sacc[1] = -INFINITY; }
-                if (ubase + g8 + 8 >= d.k_end) { sacc[2] = -INFINITY; sacc[3] = -INFINITY; }
+                const int ubase = k_begin + it * TK + key0;
+                if (ubase + g8 >= k_end) { sacc[0] = -INFINITY; sacc[1] = -INFINITY; }
+                if (ubase + g8 + 8 >= k_end) { sacc[2] = -INFINITY; sacc[3] = -INFINITY; }
                 float mx0 = fmaxf(sacc[0], sacc[2]) * c_log2, mx1 = fmaxf(sacc[1], sacc[3]) * c_log2;
 #pragma unroll
                 for (int off = 4; off < 32; off <<= 1) {
@@ -321,7 +386,7 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 if (lane == 0) mbar_arrive(empty + st);
             }
             if (!ok) break;
-            // ---- merge the four warps: per head max, then rescaled sums ----
+            // ---- merge the warps: per head max, then rescaled sums ----
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) {
                 l0 += __shfl_xor_sync(0xffffffffu, l0, off);
@@ -356,56 +421,59 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
                 }
             }
             asm volatile("bar.sync 1, %0;" ::"n"(NCT) : "memory");
-            // each thread sums the warps for every head of its columns, fixed order
-            float hm[HEADS], hl[HEADS];
-#pragma unroll
-            for (int h = 0; h < HEADS; ++h) {
-                float M = -INFINITY;
-#pragma unroll
-                for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) M = fmaxf(M, ml[(w4 * 8 + h) * 2]);
-                float Ls = 0.f;
-#pragma unroll
-                for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) {
-                    const float mw = ml[(w4 * 8 + h) * 2];
-                    Ls += ml[(w4 * 8 + h) * 2 + 1] * ((mw == -INFINITY) ? 0.f : fast_exp2(mw - M));
-                }
-                hm[h] = M;
-                hl[h] = Ls;
-            }
-#pragma unroll
-            for (int j = 0; j < COLS; ++j) {
-                const int col = dcol + j * NCT;
-                float hsum[HEADS];
+            if (merger) {
+                // each merge thread sums the warps for every head of its columns, fixed order
+                float hm[HEADS], hl[HEADS];
 #pragma unroll
                 for (int h = 0; h < HEADS; ++h) {
-                    float Os = 0.f;
+                    float M = -INFINITY;
 #pragma unroll
-                    for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) Os += red[(w4 * HEADS + h) * DV + col];
-                    hsum[h] = Os;
-                }
-                if (ns == 1) {
-                    // one split holds every key: finish here (gate values fetched at the item start)
-                    float hv[HEADS];
+                    for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) M = fmaxf(M, ml[(w4 * 8 + h) * 2]);
+                    float Ls = 0.f;
 #pragma unroll
-                    for (int h = 0; h < HEADS; ++h) hv[h] = (hl[h] > 0.f) ? hsum[h] / hl[h] : 0.f;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float dd = hv[i] - lam_pre[i] * hv[4];
-                        out[(orow0 + i) * DV + col] = __float2bfloat16_rn(__fdividef(dd, 1.f + __expf(-g_pre[j][i])));
+                    for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) {
+                        const float mw = ml[(w4 * 8 + h) * 2];
+                        Ls += ml[(w4 * 8 + h) * 2 + 1] * ((mw == -INFINITY) ? 0.f : fast_exp2(mw - M));
                     }
-                } else {
-                    const size_t slot = (static_cast<size_t>(d.b) * hkv + d.group) * ns + d.split;
-                    float *wo = ws + slot * (HEADS * DV);
+                    hm[h] = M;
+                    hl[h] = Ls;
+                }
 #pragma unroll
-                    for (int h = 0; h < HEADS; ++h) wo[h * DV + col] = hsum[h];
-                    if (j == 0) {
-                        float *wml = ws + plan.ml_offset_floats + slot * (HEADS * 2);
+                for (int j = 0; j < COLS; ++j) {
+                    const int col = tid + j * MT;
+                    float hsum[HEADS];
 #pragma unroll
-                        for (int h = 0; h < HEADS; ++h)
-                            if (dcol == h) {
-                                wml[h * 2 + 0] = hm[h];
-                                wml[h * 2 + 1] = hl[h];
-                            }
+                    for (int h = 0; h < HEADS; ++h) {
+                        float Os = 0.f;
+#pragma unroll
+                        for (int w4 = 0; w4 < CONSUMER_WARPS; ++w4) Os += red[(w4 * HEADS + h) * DV + col];
+                        hsum[h] = Os;
+                    }
+                    if (ns == 1) {
+                        // one split holds every key: finish here (gate values staged with the item)
+                        float hv[HEADS];
+#pragma unroll
+                        for (int h = 0; h < HEADS; ++h) hv[h] = (hl[h] > 0.f) ? hsum[h] / hl[h] : 0.f;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float dd = hv[i] - lam_pre[i] * hv[4];
+                            out[(orow0 + i) * DV + col] =
+                                __float2bfloat16_rn(__fdividef(dd, 1.f + __expf(-g_pre[j][i])));
+                        }
+                    } else {
+                        const size_t slot = static_cast<size_t>(w);  // ((b * hkv + group) * ns + split)
+                        float *wo = ws + slot * (HEADS * DV);
+#pragma unroll
+                        for (int h = 0; h < HEADS; ++h) wo[h * DV + col] = hsum[h];
+                        if (j == 0 && tid < HEADS) {
+                            float *wml = ws + plan.ml_offset_floats + slot * (HEADS * 2);
+#pragma unroll
+                            for (int h = 0; h < HEADS; ++h)
+                                if (tid == h) {
+                                    wml[h * 2 + 0] = hm[h];
+                                    wml[h * 2 + 1] = hl[h];
+                                }
+                        }
                     }
                 }
             }
@@ -478,13 +546,13 @@ template <class C>
 static cudaError_t launch_split(const DecodeLaunch &L, const DecodePlan &plan, int dev, int num_sms,
                                 cudaStream_t stream) {
     // shared-memory opt-in once per device
-    static std::atomic<uint64_t> attr_set{0};
-    const uint64_t bit = (dev >= 0 && dev < kMaxCachedDevices) ? (1ull << dev) : 0ull;
-    if (!bit || !(attr_set.load(std::memory_order_relaxed) & bit)) {
+    static PerContextFlag attr_set;  // per device, for the context it was set in
+    const unsigned long long ctx = current_context_id();
+    if (!attr_set.is_set(dev, ctx)) {
         cudaError_t e = cudaFuncSetAttribute(gdla_decode_split_kernel<C>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set.fetch_or(bit, std::memory_order_relaxed);
+        attr_set.set(dev, current_context_id());
     }
     // One split per sequence (windows, short caches): few small items whose
     // latency chains dominate, so persistent CTAs (all resident) pipeline them.

@@ -15,7 +15,8 @@
 // In host code `g_decode_scratch` names a host-side stand-in, not a device
 // address: passing it to a kernel would fault (or, where the GPU can reach
 // host memory, silently use the wrong memory). The device address is looked
-// up with cudaGetSymbolAddress once per device, with that device current.
+// up with cudaGetSymbolAddress once per device and context, with that device
+// current.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -33,20 +34,25 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
 void *g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // context the cached address belongs to
 
-// Device address of g_decode_scratch on the current device; the first call for
-// a device performs the lookup (with that device current) and caches it.
+// Device address of g_decode_scratch on the current device. The first call in
+// a context performs the lookup (with that device current) and caches it for
+// that context; after a device reset the module is loaded afresh in a new
+// context, so the address is looked up again rather than reused.
 cudaError_t static_scratch_address(void **addr) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (g_scratch_addr[dev] == nullptr) {
+    unsigned long long ctx = current_context_id();
+    if (ctx == 0 || g_scratch_addr[dev] == nullptr || g_scratch_ctx[dev] != ctx) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_decode_scratch);
         if (e != cudaSuccess) return e;
         g_scratch_addr[dev] = p;
+        g_scratch_ctx[dev] = current_context_id();  // the lookup made the context current if it was not
     }
     *addr = g_scratch_addr[dev];
     return cudaSuccess;

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace gdla {
 
 // Prefill: one MMA tile = 24 tokens x 5 heads = 120 of the 128 MMA rows. The
@@ -14,8 +16,10 @@ constexpr int kPrefillTileTokens = 24;
 constexpr int kPrefillSlidingMaxWindow = 256;  // windows up to this use the sliding configuration
 
 struct PrefillGeometry {
-    int cta_tokens;  // tokens per CTA (a multiple of kPrefillTileTokens)
-    int key_tile;    // keys per K/V tile
+    int cta_tokens;       // tokens per CTA (a multiple of kPrefillTileTokens)
+    int key_tile;         // keys per K/V tile
+    int v_box;            // keys per V TMA box
+    bool async_epilogue;  // gate/lambda/output tensor maps are used
 };
 PrefillGeometry prefill_geometry(int window);
 constexpr int kPlanMaxSeqs = 256;    // sequences per launch (more are split across launches)
@@ -44,6 +48,7 @@ using PrefillPlanSmall = PrefillPlanT<768, 32>;
 
 struct PrefillLaunch {
     CUtensorMap tm_qs, tm_qn, tm_k, tm_v;
+    CUtensorMap tm_gate, tm_lam, tm_out;  // used by the asynchronous epilogue (short windows)
     const float *lambda;
     const __nv_bfloat16 *gate;
     __nv_bfloat16 *out;
@@ -54,6 +59,25 @@ cudaError_t launch_prefill(const PrefillLaunch &launch, const PrefillPlan &plan,
 // SM count of a device, queried once per device and cached (0 on failure).
 constexpr int kMaxCachedDevices = 64;
 int device_sm_count(int dev);
+
+// Identifier of the CUDA context current on the calling thread (0 if none is
+// current or it cannot be read). Tearing the primary context down (a device
+// reset) and re-creating it gives a new identifier, so host caches of facts
+// that belong to a context (kernel attribute opt-ins, symbol addresses) key
+// on it and are refreshed after a reset.
+unsigned long long current_context_id();
+
+// One flag per device, valid for one context: set() records the context it was
+// set in, is_set() holds only while that context is still the current one.
+struct PerContextFlag {
+    std::atomic<unsigned long long> ctx[kMaxCachedDevices];
+    bool is_set(int dev, unsigned long long id) const {
+        return id != 0 && dev >= 0 && dev < kMaxCachedDevices && ctx[dev].load(std::memory_order_relaxed) == id;
+    }
+    void set(int dev, unsigned long long id) {
+        if (id != 0 && dev >= 0 && dev < kMaxCachedDevices) ctx[dev].store(id, std::memory_order_relaxed);
+    }
+};
 
 // Decode: split-KV.
 constexpr int kDecodeMaxSplits = 64;
@@ -82,6 +106,35 @@ struct DecodeLaunch {
 
 cudaError_t launch_decode(const DecodeLaunch &launch, const DecodePlan &plan, cudaStream_t stream);
 int decode_smem_bytes();
+
+// Decode over the latent cache: split-KV, then a combine with the W^UV up-projection.
+constexpr int kLatentMaxSplits = 32;
+constexpr int kLatentMinSplitKeys = 2048;
+
+struct LatentPlan {
+    int batch;
+    int hkv;
+    int window;
+    int max_seqlen_k;
+    int num_cache_rows;
+    int num_splits;
+    int split_keys;              // keys per split (multiple of the 48-key stage)
+    long long ml_offset_floats;  // start of the (m, l) area in the workspace, in floats
+};
+
+struct LatentLaunch {
+    CUtensorMap tm_qs, tm_qn, tm_c;
+    const int32_t *cu_seqlens_k;
+    const __nv_bfloat16 *w_uv;
+    const float *lambda;
+    const __nv_bfloat16 *gate;
+    __nv_bfloat16 *out;
+    float *ws;
+};
+
+LatentPlan make_latent_plan(int batch, int hkv, int max_seqlen_k, int window, int num_cache_rows);
+size_t latent_workspace_bytes(const LatentPlan &plan);
+cudaError_t launch_decode_latent(const LatentLaunch &launch, const LatentPlan &plan, cudaStream_t stream);
 
 // Host-side decode split plan (shared by the workspace query and the launch).
 DecodePlan make_decode_plan(int batch, int hkv, int max_seqlen_k, int window, int num_cache_rows);

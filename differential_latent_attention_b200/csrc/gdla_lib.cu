@@ -4,4 +4,5 @@
 #include "gdla_prefill.cu"
 #include "gdla_decode.cu"
 #include "gdla_decode_noalloc.cu"
+#include "gdla_decode_latent.cu"
 #include "gdla_selftest.cu"

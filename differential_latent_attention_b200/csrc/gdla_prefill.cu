@@ -84,11 +84,26 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 constexpr int kPolyEvery = 4;              // one exponential pair in 4 on the FMA pipe
 
-template <int TILES_, int BN_, int STAGES_>
+// Gate / output staging of the asynchronous epilogue, per q tile: the gate
+// logits of its 24 tokens x 4 signal heads as two 128-byte-swizzled boxes
+// (dims 0..63, 64..127) of [token][head][64] bf16, 12 KB each; the output is
+// written over them in place and stored from there by TMA, one 3 KB box
+// (6 tokens) per warp and half.
+constexpr int G_HALF = TOK * 4 * 128;      // 12 KB
+constexpr int G_TILE = 2 * G_HALF;         // 24 KB
+constexpr int G_WARP_BOX = 6 * 4 * 128;    // 3 KB: one warp's tokens in one half
+constexpr int LAM_TILE = TOK * 4 * 4;      // 384 B: [token][head] fp32
+constexpr uint32_t G_TX = G_TILE + LAM_TILE;
+
+template <int TILES_, int BN_, int STAGES_, bool ASYNC_EPI_>
 struct Cfg {
     static constexpr int TILES = TILES_;
     static constexpr int BN = BN_;          // keys per KV tile
     static constexpr int STAGES = STAGES_;
+    static constexpr int V_BOX = BN;        // keys per V TMA box
+    // Asynchronous epilogue: gate and lambda arrive in shared memory by TMA
+    // during the item, the output leaves by TMA store.
+    static constexpr bool ASYNC_EPI = ASYNC_EPI_;
     static constexpr int CTA_TOK = TILES * TOK;
     static constexpr int KV_CHUNK = BN * 128;            // one 64-dim swizzled chunk
     static constexpr int K_STAGE = KCHUNKS * KV_CHUNK;
@@ -96,7 +111,9 @@ struct Cfg {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + TILES * Q_TILE;
     static constexpr int OFF_V = OFF_K + STAGES * K_STAGE;
-    static constexpr int OFF_BAR = OFF_V + STAGES * V_STAGE;
+    static constexpr int OFF_G = OFF_V + STAGES * V_STAGE;  // 1024-byte aligned (swizzled boxes)
+    static constexpr int OFF_LAM = OFF_G + (ASYNC_EPI ? TILES * G_TILE : 0);
+    static constexpr int OFF_BAR = OFF_LAM + (ASYNC_EPI ? TILES * LAM_TILE : 0);
     static constexpr int NUM_BARS = 32;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;  // + alignment slack
@@ -117,8 +134,8 @@ struct Cfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(BN == 64 || BN == 128, "key tile");
 };
-using CausalCfg = Cfg<1, 128, 2>;
-using SlidingCfg = Cfg<2, 64, 3>;
+using CausalCfg = Cfg<1, 128, 2, false>;
+using SlidingCfg = Cfg<2, 64, 2, true>;
 
 // ------------------------------- epilogue ----------------------------------
 // Per warp: the 24 signal rows of its 6 tokens. gate/out rows are 256 bytes;
@@ -172,14 +189,54 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&o)[32], float inv_l, 
         }
     }
 }
+// Asynchronous-epilogue form of epi_chunk: this lane's gate columns
+// 32ch..32ch+31 come from its 128-byte row of the swizzled staging box
+// (`row_addr` = the row's shared address, `key` = row & 7 selects the
+// swizzle); the bf16 result goes back over them (to_smem) or, for a warp
+// whose tokens are not all inside the sequence, straight to `dst` (to_global).
+__device__ __forceinline__ void epi_chunk_staged(const uint32_t (&o)[32], float inv_l, float lam, int hsrc, bool sig,
+                                                 uint32_t row_addr, int key, int ch, bool to_smem, bool to_global,
+                                                 __nv_bfloat16 *__restrict__ dst) {
+    uint32_t g[16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (sig) {
+            lds128(row_addr + ((((ch & 1) * 4 + i) ^ key) << 4), g + 4 * i);
+        } else {
+            g[4 * i] = g[4 * i + 1] = g[4 * i + 2] = g[4 * i + 3] = 0u;
+        }
+    }
+    uint32_t res[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float h0 = __uint_as_float(o[2 * i]) * inv_l;
+        const float h1 = __uint_as_float(o[2 * i + 1]) * inv_l;
+        const float n0 = __shfl_sync(0xffffffffu, h0, hsrc);  // H_N of this row's token
+        const float n1 = __shfl_sync(0xffffffffu, h1, hsrc);
+        const float2 g2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&g[i]));
+        res[i] = pack_bf16x2(fmaf(-lam, n0, h0) * fast_sigmoid(g2.x), fmaf(-lam, n1, h1) * fast_sigmoid(g2.y));
+    }
+    if (sig && to_smem) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sts128(row_addr + ((((ch & 1) * 4 + i) ^ key) << 4), res + 4 * i);
+    }
+    if (to_global) {
+        uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d[i] = make_uint4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
+    }
+}
+
 }  // namespace pf
 
 template <class C, class Plan>
 __global__ void __launch_bounds__(C::NUM_THREADS, 1)
 gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_qn,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                    const float *__restrict__ lambda, const __nv_bfloat16 *__restrict__ gate,
-                    __nv_bfloat16 *__restrict__ out, const __grid_constant__ Plan plan) {
+                    const __grid_constant__ CUtensorMap tm_gate, const __grid_constant__ CUtensorMap tm_lam,
+                    const __grid_constant__ CUtensorMap tm_out, const float *__restrict__ lambda,
+                    const __nv_bfloat16 *__restrict__ gate, __nv_bfloat16 *__restrict__ out,
+                    const __grid_constant__ Plan plan) {
     using namespace pf;
     constexpr int TILES = C::TILES, BN = C::BN, STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -195,6 +252,8 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
     uint64_t *p_full = bars + 20;   // [tile * 2 + buffer]
     uint64_t *o_done = bars + 24;   // [tile]: one phase per PV product of the tile
     uint64_t *o_final = bars + 26;  // [tile]: one phase per item, its last PV product is done
+    uint64_t *g_full = bars + 28;   // [tile]: one phase per item, its gate and lambda landed (async epilogue)
+    uint64_t *g_empty = bars + 30;  // [tile]: one phase per item, its output left the staging buffer
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -231,6 +290,8 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
             mbar_init(q_empty + i, 1);
             mbar_init(o_done + i, 1);
             mbar_init(o_final + i, 1);
+            mbar_init(g_full + i, 1);
+            mbar_init(g_empty + i, 4);
             for (int b = 0; b < 2; ++b) {
                 mbar_init(s_full + 2 * i + b, 1);
                 mbar_init(p_full + 2 * i + b, 128);
@@ -272,7 +333,12 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
             tma_prefetch_desc(&tm_qn);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
+            if constexpr (C::ASYNC_EPI) {
+                tma_prefetch_desc(&tm_gate);
+                tma_prefetch_desc(&tm_lam);
+            }
             int kv = 0, issued_kv = 0;  // K/V tiles issued by this CTA (ring position)
+            int gate_items = 0;         // items whose gate/lambda loads were issued
             int n_item = 0;
             bool ok = true;
             for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
@@ -292,6 +358,28 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                             tma_load_3d(qc + (32 * q + 24) * 128, &tm_qn, q_full + x, c * 64, it.group, row0 + 6 * q);
                         }
                     }
+                }
+                // Async epilogue: each q tile's gate logits and lambda, issued once the
+                // item's first K/V tiles are on their way (the staging buffer is free
+                // once the previous item's output store has read it).
+                auto issue_gate = [&]() {
+                    for (int x = 0; x < TILES; ++x) {
+                        if (n_item > 0 && !mbar_wait(g_empty + x, (n_item - 1) & 1, abort_flag, ERR_SITE_PREFILL | 11))
+                            return false;
+                        mbar_arrive_expect_tx(g_full + x, G_TX);
+                        const int row0 = it.s0 + it.t0 + x * TOK;
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_3d(smem + C::OFF_G + x * G_TILE + h * G_HALF, &tm_gate, g_full + x, h * 64,
+                                        4 * it.group, row0);
+                        tma_load_2d(smem + C::OFF_LAM + x * LAM_TILE, &tm_lam, g_full + x, 4 * it.group, row0);
+                    }
+                    gate_items = n_item + 1;
+                    return true;
+                };
+                const int gate_after = min(1, it.n_tiles[TILES - 1] - 1);  // K/V tile after which to issue
+                if (C::ASYNC_EPI && gate_after < 0 && !issue_gate()) {
+                    ok = false;
+                    break;
                 }
                 for (int k = 0; ok && k < it.n_tiles[TILES - 1]; ++k, ++kv) {
                     const int st = kv % STAGES;
@@ -314,6 +402,10 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                         tma_load_3d(smem + C::OFF_V + st * C::V_STAGE + c * C::KV_CHUNK, &tm_v, v_full + st, c * 64,
                                     it.group, row);
                     issued_kv = kv + 1;
+                    if (C::ASYNC_EPI && k == gate_after && !issue_gate()) {
+                        ok = false;
+                        break;
+                    }
                 }
             }
             if (*abort_flag) {
@@ -324,6 +416,8 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                     mbar_wait_cycles(v_full + k % STAGES, (k / STAGES) & 1, 1ll << 22);
                 }
                 for (int x = 0; x < TILES; ++x) mbar_wait_cycles(q_full + x, (n_item & 1) ^ 1, 1ll << 22);
+                if (C::ASYNC_EPI && gate_items > 0)
+                    for (int x = 0; x < TILES; ++x) mbar_wait_cycles(g_full + x, (gate_items - 1) & 1, 1ll << 22);
             }
         }
     } else if (warp == C::MMA_WARP) {
@@ -501,12 +595,12 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                     resc = true;
                 }
                 const float mb = (m_run == -INFINITY) ? 0.f : m_run;
-                // p = exp2(s * log2(e)/sqrt(192) - m): scaling and row sums in packed
-                // fp32 pairs; one pair in kPolyEvery through the FMA-pipe polynomial,
-                // the others through MUFU ex2, so both pipes share the work.
                 const uint64_t scale2 = f2_pack(c_log2, c_log2);
                 const uint64_t neg_m2 = f2_pack(-mb, -mb);
                 uint64_t lsum_a = f2_pack(0.f, 0.f), lsum_b = f2_pack(0.f, 0.f);
+                // p = exp2(s * log2(e)/sqrt(192) - m): scaling and row sums in packed
+                // fp32 pairs; one pair in kPolyEvery through the FMA-pipe polynomial,
+                // the others through MUFU ex2, so both pipes share the work.
 #pragma unroll
                 for (int h = 0; h < BN / 64; ++h) {
                     uint32_t pk[32];
@@ -562,25 +656,65 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
             pv += nt;
 
             // ----------------------------- epilogue ------------------------------
-            // Signal rows fetch their gate row and lambda before waiting for the last PV.
             const bool valid = is_sig && (t < it.L);
             const size_t row = static_cast<size_t>(it.s0 + t) * hs + 4 * it.group + (lane & 3);
-            uint32_t gw[DV / 32][16];
+            if constexpr (C::ASYNC_EPI) {
+                // Gate and lambda were staged in shared memory during the item; the
+                // output replaces the gate in place and leaves by one TMA store per
+                // warp and half, or (a warp with tokens past the sequence end)
+                // by direct stores of its valid rows.
+                const bool warp_full = (tx0 + 6 * wq + 5) < it.L;
+                bool ok_w = mbar_wait(g_full + x, n_item & 1, abort_flag, ERR_SITE_PREFILL | 12);
+                ok_w = ok_w && mbar_wait(o_final + x, n_item & 1, abort_flag, ERR_SITE_PREFILL | 9);
+                if (!__all_sync(0xffffffffu, ok_w)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+                const float lam = is_sig ? reinterpret_cast<const float *>(smem + C::OFF_LAM + x * LAM_TILE)[24 * wq + lane]
+                                         : 0.f;
+                const uint32_t g_base = smem_u32(smem + C::OFF_G + x * G_TILE) + (24 * wq + lane) * 128;
 #pragma unroll
-            for (int ch = 0; ch < DV / 32; ++ch) epi_fetch_gate(valid, row, gate, wide, ch, gw[ch]);
-            const float lam = valid ? __ldg(lambda + row) : 0.f;
-            // o_final completes once per item, after this tile's last PV product.
-            if (!__all_sync(0xffffffffu, mbar_wait(o_final + x, n_item & 1, abort_flag, ERR_SITE_PREFILL | 9))) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+                for (int ch = 0; ch < DV / 32; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + ch * 32, o);
+                    epi_chunk_staged(o, inv_l, lam, hsrc, is_sig, g_base + (ch >> 1) * G_HALF, lane & 7, ch, warp_full,
+                                     valid && !warp_full, out + row * DV + ch * 32);
+                }
+                if (warp_full) {
+                    fence_proxy_async_smem();  // the generic writes above, before the TMA store reads them
+                    __syncwarp();
+                    if (lane == 0) {
+                        const int row0_w = it.s0 + tx0 + 6 * wq;
+                        for (int h = 0; h < 2; ++h)
+                            tma_store_3d(&tm_out, smem + C::OFF_G + x * G_TILE + h * G_HALF + wq * G_WARP_BOX, h * 64,
+                                         4 * it.group, row0_w);
+                        bulk_commit_group();
+                        bulk_wait_group_read0();  // the staging buffer may be refilled
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(g_empty + x);
+            } else {
+                // Signal rows fetch their gate row and lambda before waiting for the last PV.
+                uint32_t gw[DV / 32][16];
 #pragma unroll
-            for (int ch = 0; ch < DV / 32; ++ch) {
-                uint32_t o[32];
-                tmem_ld32(o_addr + ch * 32, o);
-                epi_chunk(o, inv_l, lam, gw[ch], hsrc, valid, wide, out + row * DV + ch * 32);
+                for (int ch = 0; ch < DV / 32; ++ch) epi_fetch_gate(valid, row, gate, wide, ch, gw[ch]);
+                const float lam = valid ? __ldg(lambda + row) : 0.f;
+                // o_final completes once per item, after this tile's last PV product.
+                if (!__all_sync(0xffffffffu, mbar_wait(o_final + x, n_item & 1, abort_flag, ERR_SITE_PREFILL | 9))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+#pragma unroll
+                for (int ch = 0; ch < DV / 32; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + ch * 32, o);
+                    epi_chunk(o, inv_l, lam, gw[ch], hsrc, valid, wide, out + row * DV + ch * 32);
+                }
             }
             // every lane's TMEM reads of O are complete before the next item's PV
             // products may overwrite it (they wait for this warpgroup's p_full).
@@ -588,6 +722,7 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         }
     }
 
+    if (C::ASYNC_EPI && warp < C::PRODUCER_WARP && lane == 0) bulk_wait_group0();  // output stores complete
     tc_fence_before();
     __syncthreads();
     if (warp == C::MMA_WARP) {
@@ -599,28 +734,32 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
 // ------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------
+// Full causal and windows over kPrefillSlidingMaxWindow.
+using LongCfg = pf::CausalCfg;
+
 PrefillGeometry prefill_geometry(int window) {
     // Short windows: 48-token items over 64-key tiles; otherwise 24-token items over 128-key tiles.
-    if (window > 0 && window <= kPrefillSlidingMaxWindow) return {pf::SlidingCfg::CTA_TOK, pf::SlidingCfg::BN};
-    return {pf::CausalCfg::CTA_TOK, pf::CausalCfg::BN};
+    if (window > 0 && window <= kPrefillSlidingMaxWindow)
+        return {pf::SlidingCfg::CTA_TOK, pf::SlidingCfg::BN, pf::SlidingCfg::V_BOX, pf::SlidingCfg::ASYNC_EPI};
+    return {LongCfg::CTA_TOK, LongCfg::BN, LongCfg::V_BOX, LongCfg::ASYNC_EPI};
 }
 
 // Each kernel instantiation opts in to its shared memory once per device (a
 // driver call that need not be repeated on every launch).
 template <class C, class Plan>
 static cudaError_t launch_cfg(const PrefillLaunch &L, const Plan &plan, int dev, int num_sms, cudaStream_t stream) {
-    static std::atomic<uint64_t> attr_set{0};  // bit per device
-    const uint64_t bit = (dev >= 0 && dev < kMaxCachedDevices) ? (1ull << dev) : 0ull;
-    if (!bit || !(attr_set.load(std::memory_order_relaxed) & bit)) {
+    static PerContextFlag attr_set;  // per device, for the context it was set in
+    const unsigned long long ctx = current_context_id();
+    if (!attr_set.is_set(dev, ctx)) {
         cudaError_t e = cudaFuncSetAttribute(gdla_prefill_kernel<C, Plan>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set.fetch_or(bit, std::memory_order_relaxed);
+        attr_set.set(dev, current_context_id());
     }
     const long long work = static_cast<long long>(plan.n_items) * plan.hkv;
     const unsigned grid = static_cast<unsigned>(work < num_sms ? work : num_sms);
-    gdla_prefill_kernel<C, Plan><<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(L.tm_qs, L.tm_qn, L.tm_k, L.tm_v,
-                                                                                L.lambda, L.gate, L.out, plan);
+    gdla_prefill_kernel<C, Plan><<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(
+        L.tm_qs, L.tm_qn, L.tm_k, L.tm_v, L.tm_gate, L.tm_lam, L.tm_out, L.lambda, L.gate, L.out, plan);
     return cudaPeekAtLastError();
 }
 
@@ -659,7 +798,7 @@ cudaError_t launch_prefill(const PrefillLaunch &L, const PrefillPlan &plan, cuda
     if (num_sms <= 0) return cudaErrorInvalidDevice;
     if (plan.window > 0 && plan.window <= kPrefillSlidingMaxWindow)
         return launch_sized<pf::SlidingCfg>(L, plan, dev, num_sms, stream);
-    return launch_sized<pf::CausalCfg>(L, plan, dev, num_sms, stream);
+    return launch_sized<LongCfg>(L, plan, dev, num_sms, stream);
 }
 
 }  // namespace gdla

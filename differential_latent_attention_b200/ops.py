@@ -21,7 +21,11 @@ MAX_KV_HEADS = 64
 STATUS = {0: "GDLA_OK", 1: "GDLA_ERR_INVALID_ARG", 2: "GDLA_ERR_UNSUPPORTED", 3: "GDLA_ERR_WORKSPACE",
           4: "GDLA_ERR_CUDA"}
 EXPORTED = ("gdla_attn_fwd", "gdla_decode_workspace_bytes", "gdla_attn_decode", "gdla_attn_decode_noalloc",
-            "gdla_device_error", "gdla_selftest_wait_timeout", "gdla_status_string", "gdla_version")
+            "gdla_decode_latent_workspace_bytes", "gdla_attn_decode_latent", "gdla_device_error",
+            "gdla_selftest_wait_timeout", "gdla_status_string", "gdla_version")
+DC, DR = 512, 64
+DL = DC + DR
+LATENT_MAX_KV_HEADS = 16
 SELFTEST_SITE = 0x30001  # GDLA_SELFTEST_SITE
 
 _lib = None
@@ -56,6 +60,10 @@ def library():
             lib.gdla_attn_decode.restype = i
             lib.gdla_attn_decode_noalloc.argtypes = [p, p, p, p, p, i, i, p, p, p, i, i, i, p]
             lib.gdla_attn_decode_noalloc.restype = i
+            lib.gdla_decode_latent_workspace_bytes.argtypes = [i, i, i, i]
+            lib.gdla_decode_latent_workspace_bytes.restype = sz
+            lib.gdla_attn_decode_latent.argtypes = [p, p, p, p, i, i, p, p, p, p, i, i, i, p, sz, p]
+            lib.gdla_attn_decode_latent.restype = i
             lib.gdla_device_error.argtypes = [i]
             lib.gdla_device_error.restype = i
             lib.gdla_selftest_wait_timeout.argtypes = [p]
@@ -161,6 +169,48 @@ def attn_decode(q_sig, q_noise, k_cache, v_cache, cu_seqlens_k, max_seqlen_k, la
                                     int(window), _ptr(workspace), ws_bytes, _stream(stream))
     if st != 0:
         raise GDLAError(st, "gdla_attn_decode")
+    return out
+
+
+def decode_latent_workspace_bytes(batch, num_kv_heads, max_seqlen_k, window=0):
+    return int(library().gdla_decode_latent_workspace_bytes(int(batch), int(num_kv_heads), int(max_seqlen_k),
+                                                            int(window)))
+
+
+def attn_decode_latent(q_abs_sig, q_abs_noise, ckv, cu_seqlens_k, max_seqlen_k, w_uv, lam, gate, window=0,
+                       out=None, workspace=None, stream=None):
+    """GDLA decode over the compressed KV cache (calls ``gdla_attn_decode_latent``).
+
+    q_abs_sig [B, 4H, 576] and q_abs_noise [B, H, 576] bf16 (queries with W^UK
+    absorbed), ckv [Nk, 576] bf16 ([c | k_rope] per token, sequences packed as
+    given by the int32 CUDA tensor cu_seqlens_k [B+1]), w_uv [H, 128, 512] bf16,
+    lam [B, 4H] fp32, gate [B, 4H, 128] bf16. ``workspace`` (uint8 CUDA tensor)
+    is allocated here when not given.
+    """
+    b = q_abs_sig.shape[0]
+    hkv = q_abs_noise.shape[1] if q_abs_noise.dim() == 3 else -1
+    hs = GROUP * hkv
+    nk = ckv.shape[0]
+    _check(q_abs_sig, "q_abs_sig", torch.bfloat16, (b, hs, DL))
+    _check(q_abs_noise, "q_abs_noise", torch.bfloat16, (b, hkv, DL))
+    _check(ckv, "ckv", torch.bfloat16, (nk, DL))
+    _check(cu_seqlens_k, "cu_seqlens_k", torch.int32, (b + 1,))
+    _check(w_uv, "w_uv", torch.bfloat16, (hkv, DV, DC))
+    _check(lam, "lam", torch.float32, (b, hs))
+    _check(gate, "gate", torch.bfloat16, (b, hs, DV))
+    if out is None:
+        out = torch.empty((b, hs, DV), dtype=torch.bfloat16, device=q_abs_sig.device)
+    _check(out, "out", torch.bfloat16, (b, hs, DV))
+    need = decode_latent_workspace_bytes(b, hkv, max_seqlen_k, window)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q_abs_sig.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = library().gdla_attn_decode_latent(_ptr(q_abs_sig), _ptr(q_abs_noise), _ptr(ckv), _ptr(cu_seqlens_k),
+                                           int(nk), int(max_seqlen_k), _ptr(w_uv), _ptr(lam), _ptr(gate),
+                                           _ptr(out), int(b), hkv, int(window), _ptr(workspace), ws_bytes,
+                                           _stream(stream))
+    if st != 0:
+        raise GDLAError(st, "gdla_attn_decode_latent")
     return out
 
 

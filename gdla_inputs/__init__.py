@@ -6,7 +6,9 @@ arithmetic: it only draws random tensors of the right shapes, dtypes and
 layouts, and describes the workloads.
 
 Distributions (the workload recipe): q_sig, q_noise, k, v and the gate logits
-are N(0, 1) drawn in fp32 and rounded to nearest-even bf16; lambda is
+are N(0, 1) drawn in fp32 and rounded to nearest-even bf16 (for the latent-cache
+decode likewise the absorbed queries and the cache rows [c | k_rope], and
+W^UV ~ N(0, 1/512), so that an up-projected value row has unit scale); lambda is
 U(0, 1) strictly inside the interval, (k + 0.5) / 2^24 for a uniform integer
 k in [0, 2^24), stored as fp32 (exact); decode KV lengths are integers drawn
 uniformly from [lo, hi] inclusive.
@@ -83,6 +85,11 @@ HYBRID_LAYERS = tuple(
 )
 DECODE_FULL = DecodeWorkload("decode_B64_H16_full", 64, 16, 0, 4)
 DECODE_W128 = DecodeWorkload("decode_B64_H16_w128", 64, 16, 128, 4)
+# The same decode batch over the compressed (latent) cache: one 576-wide row per token.
+LATENT_FULL = DecodeWorkload("latent_decode_B64_H16_full", 64, 16, 0, 4)
+LATENT_W128 = DecodeWorkload("latent_decode_B64_H16_w128", 64, 16, 128, 4)
+DC, DR = 512, 64
+DL = DC + DR
 
 
 def _normal_bf16(shape, gen, device):
@@ -123,6 +130,30 @@ def make_decode_inputs(kv_lengths, num_kv_heads, seed, device="cpu"):
         "q_noise": _normal_bf16((b, num_kv_heads, DQK), gen, device),
         "k_cache": _normal_bf16((nk, num_kv_heads, DQK), gen, device),
         "v_cache": _normal_bf16((nk, num_kv_heads, DV), gen, device),
+        "lam": _lambda((b, hs), gen, device),
+        "gate": _normal_bf16((b, hs, DV), gen, device),
+        "cu_seqlens_k": torch.from_numpy(cu.astype(np.int32)).to(device),
+    }
+
+
+def make_latent_decode_inputs(kv_lengths, num_kv_heads, seed, device="cpu"):
+    """Decode inputs over the latent cache: absorbed queries q_abs_sig [B, 4H, 576],
+    q_abs_noise [B, H, 576], cache rows ckv [Nk, 576], w_uv [H, 128, 512] (bf16),
+    lam [B, 4H] (fp32), gate [B, 4H, 128] (bf16) and cu_seqlens_k (int32)."""
+    lengths = np.asarray(kv_lengths, dtype=np.int64)
+    b = int(lengths.shape[0])
+    nk = int(lengths.sum())
+    hs = GROUP * num_kv_heads
+    gen = torch.Generator(device=device).manual_seed(int(seed))
+    cu = np.zeros(b + 1, dtype=np.int64)
+    cu[1:] = np.cumsum(lengths)
+    w_uv = (torch.randn((num_kv_heads, DV, DC), generator=gen, device=device, dtype=torch.float32)
+            / float(np.sqrt(DC))).to(torch.bfloat16)
+    return {
+        "q_abs_sig": _normal_bf16((b, hs, DL), gen, device),
+        "q_abs_noise": _normal_bf16((b, num_kv_heads, DL), gen, device),
+        "ckv": _normal_bf16((nk, DL), gen, device),
+        "w_uv": w_uv,
         "lam": _lambda((b, hs), gen, device),
         "gate": _normal_bf16((b, hs, DV), gen, device),
         "cu_seqlens_k": torch.from_numpy(cu.astype(np.int32)).to(device),

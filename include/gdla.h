@@ -57,6 +57,9 @@ extern "C" {
 #define GDLA_DQK 192          /* query-key head dim */
 #define GDLA_DV 128           /* value head dim */
 #define GDLA_MAX_KV_HEADS 64  /* largest num_kv_heads accepted */
+#define GDLA_LATENT_MAX_KV_HEADS 16  /* largest num_kv_heads of the latent-cache decode */
+#define GDLA_DC 512           /* latent (compressed KV) dim */
+#define GDLA_DR 64            /* shared rotary key dim */
 #define GDLA_VERSION 1
 
 typedef enum {
@@ -139,6 +142,50 @@ GDLA_API gdla_status_t gdla_attn_decode(const void *q_sig, const void *q_noise, 
                                const float *lambda, const void *gate_logits, void *out,
                                int batch, int num_kv_heads, int window,
                                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Decode over the compressed (latent) KV cache, with the key and value
+ * up-projections absorbed (aitrends.kr/articles/94908, head-configuration
+ * paragraph: KV low-rank dimension 512 and one 64-wide rotary key shared by
+ * every KV head, the KV heads being an up-projection of that compressed row;
+ * the paragraph on MLA's compressed KV cache for decoding). The cache holds
+ * one 576-wide row per token, [c (512) | k_rope (64)], 1,152 bytes instead of
+ * the 10,240 of 16 expanded KV heads. Readings where the pages are silent:
+ * the 192 query-key dims are 128 non-rotary then 64 rotary; per KV head j,
+ * K_j = [W^UK_j c | k_rope] and V_j = W^UV_j c with W^UK_j, W^UV_j [128 x 512].
+ * With q_abs = [W^UK_j^T q_nope | q_rope] (prepared by the caller), every
+ * query head attends over the shared rows with scale 1/sqrt(192); its output
+ * is H = W^UV_j (softmax-weighted average of c), followed by the same
+ * D = H_S - lambda H_N and sigmoid gate as gdla_attn_decode.
+ *   q_abs_sig    bf16 [batch, 4*num_kv_heads, 576]
+ *   q_abs_noise  bf16 [batch, num_kv_heads, 576]
+ *   ckv          bf16 [Nk, 576], sequences packed back to back
+ *   cu_seqlens_k DEVICE int32 [batch + 1], as for gdla_attn_decode (a sequence
+ *                whose length is not in 1 .. max_seqlen_k, or that ends past
+ *                num_cache_rows, gets an all-zero output)
+ *   num_cache_rows HOST number of rows Nk of ckv, >= 1; reads never pass it
+ *   max_seqlen_k HOST upper bound on every L_b, >= 1 (sizes the split plan)
+ *   w_uv         bf16 [num_kv_heads, 128, 512]
+ *   lambda       fp32 [batch, 4*num_kv_heads]
+ *   gate_logits  bf16 [batch, 4*num_kv_heads, 128]
+ *   out          bf16 [batch, 4*num_kv_heads, 128], written
+ *   num_kv_heads 1 .. 16 (all 5 * num_kv_heads query heads of a sequence share
+ *                one CTA)
+ *   window       <= 0: full context; > 0: the last `window` cache rows
+ *   workspace    DEVICE scratch of at least gdla_decode_latent_workspace_bytes(
+ *                batch, num_kv_heads, max_seqlen_k, window) bytes, 256-byte
+ *                aligned; its contents need no initialisation
+ * Errors: GDLA_ERR_INVALID_ARG (null/misaligned pointers, batch < 1,
+ * num_cache_rows < 1, max_seqlen_k < 1), GDLA_ERR_UNSUPPORTED (num_kv_heads
+ * outside 1..16), GDLA_ERR_WORKSPACE (workspace NULL, misaligned or smaller
+ * than required), GDLA_ERR_CUDA (launch failure).
+ */
+GDLA_API size_t gdla_decode_latent_workspace_bytes(int batch, int num_kv_heads, int max_seqlen_k, int window);
+GDLA_API gdla_status_t gdla_attn_decode_latent(const void *q_abs_sig, const void *q_abs_noise, const void *ckv,
+                                               const int32_t *cu_seqlens_k, int num_cache_rows, int max_seqlen_k,
+                                               const void *w_uv, const float *lambda, const void *gate_logits,
+                                               void *out, int batch, int num_kv_heads, int window,
+                                               void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Decode for callers that cannot allocate device memory. The paper has no

@@ -105,3 +105,39 @@ def test_binding_rejects_cpu_tensors():
     t = torch.zeros((4, 4, 192), dtype=torch.bfloat16)
     with pytest.raises((ValueError, TypeError)):
         gdla.attn_fwd(t, t[:, :1], t[:, :1], t[:, :1, :128], torch.zeros(4, 4), t[..., :128], [4])
+
+
+def _lat(lib, ws=FAKE, ws_bytes=1 << 40, batch=2, hkv=1, nk=10, max_len=5, window=0, ptrs=None, cu=FAKE):
+    p = ptrs or [FAKE] * 3
+    tail = [FAKE] * 4   # w_uv, lambda, gate, out
+    return lib.gdla_attn_decode_latent(*[ctypes.c_void_p(x) for x in p], ctypes.c_void_p(cu), nk, max_len,
+                                       *[ctypes.c_void_p(x) for x in tail], batch, hkv, window,
+                                       ctypes.c_void_p(ws), ws_bytes, None)
+
+
+def test_latent_decode_argument_checks(lib):
+    assert _lat(lib, batch=0) == 1
+    assert _lat(lib, nk=0) == 1
+    assert _lat(lib, max_len=0) == 1
+    assert _lat(lib, hkv=17) == 2                   # 5 * 16 query heads per CTA at most
+    assert _lat(lib, hkv=0) == 2
+    assert _lat(lib, cu=0) == 1
+    assert _lat(lib, cu=FAKE + 2) == 1
+    p = [FAKE] * 3
+    p[2] = FAKE + 8
+    assert _lat(lib, ptrs=p) == 1
+    need = lib.gdla_decode_latent_workspace_bytes(2, 1, 5000, 0)
+    assert need > 0
+    assert _lat(lib, max_len=5000, ws=0) == 3
+    assert _lat(lib, max_len=5000, ws_bytes=need - 1) == 3
+    assert _lat(lib, max_len=5000, ws=FAKE + 16) == 3
+
+
+def test_latent_workspace_sizes(lib):
+    # per (sequence, split): 80 head rows x (512 latent dims + max and sum) fp32
+    per = 80 * (512 + 2) * 4
+    assert lib.gdla_decode_latent_workspace_bytes(64, 16, 32768, 0) == 64 * 16 * per   # 16 splits of 2,048 keys
+    assert lib.gdla_decode_latent_workspace_bytes(64, 16, 32768, 128) == 64 * 1 * per   # a window: one split
+    assert lib.gdla_decode_latent_workspace_bytes(1, 16, 1 << 20, 0) == 32 * per        # at most 32 splits
+    assert lib.gdla_decode_latent_workspace_bytes(1, 17, 4096, 0) == 0
+    assert lib.gdla_decode_latent_workspace_bytes(0, 16, 4096, 0) == 0

@@ -31,6 +31,16 @@ def test_bytes_per_token_and_per_key():
     assert bench.decode_bytes([1000, 100], 16, 128) == (128 + 100) * 10240 + 2 * 63744
 
 
+def test_latent_decode_accounting():
+    # 1,152 B per visible key (576 bf16, shared by all 80 heads); per query 80 x 576 absorbed query
+    # dims, 64 x 128 gate and output (bf16) and 64 lambdas; W^UV (16 x 128 x 512 bf16) once
+    per_query = 2 * (80 * 576 + 64 * 128 + 64 * 128) + 4 * 64
+    assert bench.latent_bytes([1000, 3000], 16, 0) == 4000 * 1152 + 2 * per_query + 16 * 128 * 512 * 2
+    assert bench.latent_bytes([1000, 100], 16, 128) == 228 * 1152 + 2 * per_query + 16 * 128 * 512 * 2
+    # flops: 80 heads x (576 score + 512 value) x 2 per key, 80 x 128 x 512 x 2 up-projection per query
+    assert bench.latent_flops([1000], 16, 0) == 1000 * 80 * 1088 * 2 + 80 * 128 * 512 * 2
+
+
 def test_code_only_ignores_comments_and_blank_lines():
     a = "int f(int x) {  // doubles\n    /* the\n       body */\n    return 2 * x;\n}\n\n"
     b = "int f(int x) {\n\n    return 2 * x;   // twice x\n}\n"

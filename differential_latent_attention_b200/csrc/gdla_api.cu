@@ -297,13 +297,13 @@ gdla_status_t gdla_attn_decode_latent(const void *q_abs_sig, const void *q_abs_n
     LatentLaunch L{};
     const int hkv = num_kv_heads;
     // Q boxes: one sequence's 4H signal rows and H noise rows, 64 dims at a time;
-    // latent cache: 48 rows x 64 dims.
+    // latent cache: 48 rows x 64 dims; W^UV_j: its 128 rows x 64 dims.
     if (!make_map(&L.tm_qs, q_abs_sig, 576, 4 * hkv, static_cast<uint64_t>(batch), 64, 4 * hkv, 1) ||
         !make_map(&L.tm_qn, q_abs_noise, 576, hkv, static_cast<uint64_t>(batch), 64, hkv, 1) ||
-        !make_map(&L.tm_c, ckv, 576, 1, static_cast<uint64_t>(num_cache_rows), 64, 1, 48))
+        !make_map(&L.tm_c, ckv, 576, 1, static_cast<uint64_t>(num_cache_rows), 64, 1, 48) ||
+        !make_map(&L.tm_w, w_uv, 512, 128, static_cast<uint64_t>(hkv), 64, 128, 1))
         return GDLA_ERR_CUDA;
     L.cu_seqlens_k = cu_seqlens_k;
-    L.w_uv = static_cast<const __nv_bfloat16 *>(w_uv);
     L.lambda = lambda;
     L.gate = static_cast<const __nv_bfloat16 *>(gate_logits);
     L.out = static_cast<__nv_bfloat16 *>(out);

@@ -137,25 +137,28 @@ struct DecodeItem {
     int n_stages;
 };
 
-__device__ __forceinline__ int decode_visible_keys(const int32_t *__restrict__ cu, int b, const DecodePlan &plan,
-                                                   int &start, int &lo) {
-    start = cu[b];
-    const int end = cu[b + 1];
+__device__ __forceinline__ int decode_visible_keys_of(int start_, int end, const DecodePlan &plan, int &start,
+                                                      int &lo) {
+    start = start_;
     const int len = end - start;
     const bool ok = (start >= 0) && (len >= 1) && (len <= plan.max_seqlen_k) && (end <= plan.num_cache_rows);
     lo = (plan.window > 0) ? max(0, len - plan.window) : 0;
     return ok ? len - lo : 0;
 }
+__device__ __forceinline__ int decode_visible_keys(const int32_t *__restrict__ cu, int b, const DecodePlan &plan,
+                                                   int &start, int &lo) {
+    return decode_visible_keys_of(cu[b], cu[b + 1], plan, start, lo);
+}
 
-__device__ __forceinline__ DecodeItem decode_item(const int32_t *__restrict__ cu, int w, const DecodePlan &plan,
-                                              int tk) {
+// Item w given its sequence's cache bounds cu[b], cu[b+1] (read by the caller).
+__device__ __forceinline__ DecodeItem decode_item(int cu_b, int cu_b1, int w, const DecodePlan &plan, int tk) {
     DecodeItem d;
     d.split = w % plan.num_splits;
     const int rest = w / plan.num_splits;
     d.group = rest % plan.hkv;
     d.b = rest / plan.hkv;
     int lo;
-    const int n_vis = decode_visible_keys(cu, d.b, plan, d.start, lo);
+    const int n_vis = decode_visible_keys_of(cu_b, cu_b1, plan, d.start, lo);
     d.k_begin = lo + d.split * plan.split_keys;
     d.k_end = lo + min(n_vis, (d.split + 1) * plan.split_keys);
     d.n_stages = max(0, (d.k_end - d.k_begin + tk - 1) / tk);
@@ -217,8 +220,22 @@ gdla_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_
             tma_prefetch_desc(&tm_v);
             int g = 0, issued = 0;  // stages issued by this CTA (ring position)
             bool ok = true;
+            // Sequence bounds one item ahead, so their load latency overlaps the
+            // current item's copies.
+            const auto seq_of = [&](int ww) { return (ww / ns) / hkv; };
+            int nb0 = 0, nb1 = 0;
+            if (blockIdx.x < n_work) {
+                nb0 = __ldg(cu_seqlens_k + seq_of(blockIdx.x));
+                nb1 = __ldg(cu_seqlens_k + seq_of(blockIdx.x) + 1);
+            }
             for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x) {
-                const DecodeItem d = decode_item(cu_seqlens_k, w, plan, TK);
+                const int cb0 = nb0, cb1 = nb1;
+                const int wn = w + gridDim.x;
+                if (wn < n_work) {
+                    nb0 = __ldg(cu_seqlens_k + seq_of(wn));
+                    nb1 = __ldg(cu_seqlens_k + seq_of(wn) + 1);
+                }
+                const DecodeItem d = decode_item(cb0, cb1, w, plan, TK);
                 const int n_issue = max(1, d.n_stages);
                 for (int it = 0; it < n_issue; ++it, ++g) {
                     const int st = g % STAGES;

@@ -359,99 +359,200 @@ gdla_decode_latent_split_kernel(const __grid_constant__ CUtensorMap tm_qs, const
     }
 }
 
-// Combine: one CTA (4 warps) per (sequence, group j): merge the splits of the
-// group's 5 head rows (log-sum-exp weights), then H = W^UV_j o (each warp 32
-// of the 128 output dims, W rows read coalesced), then the GDLA epilogue.
-__global__ void __launch_bounds__(128)
-gdla_decode_latent_combine_kernel(const float *__restrict__ ws, const int32_t *__restrict__ cu_seqlens_k,
-                                  const __nv_bfloat16 *__restrict__ w_uv, const float *__restrict__ lambda,
+// Combine: one CTA per (group j, block of BB sequences). It merges each
+// sequence's splits of the group's 5 head rows (log-sum-exp weights) into
+// o [BB x 5 x 512] fp32, then forms H = W^UV_j o on the tensor cores:
+//     D [128 dims x 80] = W^UV_j [128 x 512] . B^T,  B [80 x 512]
+// with B's rows (sequence, head, part): part 0 the bf16 rounding of o, part 1
+// the bf16 rounding of the remainder, so that the product carries o to about
+// 16 bits (one bf16 rounding alone would leave ~1e-3 relative error in H,
+// which D = H_S - lambda H_N can magnify). W^UV_j (128 KB) comes in by TMA
+// once per BB sequences; warps 0-3 (one TMEM lane = one output dim each) add
+// the parts and apply the GDLA epilogue.
+namespace lc {
+constexpr int BB = 8;                  // sequences per CTA
+constexpr int NCOMBO = BB * 5;         // (sequence, head) rows of o
+constexpr int NR = 2 * NCOMBO;         // B rows: 80
+constexpr int W_CH = 128 * 128;        // a 64-dim chunk of W^UV_j: 128 rows x 128 B
+constexpr int B_CH = NR * 128;         // a 64-dim chunk of B: 80 rows x 128 B
+constexpr int OFF_W = 0;
+constexpr int OFF_B = OFF_W + 8 * W_CH;
+constexpr int OFF_WGT = OFF_B + 8 * B_CH;                 // [NCOMBO][kLatentMaxSplits] merge weights
+constexpr int OFF_INVL = OFF_WGT + NCOMBO * kLatentMaxSplits * 4;
+constexpr int OFF_BAR = OFF_INVL + NCOMBO * 4;
+constexpr int OFF_MISC = OFF_BAR + 2 * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+constexpr int NUM_THREADS = 256;
+constexpr uint32_t TMEM_COLS = 128;
+static_assert(OFF_B % 1024 == 0 && B_CH % 1024 == 0, "swizzle atoms");
+static_assert(OFF_BAR % 8 == 0, "barrier alignment");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+}  // namespace lc
+
+__global__ void __launch_bounds__(lc::NUM_THREADS, 1)
+gdla_decode_latent_combine_kernel(const __grid_constant__ CUtensorMap tm_w, const float *__restrict__ ws,
+                                  const int32_t *__restrict__ cu_seqlens_k, const float *__restrict__ lambda,
                                   const __nv_bfloat16 *__restrict__ gate, __nv_bfloat16 *__restrict__ out,
                                   const LatentPlan plan) {
-    using namespace lt;
-    __shared__ __align__(16) float o_s[5][DC];
-    __shared__ float w_s[5][kLatentMaxSplits];
-    __shared__ float inv_ls[5];
-    __shared__ float h_s[5][DV];
-    const int j = blockIdx.x, b = blockIdx.y;
-    const int hkv = plan.hkv, ns = plan.num_splits;
+    using namespace lc;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *wgt_s = reinterpret_cast<float *>(smem + OFF_WGT);
+    float *inv_l_s = reinterpret_cast<float *>(smem + OFF_INVL);
+    uint64_t *w_full = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint64_t *mma_done = w_full + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    const int j = blockIdx.x, b0 = blockIdx.y * BB;
+    const int hkv = plan.hkv, ns = plan.num_splits, batch = plan.batch;
     const int ns_pad = latent_ns_pad(hkv);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // splits holding keys of this sequence (the split kernel wrote the others' nothing)
-    const int start = cu_seqlens_k[b], end = cu_seqlens_k[b + 1];
-    const int len = end - start;
-    const bool valid = (start >= 0) && (len >= 1) && (len <= plan.max_seqlen_k) && (end <= plan.num_cache_rows);
-    const int lo = (plan.window > 0) ? max(0, len - plan.window) : 0;
-    const int n_vis = valid ? len - lo : 0;
-    const int ns_b = min(ns, (n_vis + plan.split_keys - 1) / plan.split_keys);
     const float *wml = ws + plan.ml_offset_floats;
-    // weights: warp h (h < 4) handles head h, warp 0 also the noise head
-    for (int hh = warp; hh < 5; hh += 4) {
+
+    if (threadIdx.x == 0) {
+        mbar_init(w_full, 1);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(w_full, 8 * W_CH);
+        for (int c = 0; c < 8; ++c) tma_load_3d(smem + OFF_W + c * W_CH, &tm_w, w_full, c * 64, 0, j);
+    }
+
+    // Splits holding keys of sequence b (the split kernel wrote the others nothing).
+    auto splits_of = [&](int b) {
+        const int start = cu_seqlens_k[b], end = cu_seqlens_k[b + 1];
+        const int len = end - start;
+        const bool valid = (start >= 0) && (len >= 1) && (len <= plan.max_seqlen_k) && (end <= plan.num_cache_rows);
+        const int lo = (plan.window > 0) ? max(0, len - plan.window) : 0;
+        const int n_vis = valid ? len - lo : 0;
+        return min(ns, (n_vis + plan.split_keys - 1) / plan.split_keys);
+    };
+    // Merge weights: warp w takes combos w, w + 8, ...; lane = split (ns <= 32).
+    for (int c = warp; c < NCOMBO; c += NUM_THREADS / 32) {
+        const int b = b0 + c / 5, hh = c % 5;
         const int row = (hh < 4) ? 4 * j + hh : ns_pad + j;
-        float M = -INFINITY;
-        for (int s = lane; s < ns_b; s += 32)
-            M = fmaxf(M, wml[(static_cast<size_t>(b) * ns + s) * (MAX_ROWS * 2) + 2 * row]);
+        const int ns_b = (b < batch) ? splits_of(b) : 0;
+        const bool mine = lane < ns_b;
+        const size_t base = (static_cast<size_t>(b) * ns + lane) * (lt::MAX_ROWS * 2) + 2 * row;
+        const float ms = mine ? wml[base] : -INFINITY;
+        const float ls = mine ? wml[base + 1] : 0.f;
+        float M = ms;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        float L = 0.f;
-        for (int s = lane; s < ns_b; s += 32) {
-            const size_t base = (static_cast<size_t>(b) * ns + s) * (MAX_ROWS * 2) + 2 * row;
-            const float ms = wml[base];
-            const float wgt = (ms == -INFINITY) ? 0.f : fast_exp2(ms - M);
-            w_s[hh][s] = wgt;
-            L += wml[base + 1] * wgt;
-        }
+        const float wgt = (ms == -INFINITY) ? 0.f : fast_exp2(ms - M);
+        float L = ls * wgt;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-        if (lane == 0) inv_ls[hh] = (L > 0.f) ? 1.f / L : 0.f;
+        wgt_s[c * kLatentMaxSplits + lane] = wgt;
+        if (lane == 0) inv_l_s[c] = (L > 0.f) ? 1.f / L : 0.f;
     }
     __syncthreads();
-    // o[h][e] = sum_s w_s O_s[row][e] / L
-    for (int idx = threadIdx.x; idx < 5 * DC; idx += 128) {
-        const int hh = idx / DC, e = idx % DC;
+    // B rows 2c (bf16 of o) and 2c+1 (bf16 of the remainder), K-major with the
+    // 128-byte swizzle: task = (combo c, 8-dim unit u of 64).
+    for (int task = threadIdx.x; task < NCOMBO * 64; task += NUM_THREADS) {
+        const int c = task >> 6, u = task & 63;
+        const int b = b0 + c / 5, hh = c % 5;
         const int row = (hh < 4) ? 4 * j + hh : ns_pad + j;
-        float acc = 0.f;
+        const int ns_b = (b < batch) ? splits_of(b) : 0;
+        float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int s = 0; s < ns_b; ++s) {
-            const float wgt = w_s[hh][s];
-            if (wgt != 0.f) acc = fmaf(wgt, ws[((static_cast<size_t>(b) * ns + s) * MAX_ROWS + row) * DC + e], acc);
+            const float wgt = wgt_s[c * kLatentMaxSplits + s];
+            if (wgt == 0.f) continue;
+            const float4 *src = reinterpret_cast<const float4 *>(
+                ws + ((static_cast<size_t>(b) * ns + s) * lt::MAX_ROWS + row) * lt::DC + u * 8);
+            const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
+            o[0] = fmaf(wgt, x0.x, o[0]);
+            o[1] = fmaf(wgt, x0.y, o[1]);
+            o[2] = fmaf(wgt, x0.z, o[2]);
+            o[3] = fmaf(wgt, x0.w, o[3]);
+            o[4] = fmaf(wgt, x1.x, o[4]);
+            o[5] = fmaf(wgt, x1.y, o[5]);
+            o[6] = fmaf(wgt, x1.z, o[6]);
+            o[7] = fmaf(wgt, x1.w, o[7]);
         }
-        o_s[hh][e] = acc * inv_ls[hh];
+        const float il = inv_l_s[c];
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float v0 = o[2 * i] * il, v1 = o[2 * i + 1] * il;
+            hi[i] = pack_bf16x2(v0, v1);
+            const float h0 = __uint_as_float(hi[i] << 16), h1 = __uint_as_float(hi[i] & 0xFFFF0000u);
+            lo[i] = pack_bf16x2(v0 - h0, v1 - h1);
+        }
+        const int kc = u >> 3, unit = u & 7;
+        uint8_t *chunk = smem + OFF_B + kc * B_CH;
+        const int r0 = 2 * c, r1 = 2 * c + 1;
+        *reinterpret_cast<uint4 *>(chunk + r0 * 128 + ((unit ^ (r0 & 7)) << 4)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(chunk + r1 * 128 + ((unit ^ (r1 & 7)) << 4)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
     }
+    fence_proxy_async_smem();
+    tc_fence_before();
     __syncthreads();
-    // H[h][d] = sum_e W^UV_j[d][e] o[h][e]: warp w covers d = w, w+4, ...; lanes over e
-    const __nv_bfloat16 *wj = w_uv + static_cast<size_t>(j) * DV * DC;
-    for (int d = warp; d < DV; d += 4) {
-        float acc[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
-        const __nv_bfloat16 *wrow = wj + static_cast<size_t>(d) * DC;
+    if (warp == 0) {
+        tc_fence_after();
+        const uint32_t leader = elect_one_sync();
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(w_full, 0, abort_flag, ERR_SITE_LATENT | 8));
+        if (ok) {
+            tc_fence_after();
+            constexpr uint32_t idesc = idesc_bf16_f32(128, NR, false, false);
+            const uint64_t w_desc0 = desc_sw128(smem_u32(smem + OFF_W), 16, 1024);
+            const uint64_t b_desc0 = desc_sw128(smem_u32(smem + OFF_B), 16, 1024);
 #pragma unroll
-        for (int e0 = 0; e0 < DC; e0 += 256) {
-            const uint4 wv = *reinterpret_cast<const uint4 *>(wrow + e0 + lane * 8);
-            const __nv_bfloat16 *wb = reinterpret_cast<const __nv_bfloat16 *>(&wv);
+            for (int kk = 0; kk < lt::DC / 16; ++kk) {
+                const uint32_t offw = ((kk >> 2) * W_CH + (kk & 3) * 32) >> 4;
+                const uint32_t offb = ((kk >> 2) * B_CH + (kk & 3) * 32) >> 4;
+                umma_ss_leader(tmem, w_desc0 + offw, b_desc0 + offb, idesc, kk > 0, leader);
+            }
+            umma_commit_leader(mma_done, leader);
+        } else if (lane == 0) {
+            mbar_wait_cycles(w_full, 0, 1ll << 22);  // the W^UV copy lands before the CTA leaves
+        }
+    }
+    if (warp < 4) {
+        // Thread = output dim d (TMEM lane); columns 10 s' + 2 hh + part.
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(mma_done, 0, abort_flag, ERR_SITE_LATENT | 9));
+        if (ok) {
+            tc_fence_after();
+            const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+            uint32_t ra[32], rb[32], rc[16];
+            tmem_ld32(lane_base, ra);
+            tmem_ld32(lane_base + 32, rb);
+            tmem_ld16(lane_base + 64, rc);
+            auto col = [&](int n) -> float {
+                return __uint_as_float(n < 32 ? ra[n] : (n < 64 ? rb[n - 32] : rc[n - 64]));
+            };
+            const int d = threadIdx.x;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float wf = __bfloat162float(wb[i]);
+            for (int sl = 0; sl < BB; ++sl) {
+                const int b = b0 + sl;
+                if (b >= batch) break;
+                const float hn = col(10 * sl + 8) + col(10 * sl + 9);
 #pragma unroll
-                for (int hh = 0; hh < 5; ++hh) acc[hh] = fmaf(wf, o_s[hh][e0 + lane * 8 + i], acc[hh]);
+                for (int i = 0; i < 4; ++i) {
+                    const float hsig = col(10 * sl + 2 * i) + col(10 * sl + 2 * i + 1);
+                    const size_t orow = static_cast<size_t>(b) * 4 * hkv + 4 * j + i;
+                    const float dd = hsig - lambda[orow] * hn;
+                    const float g = __bfloat162float(gate[orow * lt::DV + d]);
+                    out[orow * lt::DV + d] = __float2bfloat16_rn(__fdividef(dd, 1.f + __expf(-g)));
+                }
             }
         }
-#pragma unroll
-        for (int hh = 0; hh < 5; ++hh) {
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) acc[hh] += __shfl_xor_sync(0xffffffffu, acc[hh], off);
-        }
-        if (lane == 0)
-#pragma unroll
-            for (int hh = 0; hh < 5; ++hh) h_s[hh][d] = acc[hh];
     }
+    tc_fence_before();
     __syncthreads();
-    // GDLA epilogue: 128 threads, one per output dim
-    const int d = threadIdx.x;
-    const float hn = h_s[4][d];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const size_t orow = static_cast<size_t>(b) * 4 * hkv + 4 * j + i;
-        const float dd = h_s[i][d] - lambda[orow] * hn;
-        const float g = __bfloat162float(gate[orow * DV + d]);
-        out[orow * DV + d] = __float2bfloat16_rn(__fdividef(dd, 1.f + __expf(-g)));
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
     }
 }
 
@@ -494,9 +595,16 @@ cudaError_t launch_decode_latent(const LatentLaunch &L, const LatentPlan &plan, 
                                                                                        L.cu_seqlens_k, L.ws, plan);
     e = cudaPeekAtLastError();
     if (e != cudaSuccess) return e;
-    dim3 grid2(plan.hkv, plan.batch);
-    gdla_decode_latent_combine_kernel<<<grid2, 128, 0, stream>>>(L.ws, L.cu_seqlens_k, L.w_uv, L.lambda, L.gate,
-                                                                 L.out, plan);
+    static PerContextFlag combine_attr_set;
+    if (!combine_attr_set.is_set(dev, ctx)) {
+        e = cudaFuncSetAttribute(gdla_decode_latent_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 lc::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        combine_attr_set.set(dev, current_context_id());
+    }
+    dim3 grid2(plan.hkv, (plan.batch + lc::BB - 1) / lc::BB);
+    gdla_decode_latent_combine_kernel<<<grid2, lc::NUM_THREADS, lc::SMEM_BYTES, stream>>>(
+        L.tm_w, L.ws, L.cu_seqlens_k, L.lambda, L.gate, L.out, plan);
     return cudaPeekAtLastError();
 }
 

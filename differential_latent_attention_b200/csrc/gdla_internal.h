@@ -123,9 +123,8 @@ struct LatentPlan {
 };
 
 struct LatentLaunch {
-    CUtensorMap tm_qs, tm_qn, tm_c;
+    CUtensorMap tm_qs, tm_qn, tm_c, tm_w;
     const int32_t *cu_seqlens_k;
-    const __nv_bfloat16 *w_uv;
     const float *lambda;
     const __nv_bfloat16 *gate;
     __nv_bfloat16 *out;

@@ -93,17 +93,27 @@ constexpr int G_HALF = TOK * 4 * 128;      // 12 KB
 constexpr int G_TILE = 2 * G_HALF;         // 24 KB
 constexpr int G_WARP_BOX = 6 * 4 * 128;    // 3 KB: one warp's tokens in one half
 constexpr int LAM_TILE = TOK * 4 * 4;      // 384 B: [token][head] fp32
-constexpr uint32_t G_TX = G_TILE + LAM_TILE;
 
-template <int TILES_, int BN_, int STAGES_, bool ASYNC_EPI_>
+// Epilogue forms.
+enum : int {
+    EPI_DIRECT = 0,   // gate rows and lambda loaded by the epilogue, output stored directly
+    EPI_STAGED = 1,   // gate and lambda arrive in shared memory by TMA during the item; the
+                      // output is written over the gate and leaves by TMA store
+    EPI_HALF = 2,     // gate dims 0..63 and lambda staged by TMA during the item (all the
+                      // shared memory left), dims 64..127 loaded by the epilogue; output
+                      // stored directly
+};
+
+template <int TILES_, int BN_, int STAGES_, int EPI_>
 struct Cfg {
     static constexpr int TILES = TILES_;
     static constexpr int BN = BN_;          // keys per KV tile
     static constexpr int STAGES = STAGES_;
     static constexpr int V_BOX = BN;        // keys per V TMA box
-    // Asynchronous epilogue: gate and lambda arrive in shared memory by TMA
-    // during the item, the output leaves by TMA store.
-    static constexpr bool ASYNC_EPI = ASYNC_EPI_;
+    static constexpr int EPI = EPI_;
+    static constexpr bool ASYNC_EPI = EPI != EPI_DIRECT;  // gate / lambda staged by the producer
+    static constexpr int G_HALVES = EPI == EPI_STAGED ? 2 : (EPI == EPI_HALF ? 1 : 0);
+    static constexpr uint32_t GATE_TX = G_HALVES * G_HALF + LAM_TILE;
     static constexpr int CTA_TOK = TILES * TOK;
     static constexpr int KV_CHUNK = BN * 128;            // one 64-dim swizzled chunk
     static constexpr int K_STAGE = KCHUNKS * KV_CHUNK;
@@ -112,7 +122,7 @@ struct Cfg {
     static constexpr int OFF_K = OFF_Q + TILES * Q_TILE;
     static constexpr int OFF_V = OFF_K + STAGES * K_STAGE;
     static constexpr int OFF_G = OFF_V + STAGES * V_STAGE;  // 1024-byte aligned (swizzled boxes)
-    static constexpr int OFF_LAM = OFF_G + (ASYNC_EPI ? TILES * G_TILE : 0);
+    static constexpr int OFF_LAM = OFF_G + TILES * G_HALVES * G_HALF;
     static constexpr int OFF_BAR = OFF_LAM + (ASYNC_EPI ? TILES * LAM_TILE : 0);
     static constexpr int NUM_BARS = 32;
     static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -133,9 +143,10 @@ struct Cfg {
     static_assert(QT_COL0 + (Q_IN_TMEM ? DQK / 2 : 0) <= TMEM_COLS, "TMEM budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(BN == 64 || BN == 128, "key tile");
+    static_assert(STAGES <= 3, "three barriers each for K and V stages");
 };
-using CausalCfg = Cfg<1, 128, 2, false>;
-using SlidingCfg = Cfg<2, 64, 2, true>;
+using CausalCfg = Cfg<1, 128, 2, EPI_HALF>;
+using SlidingCfg = Cfg<2, 64, 2, EPI_STAGED>;
 
 // ------------------------------- epilogue ----------------------------------
 // Per warp: the 24 signal rows of its 6 tokens. gate/out rows are 256 bytes;
@@ -186,6 +197,18 @@ __device__ __forceinline__ void epi_chunk(const uint32_t (&o)[32], float inv_l, 
             uint4 *d = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
             for (int i = 0; i < 4; ++i) d[i] = make_uint4(res[4 * i], res[4 * i + 1], res[4 * i + 2], res[4 * i + 3]);
+        }
+    }
+}
+// This lane's staged gate columns 32ch..32ch+31 (ch 0 or 1 of a 64-dim half):
+// 16 words from its 128-byte swizzled row (`key` = row & 7).
+__device__ __forceinline__ void epi_gate_staged(bool sig, uint32_t row_addr, int key, int ch, uint32_t (&g)[16]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (sig) {
+            lds128(row_addr + ((((ch & 1) * 4 + i) ^ key) << 4), g + 4 * i);
+        } else {
+            g[4 * i] = g[4 * i + 1] = g[4 * i + 2] = g[4 * i + 3] = 0u;
         }
     }
 }
@@ -366,10 +389,10 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                     for (int x = 0; x < TILES; ++x) {
                         if (n_item > 0 && !mbar_wait(g_empty + x, (n_item - 1) & 1, abort_flag, ERR_SITE_PREFILL | 11))
                             return false;
-                        mbar_arrive_expect_tx(g_full + x, G_TX);
+                        mbar_arrive_expect_tx(g_full + x, C::GATE_TX);
                         const int row0 = it.s0 + it.t0 + x * TOK;
-                        for (int h = 0; h < 2; ++h)
-                            tma_load_3d(smem + C::OFF_G + x * G_TILE + h * G_HALF, &tm_gate, g_full + x, h * 64,
+                        for (int h = 0; h < C::G_HALVES; ++h)
+                            tma_load_3d(smem + C::OFF_G + (x * C::G_HALVES + h) * G_HALF, &tm_gate, g_full + x, h * 64,
                                         4 * it.group, row0);
                         tma_load_2d(smem + C::OFF_LAM + x * LAM_TILE, &tm_lam, g_full + x, 4 * it.group, row0);
                     }
@@ -399,8 +422,8 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                     }
                     mbar_arrive_expect_tx(v_full + st, C::V_TX);
                     for (int c = 0; c < VCHUNKS; ++c)
-                        tma_load_3d(smem + C::OFF_V + st * C::V_STAGE + c * C::KV_CHUNK, &tm_v, v_full + st, c * 64,
-                                    it.group, row);
+                        tma_load_3d(smem + C::OFF_V + st * C::V_STAGE + c * C::KV_CHUNK, &tm_v, v_full + st,
+                                    c * 64, it.group, row);
                     issued_kv = kv + 1;
                     if (C::ASYNC_EPI && k == gate_after && !issue_gate()) {
                         ok = false;
@@ -658,7 +681,7 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
             // ----------------------------- epilogue ------------------------------
             const bool valid = is_sig && (t < it.L);
             const size_t row = static_cast<size_t>(it.s0 + t) * hs + 4 * it.group + (lane & 3);
-            if constexpr (C::ASYNC_EPI) {
+            if constexpr (C::EPI == EPI_STAGED) {
                 // Gate and lambda were staged in shared memory during the item; the
                 // output replaces the gate in place and leaves by one TMA store per
                 // warp and half, or (a warp with tokens past the sequence end)
@@ -696,6 +719,39 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(g_empty + x);
+            } else if constexpr (C::EPI == EPI_HALF) {
+                // Gate dims 0..63 and lambda were staged during the item; dims 64..127
+                // are fetched now, while dims 0..63 are computed and stored.
+                uint32_t gw[2][16];
+                epi_fetch_gate(valid, row, gate, wide, 2, gw[0]);
+                epi_fetch_gate(valid, row, gate, wide, 3, gw[1]);
+                bool ok_w = mbar_wait(g_full + x, n_item & 1, abort_flag, ERR_SITE_PREFILL | 12);
+                ok_w = ok_w && mbar_wait(o_final + x, n_item & 1, abort_flag, ERR_SITE_PREFILL | 9);
+                if (!__all_sync(0xffffffffu, ok_w)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+                const float lam = is_sig ? reinterpret_cast<const float *>(smem + C::OFF_LAM + x * LAM_TILE)[24 * wq + lane]
+                                         : 0.f;
+                const uint32_t g_base = smem_u32(smem + C::OFF_G + x * G_HALF) + (24 * wq + lane) * 128;
+#pragma unroll
+                for (int ch = 0; ch < 2; ++ch) {
+                    uint32_t g[16];
+                    epi_gate_staged(is_sig, g_base, lane & 7, ch, g);
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + ch * 32, o);
+                    epi_chunk(o, inv_l, lam, g, hsrc, valid, wide, out + row * DV + ch * 32);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(g_empty + x);  // the staged gate half has been read
+#pragma unroll
+                for (int ch = 2; ch < 4; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32(o_addr + ch * 32, o);
+                    epi_chunk(o, inv_l, lam, gw[ch - 2], hsrc, valid, wide, out + row * DV + ch * 32);
+                }
             } else {
                 // Signal rows fetch their gate row and lambda before waiting for the last PV.
                 uint32_t gw[DV / 32][16];
@@ -722,7 +778,7 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         }
     }
 
-    if (C::ASYNC_EPI && warp < C::PRODUCER_WARP && lane == 0) bulk_wait_group0();  // output stores complete
+    if (C::EPI == EPI_STAGED && warp < C::PRODUCER_WARP && lane == 0) bulk_wait_group0();  // output stores complete
     tc_fence_before();
     __syncthreads();
     if (warp == C::MMA_WARP) {
@@ -734,7 +790,7 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
 // ------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------
-// Full causal and windows over kPrefillSlidingMaxWindow.
+// Full causal and windows over kPrefillSlidingMaxWindow: the one-tile configuration.
 using LongCfg = pf::CausalCfg;
 
 PrefillGeometry prefill_geometry(int window) {

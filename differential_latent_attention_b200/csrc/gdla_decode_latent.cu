@@ -379,7 +379,8 @@ constexpr int OFF_W = 0;
 constexpr int OFF_B = OFF_W + 8 * W_CH;
 constexpr int OFF_WGT = OFF_B + 8 * B_CH;                 // [NCOMBO][kLatentMaxSplits] merge weights
 constexpr int OFF_INVL = OFF_WGT + NCOMBO * kLatentMaxSplits * 4;
-constexpr int OFF_BAR = OFF_INVL + NCOMBO * 4;
+constexpr int OFF_NSB = OFF_INVL + NCOMBO * 4;           // [BB] splits of each sequence
+constexpr int OFF_BAR = OFF_NSB + BB * 4;
 constexpr int OFF_MISC = OFF_BAR + 2 * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
 constexpr int NUM_THREADS = 256;
@@ -399,6 +400,7 @@ gdla_decode_latent_combine_kernel(const __grid_constant__ CUtensorMap tm_w, cons
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *wgt_s = reinterpret_cast<float *>(smem + OFF_WGT);
     float *inv_l_s = reinterpret_cast<float *>(smem + OFF_INVL);
+    int *nsb_s = reinterpret_cast<int *>(smem + OFF_NSB);
     uint64_t *w_full = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint64_t *mma_done = w_full + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
@@ -428,72 +430,148 @@ gdla_decode_latent_combine_kernel(const __grid_constant__ CUtensorMap tm_w, cons
         for (int c = 0; c < 8; ++c) tma_load_3d(smem + OFF_W + c * W_CH, &tm_w, w_full, c * 64, 0, j);
     }
 
-    // Splits holding keys of sequence b (the split kernel wrote the others nothing).
-    auto splits_of = [&](int b) {
-        const int start = cu_seqlens_k[b], end = cu_seqlens_k[b + 1];
-        const int len = end - start;
-        const bool valid = (start >= 0) && (len >= 1) && (len <= plan.max_seqlen_k) && (end <= plan.num_cache_rows);
-        const int lo = (plan.window > 0) ? max(0, len - plan.window) : 0;
-        const int n_vis = valid ? len - lo : 0;
-        return min(ns, (n_vis + plan.split_keys - 1) / plan.split_keys);
-    };
-    // Merge weights: warp w takes combos w, w + 8, ...; lane = split (ns <= 32).
-    for (int c = warp; c < NCOMBO; c += NUM_THREADS / 32) {
-        const int b = b0 + c / 5, hh = c % 5;
-        const int row = (hh < 4) ? 4 * j + hh : ns_pad + j;
-        const int ns_b = (b < batch) ? splits_of(b) : 0;
-        const bool mine = lane < ns_b;
-        const size_t base = (static_cast<size_t>(b) * ns + lane) * (lt::MAX_ROWS * 2) + 2 * row;
-        const float ms = mine ? wml[base] : -INFINITY;
-        const float ls = mine ? wml[base + 1] : 0.f;
-        float M = ms;
+    // Splits holding keys of each sequence of the block (the split kernel wrote
+    // the others nothing); 0 past the batch.
+    if (threadIdx.x < BB) {
+        const int b = b0 + threadIdx.x;
+        int n = 0;
+        if (b < batch) {
+            const int start = cu_seqlens_k[b], end = cu_seqlens_k[b + 1];
+            const int len = end - start;
+            const bool valid =
+                (start >= 0) && (len >= 1) && (len <= plan.max_seqlen_k) && (end <= plan.num_cache_rows);
+            const int lo = (plan.window > 0) ? max(0, len - plan.window) : 0;
+            const int n_vis = valid ? len - lo : 0;
+            n = min(ns, (n_vis + plan.split_keys - 1) / plan.split_keys);
+        }
+        nsb_s[threadIdx.x] = n;
+    }
+    // Epilogue operands (warps 0-3: output dim d = threadIdx.x), loaded while the
+    // rest runs: gate logit and lambda of each (sequence, signal head).
+    uint32_t g_pre[BB * 4 / 2];  // bf16 pairs
+    float lam_pre[BB * 4];
+    if (warp < 4) {
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        const float wgt = (ms == -INFINITY) ? 0.f : fast_exp2(ms - M);
-        float L = ls * wgt;
+        for (int sl = 0; sl < BB; ++sl)
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-        wgt_s[c * kLatentMaxSplits + lane] = wgt;
-        if (lane == 0) inv_l_s[c] = (L > 0.f) ? 1.f / L : 0.f;
+            for (int i = 0; i < 4; ++i) {
+                const int b = min(b0 + sl, batch - 1);
+                const size_t orow = static_cast<size_t>(b) * 4 * hkv + 4 * j + i;
+                const uint16_t gv = __ldg(reinterpret_cast<const unsigned short *>(gate) + orow * lt::DV + threadIdx.x);
+                if (i & 1)
+                    g_pre[sl * 2 + (i >> 1)] |= static_cast<uint32_t>(gv) << 16;
+                else
+                    g_pre[sl * 2 + (i >> 1)] = gv;
+                lam_pre[sl * 4 + i] = __ldg(lambda + orow);
+            }
+    }
+    __syncthreads();
+    // Merge weights: warp w takes combos w, w + 8, ... (all loads first); lane = split (ns <= 32).
+    {
+        constexpr int PER_WARP = NCOMBO / (NUM_THREADS / 32);
+        static_assert(NCOMBO % (NUM_THREADS / 32) == 0, "combos per warp");
+        float ms[PER_WARP], ls[PER_WARP];
+#pragma unroll
+        for (int q = 0; q < PER_WARP; ++q) {
+            const int c = warp + q * (NUM_THREADS / 32);
+            const int hh = c % 5;
+            const int row = (hh < 4) ? 4 * j + hh : ns_pad + j;
+            const bool mine = lane < nsb_s[c / 5];
+            const size_t base = (static_cast<size_t>(b0 + c / 5) * ns + lane) * (lt::MAX_ROWS * 2) + 2 * row;
+            ms[q] = mine ? wml[base] : -INFINITY;
+            ls[q] = mine ? wml[base + 1] : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < PER_WARP; ++q) {
+            const int c = warp + q * (NUM_THREADS / 32);
+            float M = ms[q];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+            const float wgt = (ms[q] == -INFINITY) ? 0.f : fast_exp2(ms[q] - M);
+            float L = ls[q] * wgt;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+            wgt_s[c * kLatentMaxSplits + lane] = wgt;
+            if (lane == 0) inv_l_s[c] = (L > 0.f) ? 1.f / L : 0.f;
+        }
     }
     __syncthreads();
     // B rows 2c (bf16 of o) and 2c+1 (bf16 of the remainder), K-major with the
-    // 128-byte swizzle: task = (combo c, 8-dim unit u of 64).
-    for (int task = threadIdx.x; task < NCOMBO * 64; task += NUM_THREADS) {
-        const int c = task >> 6, u = task & 63;
-        const int b = b0 + c / 5, hh = c % 5;
-        const int row = (hh < 4) ? 4 * j + hh : ns_pad + j;
-        const int ns_b = (b < batch) ? splits_of(b) : 0;
-        float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int s = 0; s < ns_b; ++s) {
-            const float wgt = wgt_s[c * kLatentMaxSplits + s];
-            if (wgt == 0.f) continue;
-            const float4 *src = reinterpret_cast<const float4 *>(
-                ws + ((static_cast<size_t>(b) * ns + s) * lt::MAX_ROWS + row) * lt::DC + u * 8);
-            const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
-            o[0] = fmaf(wgt, x0.x, o[0]);
-            o[1] = fmaf(wgt, x0.y, o[1]);
-            o[2] = fmaf(wgt, x0.z, o[2]);
-            o[3] = fmaf(wgt, x0.w, o[3]);
-            o[4] = fmaf(wgt, x1.x, o[4]);
-            o[5] = fmaf(wgt, x1.y, o[5]);
-            o[6] = fmaf(wgt, x1.z, o[6]);
-            o[7] = fmaf(wgt, x1.w, o[7]);
-        }
-        const float il = inv_l_s[c];
-        uint32_t hi[4], lo[4];
+    // 128-byte swizzle: task = (combo c, 8-dim unit u of 64). Every thread's
+    // tasks load their first split together, then the remaining splits.
+    {
+        constexpr int TASKS = NCOMBO * 64 / NUM_THREADS;  // 10
+        static_assert((NCOMBO * 64) % NUM_THREADS == 0, "tasks per thread");
+        float acc[TASKS][8];
+        auto src_of = [&](int q, int sp) {
+            const int task = threadIdx.x + q * NUM_THREADS;
+            const int c = task >> 6, u = task & 63;
+            const int hh = c % 5;
+            const int row = (hh < 4) ? 4 * j + hh : ns_pad + j;
+            return reinterpret_cast<const float4 *>(
+                ws + ((static_cast<size_t>(b0 + c / 5) * ns + sp) * lt::MAX_ROWS + row) * lt::DC + u * 8);
+        };
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float v0 = o[2 * i] * il, v1 = o[2 * i + 1] * il;
-            hi[i] = pack_bf16x2(v0, v1);
-            const float h0 = __uint_as_float(hi[i] << 16), h1 = __uint_as_float(hi[i] & 0xFFFF0000u);
-            lo[i] = pack_bf16x2(v0 - h0, v1 - h1);
+        for (int q = 0; q < TASKS; ++q) {
+            const int c = (threadIdx.x + q * NUM_THREADS) >> 6;
+            float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0;
+            if (nsb_s[c / 5] > 0) {
+                const float4 *src = src_of(q, 0);
+                x0 = __ldg(src);
+                x1 = __ldg(src + 1);
+            }
+            const float wgt = wgt_s[c * kLatentMaxSplits];
+            acc[q][0] = wgt * x0.x;
+            acc[q][1] = wgt * x0.y;
+            acc[q][2] = wgt * x0.z;
+            acc[q][3] = wgt * x0.w;
+            acc[q][4] = wgt * x1.x;
+            acc[q][5] = wgt * x1.y;
+            acc[q][6] = wgt * x1.z;
+            acc[q][7] = wgt * x1.w;
         }
-        const int kc = u >> 3, unit = u & 7;
-        uint8_t *chunk = smem + OFF_B + kc * B_CH;
-        const int r0 = 2 * c, r1 = 2 * c + 1;
-        *reinterpret_cast<uint4 *>(chunk + r0 * 128 + ((unit ^ (r0 & 7)) << 4)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4 *>(chunk + r1 * 128 + ((unit ^ (r1 & 7)) << 4)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        int ns_max = 0;
+#pragma unroll
+        for (int sl = 0; sl < BB; ++sl) ns_max = max(ns_max, nsb_s[sl]);
+        for (int sp = 1; sp < ns_max; ++sp) {
+#pragma unroll
+            for (int q = 0; q < TASKS; ++q) {
+                const int c = (threadIdx.x + q * NUM_THREADS) >> 6;
+                const float wgt = wgt_s[c * kLatentMaxSplits + sp];
+                if (sp >= nsb_s[c / 5] || wgt == 0.f) continue;
+                const float4 *src = src_of(q, sp);
+                const float4 x0 = __ldg(src), x1 = __ldg(src + 1);
+                acc[q][0] = fmaf(wgt, x0.x, acc[q][0]);
+                acc[q][1] = fmaf(wgt, x0.y, acc[q][1]);
+                acc[q][2] = fmaf(wgt, x0.z, acc[q][2]);
+                acc[q][3] = fmaf(wgt, x0.w, acc[q][3]);
+                acc[q][4] = fmaf(wgt, x1.x, acc[q][4]);
+                acc[q][5] = fmaf(wgt, x1.y, acc[q][5]);
+                acc[q][6] = fmaf(wgt, x1.z, acc[q][6]);
+                acc[q][7] = fmaf(wgt, x1.w, acc[q][7]);
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < TASKS; ++q) {
+            const int task = threadIdx.x + q * NUM_THREADS;
+            const int c = task >> 6, u = task & 63;
+            const float il = inv_l_s[c];
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float v0 = acc[q][2 * i] * il, v1 = acc[q][2 * i + 1] * il;
+                hi[i] = pack_bf16x2(v0, v1);
+                const float h0 = __uint_as_float(hi[i] << 16), h1 = __uint_as_float(hi[i] & 0xFFFF0000u);
+                lo[i] = pack_bf16x2(v0 - h0, v1 - h1);
+            }
+            const int kc = u >> 3, unit = u & 7;
+            uint8_t *chunk = smem + OFF_B + kc * B_CH;
+            const int r0 = 2 * c, r1 = 2 * c + 1;
+            *reinterpret_cast<uint4 *>(chunk + r0 * 128 + ((unit ^ (r0 & 7)) << 4)) =
+                make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4 *>(chunk + r1 * 128 + ((unit ^ (r1 & 7)) << 4)) =
+                make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -541,8 +619,9 @@ gdla_decode_latent_combine_kernel(const __grid_constant__ CUtensorMap tm_w, cons
                 for (int i = 0; i < 4; ++i) {
                     const float hsig = col(10 * sl + 2 * i) + col(10 * sl + 2 * i + 1);
                     const size_t orow = static_cast<size_t>(b) * 4 * hkv + 4 * j + i;
-                    const float dd = hsig - lambda[orow] * hn;
-                    const float g = __bfloat162float(gate[orow * lt::DV + d]);
+                    const float dd = hsig - lam_pre[sl * 4 + i] * hn;
+                    const uint32_t gp = g_pre[sl * 2 + (i >> 1)];
+                    const float g = __uint_as_float((i & 1) ? (gp & 0xFFFF0000u) : (gp << 16));
                     out[orow * lt::DV + d] = __float2bfloat16_rn(__fdividef(dd, 1.f + __expf(-g)));
                 }
             }

@@ -593,11 +593,10 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                 const int u0 = it.kv_lo + k * BN;
                 const bool need_mask = (u0 + BN - 1 > tx0) || (window > 0 && u0 < tx0 + TOK - window);
                 if (need_mask) {
+                    // visible columns: keys lo_t..t of this row
+                    const int c_lo = lo_t - u0, c_hi = t - u0;
 #pragma unroll
-                    for (int i = 0; i < BN; ++i) {
-                        const int u = u0 + i;
-                        if (u > t || u < lo_t) s[i] = -INFINITY;
-                    }
+                    for (int i = 0; i < BN; ++i) s[i] = (i >= c_lo && i <= c_hi) ? s[i] : -INFINITY;
                 }
                 float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll

@@ -129,6 +129,8 @@ def load_peaks():
 KERNEL_SOURCES = {
     "gdla_prefill_kernel": ("gdla_prefill.cu", "gdla_ptx.cuh", "gdla_internal.h"),
     "gdla_decode_split_kernel": ("gdla_decode.cu", "gdla_ptx.cuh", "gdla_internal.h"),
+    "gdla_decode_latent_split_kernel": ("gdla_decode_latent.cu", "gdla_ptx.cuh", "gdla_internal.h"),
+    "gdla_decode_latent_combine_kernel": ("gdla_decode_latent.cu", "gdla_ptx.cuh", "gdla_internal.h"),
 }
 
 

@@ -152,6 +152,26 @@ using SlidingCfg = Cfg<2, 64, 2, EPI_STAGED>;
 // Per warp: the 24 signal rows of its 6 tokens. gate/out rows are 256 bytes;
 // with 32-byte aligned bases each lane moves whole 32-byte sectors (half the
 // memory instructions of 16-byte accesses over the same scattered rows).
+// The gated output of 32 columns of this lane's O row, as 16 bf16 pairs:
+// H = O/l; the token's noise row H_N comes from lane hsrc by shuffle;
+// out = sigmoid(g) (H_S - lambda H_N), in packed fp32 pairs.
+__device__ __forceinline__ void epi_gate_pairs(const uint32_t (&o)[32], float inv_l, float lam,
+                                               const uint32_t (&g)[16], int hsrc, uint32_t (&res)[16]) {
+    const uint64_t inv_l2 = f2_pack(inv_l, inv_l);
+    const uint64_t neg_lam2 = f2_pack(-lam, -lam);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const uint64_t h = f2_mul(f2_pack(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1])), inv_l2);
+        float h0, h1;
+        f2_unpack(h, h0, h1);
+        const float n0 = __shfl_sync(0xffffffffu, h0, hsrc);  // H_N of this row's token
+        const float n1 = __shfl_sync(0xffffffffu, h1, hsrc);
+        const uint64_t d = f2_fma(f2_pack(n0, n1), neg_lam2, h);
+        float r0, r1;
+        f2_unpack(f2_mul(d, sigmoid2_bf16(g[i])), r0, r1);
+        res[i] = pack_bf16x2(r0, r1);
+    }
+}
 // Gate columns 32ch..32ch+31 of one row (16 words of bf16 pairs).
 __device__ __forceinline__ void epi_fetch_gate(bool valid, size_t row, const __nv_bfloat16 *__restrict__ gate,
                                                bool wide, int ch, uint32_t (&g)[16]) {
@@ -180,15 +200,7 @@ __device__ __forceinline__ void epi_fetch_gate(bool valid, size_t row, const __n
 __device__ __forceinline__ void epi_chunk(const uint32_t (&o)[32], float inv_l, float lam, const uint32_t (&g)[16],
                                           int hsrc, bool valid, bool wide, __nv_bfloat16 *__restrict__ dst) {
     uint32_t res[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float h0 = __uint_as_float(o[2 * i]) * inv_l;
-        const float h1 = __uint_as_float(o[2 * i + 1]) * inv_l;
-        const float n0 = __shfl_sync(0xffffffffu, h0, hsrc);  // H_N of this row's token
-        const float n1 = __shfl_sync(0xffffffffu, h1, hsrc);
-        const float2 g2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&g[i]));
-        res[i] = pack_bf16x2(fmaf(-lam, n0, h0) * fast_sigmoid(g2.x), fmaf(-lam, n1, h1) * fast_sigmoid(g2.y));
-    }
+    epi_gate_pairs(o, inv_l, lam, g, hsrc, res);
     if (valid) {
         if (wide) {
             st_v8(dst, res);
@@ -230,15 +242,7 @@ __device__ __forceinline__ void epi_chunk_staged(const uint32_t (&o)[32], float 
         }
     }
     uint32_t res[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float h0 = __uint_as_float(o[2 * i]) * inv_l;
-        const float h1 = __uint_as_float(o[2 * i + 1]) * inv_l;
-        const float n0 = __shfl_sync(0xffffffffu, h0, hsrc);  // H_N of this row's token
-        const float n1 = __shfl_sync(0xffffffffu, h1, hsrc);
-        const float2 g2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&g[i]));
-        res[i] = pack_bf16x2(fmaf(-lam, n0, h0) * fast_sigmoid(g2.x), fmaf(-lam, n1, h1) * fast_sigmoid(g2.y));
-    }
+    epi_gate_pairs(o, inv_l, lam, g, hsrc, res);
     if (sig && to_smem) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) sts128(row_addr + ((((ch & 1) * 4 + i) ^ key) << 4), res + 4 * i);

@@ -341,13 +341,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
 }
-// sigmoid(x) = 0.5 * tanh(x / 2) + 0.5 with the hardware tanh approximation
-// (absolute error below 2.5e-4): one MUFU operation instead of exp + reciprocal.
-__device__ __forceinline__ float fast_sigmoid(float x) {
-    float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
-    return fmaf(0.5f, t, 0.5f);
-}
 __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -366,6 +359,30 @@ __device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi) {
 __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
     uint64_t d;
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// sigmoid of a bf16 pair (low half = first element) as an fp32 pair:
+// sigma(x) = 1/2 tanh(x/2) + 1/2 with tanh taken on an f16 pair, one MUFU op for
+// both (x/2 rounded to f16 is exact for any bf16 x in f16's normal range; the
+// f16 tanh adds ~2^-11 relative error, about that of the f32 form).
+__device__ __forceinline__ uint64_t sigmoid2_bf16(uint32_t g2) {
+    const uint64_t half2 = (static_cast<uint64_t>(__float_as_uint(0.5f)) << 32) | __float_as_uint(0.5f);
+    const uint64_t x = f2_mul((static_cast<uint64_t>(g2 & 0xFFFF0000u) << 32) | (g2 << 16), half2);
+    uint32_t h, t;
+    asm("{\n\t.reg .f32 a, b;\n\tmov.b64 {a, b}, %1;\n\tcvt.rn.f16x2.f32 %0, b, a;\n\t}" : "=r"(h) : "l"(x));
+    asm("tanh.approx.f16x2 %0, %1;" : "=r"(t) : "r"(h));
+    uint64_t tf;
+    asm("{\n\t.reg .f16 lo, hi;\n\t.reg .f32 a, b;\n\tmov.b32 {lo, hi}, %1;\n\tcvt.f32.f16 a, lo;\n\t"
+        "cvt.f32.f16 b, hi;\n\tmov.b64 %0, {a, b};\n\t}"
+        : "=l"(tf)
+        : "r"(t));
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %2;" : "=l"(d) : "l"(tf), "l"(half2));
     return d;
 }
 __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {

@@ -116,6 +116,13 @@ def make_prefill_inputs(seqlens, num_kv_heads, seed, device="cpu"):
     }
 
 
+def make_prefill_grad(seqlens, num_kv_heads, seed, device="cpu"):
+    """Upstream gradient of the prefill output for the backward: dout [N, 4H, 128] bf16."""
+    n = int(sum(int(s) for s in seqlens))
+    gen = torch.Generator(device=device).manual_seed(int(seed) + 7919)
+    return _normal_bf16((n, GROUP * num_kv_heads, DV), gen, device)
+
+
 def make_decode_inputs(kv_lengths, num_kv_heads, seed, device="cpu"):
     """Decode inputs: one query per sequence plus the packed KV cache and cu_seqlens_k (int32)."""
     lengths = np.asarray(kv_lengths, dtype=np.int64)

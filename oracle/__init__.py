@@ -12,6 +12,11 @@ Parity status per function:
   brute force; see ``tests/test_oracle_pins.py``).
 * ``decode`` - pinned through the decode == last prefill row identity and the
   same closed forms.
+* ``decode_latent`` - pinned exactly to ``decode`` through an integer construction
+  (``tests/test_oracle_latent.py``).
+* ``prefill_bwd`` - pinned to fp64 automatic differentiation (torch autograd) of
+  the forward composed from library operations, on full-causal, windowed and
+  ragged inputs (``tests/test_oracle_bwd.py``).
 
 The choice of lambda granularity (one scalar per token and signal head), the
 absence of any normalisation after the subtract and the 1/sqrt(192) softmax
@@ -69,6 +74,9 @@ def _load():
             lib.gdla_oracle_decode_latent.argtypes = [p, p, p, p, p, p, p, ctypes.c_int, ctypes.c_int,
                                                       ctypes.c_int, p, ctypes.c_int]
             lib.gdla_oracle_decode_latent.restype = ctypes.c_int
+            lib.gdla_oracle_prefill_bwd.argtypes = [p, p, p, p, p, p, p, ctypes.c_int, ctypes.c_int, p,
+                                                    ctypes.c_int, p, p, p, p, p, p, ctypes.c_int]
+            lib.gdla_oracle_prefill_bwd.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -191,3 +199,39 @@ def decode_latent(q_abs_sig, q_abs_noise, ckv, cu_seqlens_k, w_uv, lam, gate, wi
     if rc != 0:
         raise ValueError("gdla_oracle_decode_latent rejected its arguments")
     return out
+
+
+def prefill_bwd(q_sig, q_noise, k, v, lam, gate, dout, seqlens, window, num_threads=None):
+    """Gradients of sum(dout * out) for the packed varlen GDLA prefill, in fp64.
+
+    Inputs as ``prefill`` plus dout [N, 4H, 128] (uint16 bf16 bits). Returns a dict
+    of float64 arrays: dq_sig [N, 4H, 192], dq_noise [N, H, 192], dk [N, H, 192],
+    dv [N, H, 128], dlambda [N, 4H], dgate [N, 4H, 128].
+    """
+    hkv = q_noise.shape[1]
+    hs = GROUP * hkv
+    q_sig = _bits(q_sig, (hs, DQK), "q_sig")
+    q_noise = _bits(q_noise, (hkv, DQK), "q_noise")
+    k = _bits(k, (hkv, DQK), "k")
+    v = _bits(v, (hkv, DV), "v")
+    gate = _bits(gate, (hs, DV), "gate")
+    dout = _bits(dout, (hs, DV), "dout")
+    lam = np.ascontiguousarray(lam, dtype=np.float32)
+    seqlens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    n = int(seqlens.sum())
+    for name, a in (("q_sig", q_sig), ("q_noise", q_noise), ("k", k), ("v", v), ("gate", gate),
+                    ("dout", dout), ("lambda", lam)):
+        if a.shape[0] != n:
+            raise ValueError(f"{name}: leading dim {a.shape[0]} != sum(seqlens) {n}")
+    if lam.shape != (n, hs):
+        raise ValueError(f"lambda: expected shape {(n, hs)}, got {lam.shape}")
+    g = {"dq_sig": np.zeros((n, hs, DQK)), "dq_noise": np.zeros((n, hkv, DQK)), "dk": np.zeros((n, hkv, DQK)),
+         "dv": np.zeros((n, hkv, DV)), "dlambda": np.zeros((n, hs)), "dgate": np.zeros((n, hs, DV))}
+    nt = int(num_threads or default_threads())
+    rc = _load().gdla_oracle_prefill_bwd(_ptr(q_sig), _ptr(q_noise), _ptr(k), _ptr(v), _ptr(lam), _ptr(gate),
+                                         _ptr(dout), hkv, int(seqlens.shape[0]), _ptr(seqlens), int(window),
+                                         _ptr(g["dq_sig"]), _ptr(g["dq_noise"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                                         _ptr(g["dlambda"]), _ptr(g["dgate"]), nt)
+    if rc != 0:
+        raise ValueError("gdla_oracle_prefill_bwd rejected its arguments")
+    return g

@@ -427,3 +427,193 @@ int gdla_oracle_decode_latent(const uint16_t *q_abs_sig, const uint16_t *q_abs_n
     free(jobs);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Prefill backward                                                         */
+/* ------------------------------------------------------------------------ */
+/*
+ * Gradients of L = sum(dout * out) with respect to every input of the packed
+ * prefill, by the chain rule written out on the definition above (the pages
+ * train GDLA end to end; they print no gradient, so this is the plain
+ * derivative of the forward as read here):
+ *   sigma_i = 1 / (1 + exp(-g_i)),  out_i = sigma_i D_i,  D_i = H_S,i - lambda_i H_N
+ *   dgate_i   = dout_i * D_i * sigma_i (1 - sigma_i)
+ *   dD_i      = dout_i * sigma_i
+ *   dlambda_i = -sum_d dD_i[d] H_N[d]
+ *   dH_S,i    = dD_i,   dH_N = -sum_i lambda_i dD_i
+ * and for every head h of the group with P_u = softmax_u(s_u), s_u = q_h.k_u / sqrt(192),
+ * H_h = sum_u P_u v_u:
+ *   dv_u += P_u dH_h
+ *   dP_u  = dH_h . v_u,   dS_u = P_u (dP_u - sum_w P_w dP_w)
+ *   dq_h += sum_u dS_u k_u / sqrt(192),   dk_u += dS_u q_h / sqrt(192)
+ * One job is one (sequence, group): it owns the dk, dv rows of that group in
+ * that sequence, so the accumulation needs no locking.
+ */
+typedef struct {
+    const uint16_t *q_sig, *q_noise, *k, *v, *gate, *dout;
+    const float *lambda;
+    int hkv, window, batch;
+    const int32_t *seqlens;
+    const int64_t *seq_start;
+    double *dq_sig, *dq_noise, *dk, *dv, *dlambda, *dgate;
+    long max_len;
+    int nthreads, tid;
+} bwd_job_t;
+
+/* Softmax weights of one head over keys u = 0..nkeys-1 (rows k_rows + u*kstride). */
+static void softmax_weights(const uint16_t *q, const uint16_t *k_rows, long kstride, long nkeys, double *p) {
+    double qd[DQK];
+    for (int d = 0; d < DQK; ++d) qd[d] = bf16_to_double(q[d]);
+    const double root = sqrt((double)DQK);
+    double smax = -INFINITY;
+    for (long u = 0; u < nkeys; ++u) {
+        const uint16_t *kr = k_rows + u * kstride;
+        double s = 0.0;
+        for (int d = 0; d < DQK; ++d) s += qd[d] * bf16_to_double(kr[d]);
+        p[u] = s / root;
+        if (p[u] > smax) smax = p[u];
+    }
+    double den = 0.0;
+    for (long u = 0; u < nkeys; ++u) {
+        p[u] = exp(p[u] - smax);
+        den += p[u];
+    }
+    for (long u = 0; u < nkeys; ++u) p[u] /= den;
+}
+
+/* Backward of one head for one query row: given P (nkeys) and dH, accumulate
+ * dq (DQK), dk rows and dv rows (doubles, strided like the keys). */
+static void head_backward(const uint16_t *q, const uint16_t *k_rows, const uint16_t *v_rows, long kstride,
+                          long vstride, long nkeys, const double *p, const double *dh, double *dp, double *dq,
+                          double *dk_rows, double *dv_rows, long dkstride, long dvstride) {
+    const double root = sqrt((double)DQK);
+    double drow = 0.0;
+    for (long u = 0; u < nkeys; ++u) {
+        const uint16_t *vr = v_rows + u * vstride;
+        double s = 0.0;
+        for (int d = 0; d < DV; ++d) s += dh[d] * bf16_to_double(vr[d]);
+        dp[u] = s;
+        drow += p[u] * s;
+    }
+    for (long u = 0; u < nkeys; ++u) {
+        const double ds = p[u] * (dp[u] - drow);
+        const uint16_t *kr = k_rows + u * kstride;
+        double *dkr = dk_rows + u * dkstride;
+        double *dvr = dv_rows + u * dvstride;
+        for (int d = 0; d < DQK; ++d) {
+            dq[d] += ds * bf16_to_double(kr[d]) / root;
+            dkr[d] += ds * bf16_to_double(q[d]) / root;
+        }
+        for (int d = 0; d < DV; ++d) dvr[d] += p[u] * dh[d];
+    }
+}
+
+static void *bwd_worker(void *arg) {
+    bwd_job_t *J = (bwd_job_t *)arg;
+    const int hkv = J->hkv, hs = GROUP * hkv;
+    const long n1 = J->max_len > 0 ? J->max_len : 1;
+    double *p = (double *)malloc(sizeof(double) * (size_t)n1 * (GROUP + 1));
+    double *dp = (double *)malloc(sizeof(double) * (size_t)n1);
+    if (!p || !dp) { free(p); free(dp); return (void *)1; }
+    const long kstride = (long)hkv * DQK, vstride = (long)hkv * DV;
+    for (int64_t task = J->tid; task < (int64_t)J->batch * hkv; task += J->nthreads) {
+        const int b = (int)(task / hkv), j = (int)(task % hkv);
+        const int64_t s0 = J->seq_start[b];
+        const long L = J->seqlens[b];
+        for (long t = 0; t < L; ++t) {
+            const int64_t n = s0 + t;
+            long lo = 0;
+            if (J->window > 0 && t - J->window + 1 > 0) lo = t - J->window + 1;
+            const long nkeys = t - lo + 1;
+            const uint16_t *krow = J->k + (s0 + lo) * kstride + (long)j * DQK;
+            const uint16_t *vrow = J->v + (s0 + lo) * vstride + (long)j * DV;
+            double *dkrow = J->dk + (s0 + lo) * kstride + (long)j * DQK;
+            double *dvrow = J->dv + (s0 + lo) * vstride + (long)j * DV;
+            const uint16_t *qs = J->q_sig + (n * hs + (long)GROUP * j) * DQK;
+            const uint16_t *qn = J->q_noise + (n * hkv + j) * DQK;
+            /* forward: P and H of the 4 signal heads (h = 0..3) and the noise head (h = 4) */
+            double hh[GROUP + 1][DV];
+            for (int h = 0; h <= GROUP; ++h) {
+                const uint16_t *q = (h < GROUP) ? qs + (long)h * DQK : qn;
+                double *ph = p + (long)h * n1;
+                softmax_weights(q, krow, kstride, nkeys, ph);
+                for (int d = 0; d < DV; ++d) hh[h][d] = 0.0;
+                for (long u = 0; u < nkeys; ++u)
+                    for (int d = 0; d < DV; ++d) hh[h][d] += ph[u] * bf16_to_double(vrow[u * vstride + d]);
+            }
+            /* the gate and the subtract */
+            double dh[GROUP + 1][DV];
+            for (int d = 0; d < DV; ++d) dh[GROUP][d] = 0.0;
+            for (int i = 0; i < GROUP; ++i) {
+                const long row = n * hs + (long)GROUP * j + i;
+                const double l = (double)J->lambda[row];
+                double dl = 0.0;
+                for (int d = 0; d < DV; ++d) {
+                    const double g = bf16_to_double(J->gate[row * DV + d]);
+                    const double sg = 1.0 / (1.0 + exp(-g));
+                    const double dd = hh[i][d] - l * hh[GROUP][d];
+                    const double go = bf16_to_double(J->dout[row * DV + d]);
+                    J->dgate[row * DV + d] = go * dd * sg * (1.0 - sg);
+                    const double ddd = go * sg;
+                    dl -= ddd * hh[GROUP][d];
+                    dh[i][d] = ddd;
+                    dh[GROUP][d] -= l * ddd;
+                }
+                J->dlambda[row] = dl;
+            }
+            /* attention backward of the five heads */
+            for (int h = 0; h <= GROUP; ++h) {
+                const uint16_t *q = (h < GROUP) ? qs + (long)h * DQK : qn;
+                double *dq = (h < GROUP) ? J->dq_sig + (n * hs + (long)GROUP * j + h) * DQK
+                                         : J->dq_noise + (n * hkv + j) * DQK;
+                head_backward(q, krow, vrow, kstride, vstride, nkeys, p + (long)h * n1, dh[h], dp, dq, dkrow,
+                              dvrow, kstride, vstride);
+            }
+        }
+    }
+    free(p);
+    free(dp);
+    return NULL;
+}
+
+/*
+ * Packed varlen prefill backward. Inputs as gdla_oracle_prefill, plus dout
+ * [N, 4*hkv, 128] bf16 bits (the gradient of the output). Outputs, all double
+ * and zeroed here: dq_sig [N, 4*hkv, 192], dq_noise [N, hkv, 192],
+ * dk [N, hkv, 192], dv [N, hkv, 128], dlambda [N, 4*hkv], dgate [N, 4*hkv, 128].
+ * Returns 0, or -1 on a bad argument or an allocation/thread failure.
+ */
+int gdla_oracle_prefill_bwd(const uint16_t *q_sig, const uint16_t *q_noise, const uint16_t *k, const uint16_t *v,
+                            const float *lambda, const uint16_t *gate, const uint16_t *dout, int hkv, int batch,
+                            const int32_t *seqlens, int window, double *dq_sig, double *dq_noise, double *dk,
+                            double *dv, double *dlambda, double *dgate, int nthreads) {
+    if (hkv < 1 || batch < 0 || nthreads < 1) return -1;
+    int64_t total = 0;
+    long max_len = 0;
+    int64_t *seq_start = (int64_t *)malloc(sizeof(int64_t) * (size_t)(batch > 0 ? batch : 1));
+    if (!seq_start) return -1;
+    for (int b = 0; b < batch; ++b) {
+        if (seqlens[b] < 0) { free(seq_start); return -1; }
+        seq_start[b] = total;
+        total += seqlens[b];
+        if (seqlens[b] > max_len) max_len = seqlens[b];
+    }
+    const int hs = GROUP * hkv;
+    memset(dq_sig, 0, sizeof(double) * (size_t)total * hs * DQK);
+    memset(dq_noise, 0, sizeof(double) * (size_t)total * hkv * DQK);
+    memset(dk, 0, sizeof(double) * (size_t)total * hkv * DQK);
+    memset(dv, 0, sizeof(double) * (size_t)total * hkv * DV);
+    memset(dlambda, 0, sizeof(double) * (size_t)total * hs);
+    memset(dgate, 0, sizeof(double) * (size_t)total * hs * DV);
+    bwd_job_t *jobs = (bwd_job_t *)malloc(sizeof(bwd_job_t) * (size_t)nthreads);
+    if (!jobs) { free(seq_start); return -1; }
+    for (int i = 0; i < nthreads; ++i) {
+        bwd_job_t J = {q_sig, q_noise, k, v, gate, dout, lambda, hkv, window, batch, seqlens, seq_start,
+                       dq_sig, dq_noise, dk, dv, dlambda, dgate, max_len, nthreads, i};
+        jobs[i] = J;
+    }
+    int rc = run_threads(bwd_worker, jobs, sizeof(bwd_job_t), nthreads);
+    free(jobs);
+    free(seq_start);
+    return rc;
+}

@@ -62,6 +62,20 @@ bool make_map_f32_2d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D fp32 tensor [d2][d1][d0] (d0 contiguous), unswizzled boxes.
+bool make_map_f32_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                     uint32_t b1, uint32_t b2) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 4, d0 * d1 * 4};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 unsigned long long current_context_id() {
@@ -108,6 +122,72 @@ struct TileItem {
     int seq;
     int qt;
 };
+
+// Every (sequence, unit) of `unit_tokens` tokens with its cost (cost(L, unit)),
+// heaviest first, in plans of at most kPlanMaxItems units and kPlanMaxSeqs
+// sequences; launch(plan) for each. Returns false on the first failed launch.
+template <class Cost, class Launch>
+bool run_plans(int batch, const int32_t *seqlens, int hkv, int window, int unit_tokens, Cost cost, Launch launch) {
+    std::vector<TileItem> items;
+    std::vector<int> seq_start(batch);
+    long long s0 = 0;
+    for (int b = 0; b < batch; ++b) {
+        seq_start[b] = static_cast<int>(s0);
+        const int L = seqlens[b];
+        s0 += L;
+        const int nu = (L + unit_tokens - 1) / unit_tokens;
+        for (int u = 0; u < nu; ++u) items.push_back({cost(L, u), b, u});
+    }
+    std::stable_sort(items.begin(), items.end(), [](const TileItem &a, const TileItem &b) {
+        if (a.cost != b.cost) return a.cost > b.cost;
+        if (a.seq != b.seq) return a.seq < b.seq;
+        return a.qt > b.qt;
+    });
+    std::unique_ptr<PrefillPlan> plan(new PrefillPlan);  // filled up to n_items / n_seqs, the rest unread
+    std::vector<int> local(batch, -1);
+    size_t pos = 0;
+    while (pos < items.size()) {
+        PrefillPlan &P = *plan;
+        P.n_items = 0;
+        P.hkv = hkv;
+        P.window = window;
+        int n_seq = 0;
+        std::vector<int> used;
+        while (pos < items.size() && P.n_items < kPlanMaxItems) {
+            const TileItem &it = items[pos];
+            if (local[it.seq] < 0) {
+                if (n_seq == kPlanMaxSeqs) break;
+                local[it.seq] = n_seq;
+                P.seq_start[n_seq] = seq_start[it.seq];
+                P.seq_len[n_seq] = seqlens[it.seq];
+                used.push_back(it.seq);
+                ++n_seq;
+            }
+            P.items[P.n_items++] = (static_cast<uint32_t>(local[it.seq]) << kItemSeqShift) |
+                                   static_cast<uint32_t>(it.qt);
+            ++pos;
+        }
+        for (int s : used) local[s] = -1;
+        P.n_seqs = n_seq;
+        if (!launch(P)) return false;
+    }
+    return true;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace of the backward: dH of the signal and noise heads (bf16) and the row statistics.
+struct BwdWorkspace {
+    size_t dh_sig, dh_noise, stats, total;
+};
+BwdWorkspace bwd_workspace(long long n, int hkv) {
+    BwdWorkspace w;
+    w.dh_sig = 0;
+    w.dh_noise = align256(static_cast<size_t>(n) * 4 * hkv * 128 * 2);
+    w.stats = w.dh_noise + align256(static_cast<size_t>(n) * hkv * 128 * 2);
+    w.total = w.stats + align256(static_cast<size_t>(n) * hkv * kBwdStats * 4);
+    return w;
+}
 
 }  // namespace
 
@@ -234,6 +314,93 @@ gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, const void *
         P.n_seqs = n_seq;
         if (launch_prefill(L, P, static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDLA_ERR_CUDA;
     }
+    return GDLA_OK;
+}
+
+size_t gdla_attn_bwd_workspace_bytes(long long total_tokens, int num_kv_heads) {
+    if (total_tokens < 0 || total_tokens >= (1ll << 31) || num_kv_heads < 1 || num_kv_heads > GDLA_MAX_KV_HEADS)
+        return 0;
+    return bwd_workspace(total_tokens, num_kv_heads).total;
+}
+
+gdla_status_t gdla_attn_bwd(const void *q_sig, const void *q_noise, const void *k, const void *v,
+                            const float *lambda, const void *gate_logits, const void *dout, void *dq_sig,
+                            void *dq_noise, void *dk, void *dv, float *dlambda, void *dgate, int batch,
+                            const int32_t *seqlens, int num_kv_heads, int window, void *workspace,
+                            size_t workspace_bytes, void *stream) {
+    if (batch < 1 || seqlens == nullptr) return GDLA_ERR_INVALID_ARG;
+    if (num_kv_heads < 1 || num_kv_heads > GDLA_MAX_KV_HEADS) return GDLA_ERR_UNSUPPORTED;
+    long long n_total = 0;
+    for (int b = 0; b < batch; ++b) {
+        if (seqlens[b] < 0) return GDLA_ERR_INVALID_ARG;
+        n_total += seqlens[b];
+    }
+    if (n_total >= (1ll << 31)) return GDLA_ERR_INVALID_ARG;
+    if (n_total == 0) return GDLA_OK;
+    if (!aligned16(q_sig) || !aligned16(q_noise) || !aligned16(k) || !aligned16(v) || !aligned16(lambda) ||
+        !aligned16(gate_logits) || !aligned16(dout) || !aligned16(dq_sig) || !aligned16(dq_noise) ||
+        !aligned16(dk) || !aligned16(dv) || !aligned16(dlambda) || !aligned16(dgate))
+        return GDLA_ERR_INVALID_ARG;
+    const int hkv = num_kv_heads;
+    const BwdWorkspace ws = bwd_workspace(n_total, hkv);
+    if (workspace == nullptr || workspace_bytes < ws.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return GDLA_ERR_WORKSPACE;
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    __nv_bfloat16 *dh_sig = reinterpret_cast<__nv_bfloat16 *>(wsb + ws.dh_sig);
+    __nv_bfloat16 *dh_noise = reinterpret_cast<__nv_bfloat16 *>(wsb + ws.dh_noise);
+    float *stats = reinterpret_cast<float *>(wsb + ws.stats);
+    const uint64_t N = static_cast<uint64_t>(n_total);
+    const int TQ = kPrefillTileTokens / 4;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // 1. forward recompute: dgate, dlambda, dH, row statistics (24-token items, 128-key tiles)
+    PrefillLaunch F{};
+    if (!make_map(&F.tm_qs, q_sig, 192, 4 * hkv, N, 64, 4, TQ) || !make_map(&F.tm_qn, q_noise, 192, hkv, N, 64, 1, TQ) ||
+        !make_map(&F.tm_k, k, 192, hkv, N, 64, 1, 128) || !make_map(&F.tm_v, v, 128, hkv, N, 64, 1, 128))
+        return GDLA_ERR_CUDA;
+    F.lambda = lambda;
+    F.gate = static_cast<const __nv_bfloat16 *>(gate_logits);
+    F.bwd = {static_cast<const __nv_bfloat16 *>(dout), static_cast<__nv_bfloat16 *>(dgate), dlambda, dh_sig, dh_noise,
+             stats};
+    const int T = kPrefillTileTokens;
+    auto q_cost = [&](int key_tile) {
+        return [=](int L, int qt) {
+            const int t0 = qt * T;
+            const int lo = (window > 0) ? std::max(0, t0 - window + 1) : 0;
+            return (std::min(L, t0 + T) - lo + key_tile - 1) / key_tile;
+        };
+    };
+    if (!run_plans(batch, seqlens, hkv, window, T, q_cost(128),
+                   [&](const PrefillPlan &P) { return launch_prefill_bwd_recompute(F, P, st) == cudaSuccess; }))
+        return GDLA_ERR_CUDA;
+
+    // 2. dQ (24-token items over 64-key tiles) and 3. dK, dV (128-key items over 12-token steps)
+    BwdLaunch B{};
+    if (!make_map(&B.tm_qs, q_sig, 192, 4 * hkv, N, 64, 4, TQ) || !make_map(&B.tm_qn, q_noise, 192, hkv, N, 64, 1, TQ) ||
+        !make_map(&B.tm_dhs, dh_sig, 128, 4 * hkv, N, 64, 4, TQ) ||
+        !make_map(&B.tm_dhn, dh_noise, 128, hkv, N, 64, 1, TQ) ||
+        !make_map(&B.tm_k64, k, 192, hkv, N, 64, 1, kBwdQKeyTile) ||
+        !make_map(&B.tm_v64, v, 128, hkv, N, 64, 1, kBwdQKeyTile) ||
+        !make_map(&B.tm_k128, k, 192, hkv, N, 64, 1, kBwdKeyTile) ||
+        !make_map(&B.tm_v128, v, 128, hkv, N, 64, 1, kBwdKeyTile) ||
+        !make_map_f32_3d(&B.tm_stats, stats, kBwdStats, hkv, N, kBwdStats, 1, kBwdStepTokens))
+        return GDLA_ERR_CUDA;
+    B.stats = stats;
+    B.dq_sig = static_cast<__nv_bfloat16 *>(dq_sig);
+    B.dq_noise = static_cast<__nv_bfloat16 *>(dq_noise);
+    B.dk = static_cast<__nv_bfloat16 *>(dk);
+    B.dv = static_cast<__nv_bfloat16 *>(dv);
+    if (!run_plans(batch, seqlens, hkv, window, T, q_cost(kBwdQKeyTile),
+                   [&](const PrefillPlan &P) { return launch_bwd_dq(B, P, st) == cudaSuccess; }))
+        return GDLA_ERR_CUDA;
+    auto kv_cost = [=](int L, int kt) {
+        const int u0 = kt * kBwdKeyTile;
+        const int t_end = (window > 0) ? std::min(L, u0 + kBwdKeyTile - 1 + window) : L;
+        return (t_end - u0 + kBwdStepTokens - 1) / kBwdStepTokens;
+    };
+    if (!run_plans(batch, seqlens, hkv, window, kBwdKeyTile, kv_cost,
+                   [&](const PrefillPlan &P) { return launch_bwd_dkv(B, P, st) == cudaSuccess; }))
+        return GDLA_ERR_CUDA;
     return GDLA_OK;
 }
 

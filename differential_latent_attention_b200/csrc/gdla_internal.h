@@ -46,15 +46,51 @@ using PrefillPlan = PrefillPlanT<kPlanMaxItems, kPlanMaxSeqs>;
 using PrefillPlanMedium = PrefillPlanT<2048, 64>;
 using PrefillPlanSmall = PrefillPlanT<768, 32>;
 
+// Backward: what the forward recompute leaves for the gradient kernels (and the
+// gradients it finishes itself). Row statistics per (token, KV group): the
+// base-2 log-sum-exp of the scaled scores of heads 0..4 (4 signal, noise) at
+// 0..4, and rowsum(dH * H) of the same heads at 8..12.
+constexpr int kBwdStats = 16;
+struct BwdIO {
+    const __nv_bfloat16 *dout;   // [N, 4H, 128]
+    __nv_bfloat16 *dgate;        // [N, 4H, 128]
+    float *dlambda;              // [N, 4H]
+    __nv_bfloat16 *dh_sig;       // [N, 4H, 128]: gradient of H_S (= dout * sigmoid(gate)), bf16
+    __nv_bfloat16 *dh_noise;     // [N, H, 128]: gradient of H_N, bf16
+    float *stats;                // [N, H, kBwdStats]
+};
+
 struct PrefillLaunch {
     CUtensorMap tm_qs, tm_qn, tm_k, tm_v;
     CUtensorMap tm_gate, tm_lam, tm_out;  // used by the asynchronous epilogue (short windows)
     const float *lambda;
     const __nv_bfloat16 *gate;
     __nv_bfloat16 *out;
+    BwdIO bwd;                            // backward recompute only
 };
 
+// Backward gradient kernels (gdla_prefill_bwd.cu). Plans: dq - items are 24-token
+// q tiles (cost: 64-key tiles visited); dkv - items are 128-key tiles (cost:
+// 12-token steps over the rows that see them).
+constexpr int kBwdQKeyTile = 64;
+constexpr int kBwdKeyTile = 128;
+constexpr int kBwdStepTokens = 12;
+struct BwdLaunch {
+    CUtensorMap tm_qs, tm_qn;       // Q boxes of 6 tokens (as the forward)
+    CUtensorMap tm_dhs, tm_dhn;     // dH boxes of 6 tokens
+    CUtensorMap tm_k64, tm_v64;     // 64-key K / V boxes (dq)
+    CUtensorMap tm_k128, tm_v128;   // 128-key K / V boxes (dkv)
+    CUtensorMap tm_stats;           // row statistics, 12 tokens of one group
+    const float *stats;
+    __nv_bfloat16 *dq_sig, *dq_noise, *dk, *dv;
+};
+cudaError_t launch_bwd_dq(const BwdLaunch &launch, const PrefillPlan &plan, cudaStream_t stream);
+cudaError_t launch_bwd_dkv(const BwdLaunch &launch, const PrefillPlan &plan, cudaStream_t stream);
+
 cudaError_t launch_prefill(const PrefillLaunch &launch, const PrefillPlan &plan, cudaStream_t stream);
+// Backward, first pass: the forward recomputed with the one-tile schedule (items of
+// kPrefillTileTokens tokens over 128-key tiles, for every window), writing launch.bwd.
+cudaError_t launch_prefill_bwd_recompute(const PrefillLaunch &launch, const PrefillPlan &plan, cudaStream_t stream);
 
 // SM count of a device, queried once per device and cached (0 on failure).
 constexpr int kMaxCachedDevices = 64;

@@ -2,6 +2,7 @@
 // device-side failure word is one symbol without relocatable device code.
 #include "gdla_api.cu"
 #include "gdla_prefill.cu"
+#include "gdla_prefill_bwd.cu"
 #include "gdla_decode.cu"
 #include "gdla_decode_noalloc.cu"
 #include "gdla_decode_latent.cu"

@@ -102,6 +102,8 @@ enum : int {
     EPI_HALF = 2,     // gate dims 0..63 and lambda staged by TMA during the item (all the
                       // shared memory left), dims 64..127 loaded by the epilogue; output
                       // stored directly
+    EPI_BWD = 3,      // backward recompute: instead of the output, the gradients of the
+                      // gate, lambda and H (from dout) and the row statistics
 };
 
 template <int TILES_, int BN_, int STAGES_, int EPI_>
@@ -111,7 +113,7 @@ struct Cfg {
     static constexpr int STAGES = STAGES_;
     static constexpr int V_BOX = BN;        // keys per V TMA box
     static constexpr int EPI = EPI_;
-    static constexpr bool ASYNC_EPI = EPI != EPI_DIRECT;  // gate / lambda staged by the producer
+    static constexpr bool ASYNC_EPI = EPI == EPI_STAGED || EPI == EPI_HALF;  // gate / lambda staged by the producer
     static constexpr int G_HALVES = EPI == EPI_STAGED ? 2 : (EPI == EPI_HALF ? 1 : 0);
     static constexpr uint32_t GATE_TX = G_HALVES * G_HALF + LAM_TILE;
     static constexpr int CTA_TOK = TILES * TOK;
@@ -146,6 +148,7 @@ struct Cfg {
     static_assert(STAGES <= 3, "three barriers each for K and V stages");
 };
 using CausalCfg = Cfg<1, 128, 2, EPI_HALF>;
+using BwdRecomputeCfg = Cfg<1, 128, 2, EPI_BWD>;  // every window: the one-tile schedule
 using SlidingCfg = Cfg<2, 64, 2, EPI_STAGED>;
 
 // ------------------------------- epilogue ----------------------------------
@@ -254,6 +257,86 @@ __device__ __forceinline__ void epi_chunk_staged(const uint32_t (&o)[32], float 
     }
 }
 
+// Backward recompute epilogue (per warp, one TMEM lane = one row): from this
+// lane's O row, l and m, the upstream gradient dout and the gate logits,
+//   sigma = sigmoid(g), D = H_S - lambda H_N,
+//   dgate = dout D sigma (1 - sigma),  dD = dout sigma,  dlambda = -sum dD H_N,
+//   dH_S = dD,  dH_N = -sum over the token's 4 signal heads of lambda dD,
+// with dH rounded to bf16 (the operand the gradient kernels multiply) and the
+// row statistics lse2 = m + log2(l) (so P = exp2(s log2(e)/sqrt(192) - lse2))
+// and rowsum(dH * H) taken with that rounded dH.
+__device__ __forceinline__ void epi_backward(uint32_t o_addr, float l_run, float m_run, bool is_sig, bool tok_valid,
+                                             int lane, int hsrc, size_t tok, int hs, int hkv, int group,
+                                             const float *__restrict__ lambda, const __nv_bfloat16 *__restrict__ gate,
+                                             const BwdIO &bwd) {
+    const bool sig = is_sig && tok_valid;
+    const bool noi = lane >= 24 && lane < 30 && tok_valid;
+    const size_t srow = tok * hs + 4 * group + (lane & 3);
+    const size_t nrow = tok * hkv + group;
+    const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+    const float lam = sig ? __ldg(lambda + srow) : 0.f;
+    const int nsrc = ((lane - 24) * 4) & 31;  // noise lane 24+i: the first signal lane of token i
+    float dl = 0.f, drow = 0.f;
+#pragma unroll 1
+    for (int ch = 0; ch < DV / 32; ++ch) {
+        uint32_t o[32], g[16], go[16];
+        tmem_ld32(o_addr + ch * 32, o);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint4 a = make_uint4(0, 0, 0, 0), c = a;
+            if (sig) {
+                a = __ldg(reinterpret_cast<const uint4 *>(gate + srow * DV + ch * 32) + i);
+                c = __ldg(reinterpret_cast<const uint4 *>(bwd.dout + srow * DV + ch * 32) + i);
+            }
+            g[4 * i] = a.x, g[4 * i + 1] = a.y, g[4 * i + 2] = a.z, g[4 * i + 3] = a.w;
+            go[4 * i] = c.x, go[4 * i + 1] = c.y, go[4 * i + 2] = c.z, go[4 * i + 3] = c.w;
+        }
+        uint32_t w_dgate[16], w_dh[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float h0 = __uint_as_float(o[2 * i]) * inv_l, h1 = __uint_as_float(o[2 * i + 1]) * inv_l;
+            const float hn0 = __shfl_sync(0xffffffffu, h0, hsrc), hn1 = __shfl_sync(0xffffffffu, h1, hsrc);
+            const float g0 = __uint_as_float(g[i] << 16), g1 = __uint_as_float(g[i] & 0xFFFF0000u);
+            const float o0 = __uint_as_float(go[i] << 16), o1 = __uint_as_float(go[i] & 0xFFFF0000u);
+            const float s0 = 1.f / (1.f + __expf(-g0)), s1 = 1.f / (1.f + __expf(-g1));
+            const float d0 = h0 - lam * hn0, d1 = h1 - lam * hn1;
+            const float dD0 = o0 * s0, dD1 = o1 * s1;
+            w_dgate[i] = pack_bf16x2(o0 * d0 * s0 * (1.f - s0), o1 * d1 * s1 * (1.f - s1));
+            dl -= dD0 * hn0 + dD1 * hn1;
+            // dH_N: the token's 4 signal lanes (4i..4i+3) sum -lambda dD; noise lane 24+i takes it
+            float c0 = -lam * dD0, c1 = -lam * dD1;
+            c0 += __shfl_xor_sync(0xffffffffu, c0, 1);
+            c1 += __shfl_xor_sync(0xffffffffu, c1, 1);
+            c0 += __shfl_xor_sync(0xffffffffu, c0, 2);
+            c1 += __shfl_xor_sync(0xffffffffu, c1, 2);
+            const float n0 = __shfl_sync(0xffffffffu, c0, nsrc), n1 = __shfl_sync(0xffffffffu, c1, nsrc);
+            const uint32_t dh = is_sig ? pack_bf16x2(dD0, dD1) : pack_bf16x2(n0, n1);
+            w_dh[i] = dh;
+            drow += __uint_as_float(dh << 16) * h0 + __uint_as_float(dh & 0xFFFF0000u) * h1;
+        }
+        if (sig) {
+            uint4 *dg = reinterpret_cast<uint4 *>(bwd.dgate + srow * DV + ch * 32);
+            uint4 *dh = reinterpret_cast<uint4 *>(bwd.dh_sig + srow * DV + ch * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                dg[i] = make_uint4(w_dgate[4 * i], w_dgate[4 * i + 1], w_dgate[4 * i + 2], w_dgate[4 * i + 3]);
+                dh[i] = make_uint4(w_dh[4 * i], w_dh[4 * i + 1], w_dh[4 * i + 2], w_dh[4 * i + 3]);
+            }
+        } else if (noi) {
+            uint4 *dh = reinterpret_cast<uint4 *>(bwd.dh_noise + nrow * DV + ch * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                dh[i] = make_uint4(w_dh[4 * i], w_dh[4 * i + 1], w_dh[4 * i + 2], w_dh[4 * i + 3]);
+        }
+    }
+    if (sig) bwd.dlambda[srow] = dl;
+    if (sig || noi) {
+        float *st = bwd.stats + nrow * kBwdStats + (sig ? (lane & 3) : 4);
+        st[0] = m_run + log2f(l_run);
+        st[8] = drow;
+    }
+}
+
 }  // namespace pf
 
 template <class C, class Plan>
@@ -262,7 +345,7 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_gate, const __grid_constant__ CUtensorMap tm_lam,
                     const __grid_constant__ CUtensorMap tm_out, const float *__restrict__ lambda,
-                    const __nv_bfloat16 *__restrict__ gate, __nv_bfloat16 *__restrict__ out,
+                    const __nv_bfloat16 *__restrict__ gate, __nv_bfloat16 *__restrict__ out, const BwdIO bwd,
                     const __grid_constant__ Plan plan) {
     using namespace pf;
     constexpr int TILES = C::TILES, BN = C::BN, STAGES = C::STAGES;
@@ -755,6 +838,15 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                     tmem_ld32(o_addr + ch * 32, o);
                     epi_chunk(o, inv_l, lam, gw[ch - 2], hsrc, valid, wide, out + row * DV + ch * 32);
                 }
+            } else if constexpr (C::EPI == EPI_BWD) {
+                if (!__all_sync(0xffffffffu, mbar_wait(o_final + x, n_item & 1, abort_flag, ERR_SITE_PREFILL | 9))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const size_t tok = static_cast<size_t>(it.s0 + t);
+                epi_backward(o_addr, l_run, m_run, is_sig, t < it.L, lane, hsrc, tok, hs, hkv, it.group, lambda, gate,
+                             bwd);
             } else {
                 // Signal rows fetch their gate row and lambda before waiting for the last PV.
                 uint32_t gw[DV / 32][16];
@@ -818,7 +910,7 @@ static cudaError_t launch_cfg(const PrefillLaunch &L, const Plan &plan, int dev,
     const long long work = static_cast<long long>(plan.n_items) * plan.hkv;
     const unsigned grid = static_cast<unsigned>(work < num_sms ? work : num_sms);
     gdla_prefill_kernel<C, Plan><<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(
-        L.tm_qs, L.tm_qn, L.tm_k, L.tm_v, L.tm_gate, L.tm_lam, L.tm_out, L.lambda, L.gate, L.out, plan);
+        L.tm_qs, L.tm_qn, L.tm_k, L.tm_v, L.tm_gate, L.tm_lam, L.tm_out, L.lambda, L.gate, L.out, L.bwd, plan);
     return cudaPeekAtLastError();
 }
 
@@ -847,6 +939,15 @@ static cudaError_t launch_sized(const PrefillLaunch &L, const PrefillPlan &plan,
         return launch_cfg<C>(L, medium, dev, num_sms, stream);
     }
     return launch_cfg<C>(L, plan, dev, num_sms, stream);
+}
+
+cudaError_t launch_prefill_bwd_recompute(const PrefillLaunch &L, const PrefillPlan &plan, cudaStream_t stream) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int num_sms = device_sm_count(dev);
+    if (num_sms <= 0) return cudaErrorInvalidDevice;
+    return launch_sized<pf::BwdRecomputeCfg>(L, plan, dev, num_sms, stream);
 }
 
 cudaError_t launch_prefill(const PrefillLaunch &L, const PrefillPlan &plan, cudaStream_t stream) {

@@ -1,0 +1,710 @@
+// gdla_prefill_bwd.cu - GDLA prefill backward: the attention gradients, for sm_100a.
+//
+// Method (aitrends.kr/articles/94908, GDLA paragraphs: 4 signal + 1 noise
+// query heads per KV group over one K_j, V_j; D = H_S - lambda H_N; sigmoid
+// gate). The forward recompute (gdla_prefill.cu, backward epilogue) leaves per
+// row the gradient dH of the head output H (bf16), lse2 = log2 of the softmax
+// denominator in the scaled base-2 units the kernels use, and rowsum(dH * H).
+// With P = exp2(S c - lse2), c = log2(e)/sqrt(192), for each head h over the
+// shared K_j, V_j:
+//     dP = dH V^T,   dS = P (dP - rowsum(dH H)),
+//     dQ_h = dS K / sqrt(192),   dK_j = sum_h dS^T Q_h / sqrt(192),   dV_j = sum_h P^T dH_h.
+// Rows keep the forward's tile layout: 24 tokens x 5 heads in the 128 lanes of
+// a tile, per TMEM lane quarter w tokens 6w..6w+5 as rows 32w+4i+h (signal head
+// h of token 6w+i), 32w+24+i (noise head), 32w+30..31 unused (zero).
+//
+// Two kernels, no atomics (deterministic):
+//   dq kernel   - item (KV group, 24-token q tile), loop over its 64-key tiles:
+//                 S = Q K^T and dP = dH V^T (tcgen05, M=128 rows, N=64 keys),
+//                 dS by the 4 row warps into TMEM, dQ += dS K (A = dS from TMEM,
+//                 B = the K tile read keys-major, N=192).
+//   dkv kernel  - item (KV group, 128-key tile), loop over the 12-token halves
+//                 of q tiles that see it: S^T = K Q^T and dP^T = V dH^T
+//                 (M=128 keys, N=64 rows), P^T and dS^T by the 4 key warps into
+//                 TMEM, dV += P^T dH and dK += dS^T Q (A from TMEM, B the row
+//                 tile read rows-major).
+// Each output row (dq of a token and head, dk / dv of a key) is owned by one
+// CTA and written once.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstring>
+
+#include "gdla_internal.h"
+#include "gdla_ptx.cuh"
+
+namespace gdla {
+
+namespace pb {
+constexpr int TOK = kPrefillTileTokens;  // 24
+constexpr int DQK = 192, DV = 128;
+constexpr int ROW_BOX = TOK / 4;         // 6 tokens per TMA box (one lane quarter)
+constexpr uint32_t QBOX_TX = 64 * 4 * ROW_BOX * 2 + 64 * 1 * ROW_BOX * 2;  // one quarter's rows of one 64-dim chunk
+constexpr float kScoreLog2 = 0.07216878364870322f * 1.4426950408889634f;  // log2(e) / sqrt(192)
+constexpr float kInvRoot = 0.07216878364870322f;                         // 1 / sqrt(192)
+constexpr int NUM_THREADS = 192;  // 4 row/key warps, producer warp 4, MMA warp 5
+constexpr int PRODUCER_WARP = 4, MMA_WARP = 5;
+
+// (row of a 32-row lane quarter) -> token offset in the quarter, head (0..3 signal, 4 noise), padding
+__host__ __device__ constexpr int quarter_token(int within) { return within < 24 ? within >> 2 : within - 24; }
+__host__ __device__ constexpr int quarter_head(int within) { return within < 24 ? (within & 3) : 4; }
+}  // namespace pb
+
+// ------------------------------------------------------------------------------
+// dQ
+// ------------------------------------------------------------------------------
+namespace pbq {
+using namespace pb;
+constexpr int BN = 64;                     // keys per tile
+constexpr int STAGES = 2;
+constexpr int Q_CHUNK = 128 * 128;         // 128 rows x 64 dims
+constexpr int Q_BYTES = 3 * Q_CHUNK;       // 48 KB
+constexpr int DH_BYTES = 2 * Q_CHUNK;      // 32 KB
+constexpr int KV_CHUNK = BN * 128;         // 64 keys x 64 dims: 8 KB
+constexpr int K_STAGE = 3 * KV_CHUNK;
+constexpr int V_STAGE = 2 * KV_CHUNK;
+constexpr int STAGE = K_STAGE + V_STAGE;   // 40 KB
+constexpr int OFF_Q = 0;
+constexpr int OFF_DH = OFF_Q + Q_BYTES;
+constexpr int OFF_KV = OFF_DH + DH_BYTES;
+constexpr int OFF_BAR = OFF_KV + STAGES * STAGE;
+constexpr int OFF_MISC = OFF_BAR + 16 * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
+constexpr uint32_t QD_TX = (3 + 2) * 4 * QBOX_TX;  // Q and dH tiles of one item
+constexpr uint32_t DQ_COL = 0, S_COL = 192, DP_COL = 256;
+constexpr uint32_t TMEM_COLS = 512;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+}  // namespace pbq
+
+template <class Plan>
+__global__ void __launch_bounds__(pb::NUM_THREADS, 1)
+gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_qn,
+                   const __grid_constant__ CUtensorMap tm_dhs, const __grid_constant__ CUtensorMap tm_dhn,
+                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const float *__restrict__ stats, __nv_bfloat16 *__restrict__ dq_sig,
+                   __nv_bfloat16 *__restrict__ dq_noise, const __grid_constant__ Plan plan) {
+    using namespace pbq;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint64_t *q_full = bars + 0;    // one phase per item: Q and dH tiles landed
+    uint64_t *q_empty = bars + 1;   // one phase per item: its last S / dP products are done
+    uint64_t *kv_full = bars + 2;   // [stage]
+    uint64_t *kv_empty = bars + 4;  // [stage]
+    uint64_t *s_full = bars + 6;    // one phase per key tile: S and dP in TMEM
+    uint64_t *ds_full = bars + 7;   // one phase per key tile: dS in TMEM (128 arrivals)
+    uint64_t *dq_final = bars + 8;  // one phase per item: its last dQ product is done
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int hkv = plan.hkv, hs = 4 * hkv, window = plan.window;
+    const int n_work = plan.n_items * hkv;
+
+    struct Item {
+        int group, s0, L, t0, kv_lo, n_tiles;
+    };
+    auto item_at = [&](int w) {
+        Item it;
+        it.group = w % hkv;
+        const uint32_t code = plan.items[w / hkv];
+        const int seq = static_cast<int>(code >> kItemSeqShift);
+        it.s0 = plan.seq_start[seq];
+        it.L = plan.seq_len[seq];
+        it.t0 = static_cast<int>(code & kItemTileMask) * TOK;
+        it.kv_lo = (window > 0) ? max(0, it.t0 - window + 1) : 0;
+        it.n_tiles = max(1, (min(it.L, it.t0 + TOK) - it.kv_lo + BN - 1) / BN);
+        return it;
+    };
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(kv_full + i, 1);
+            mbar_init(kv_empty + i, 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(ds_full, 128);
+        mbar_init(dq_final, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == PRODUCER_WARP) {
+        // rows 32w+30, 32w+31 of the Q and dH tiles are never loaded: zero them once
+        for (int c = 0; c < 5; ++c)
+            for (int i = lane; i < 4 * 2 * 8; i += 32) {
+                const int row = 32 * (i >> 4) + 30 + ((i >> 3) & 1);
+                reinterpret_cast<uint4 *>(smem + OFF_Q + c * Q_CHUNK + row * 128)[i & 7] = make_uint4(0, 0, 0, 0);
+            }
+        fence_proxy_async_smem();
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == PRODUCER_WARP) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            int kv = 0, issued = 0, n_item = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+                const Item it = item_at(w);
+                if (n_item > 0 && !mbar_wait(q_empty, (n_item - 1) & 1, abort_flag, ERR_SITE_BWD | 1)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(q_full, QD_TX);
+                const int row0 = it.s0 + it.t0;
+                for (int q = 0; q < 4; ++q) {
+                    for (int c = 0; c < 3; ++c) {
+                        uint8_t *dst = smem + OFF_Q + c * Q_CHUNK + 32 * q * 128;
+                        tma_load_3d(dst, &tm_qs, q_full, c * 64, 4 * it.group, row0 + 6 * q);
+                        tma_load_3d(dst + 24 * 128, &tm_qn, q_full, c * 64, it.group, row0 + 6 * q);
+                    }
+                    for (int c = 0; c < 2; ++c) {
+                        uint8_t *dst = smem + OFF_DH + c * Q_CHUNK + 32 * q * 128;
+                        tma_load_3d(dst, &tm_dhs, q_full, c * 64, 4 * it.group, row0 + 6 * q);
+                        tma_load_3d(dst + 24 * 128, &tm_dhn, q_full, c * 64, it.group, row0 + 6 * q);
+                    }
+                }
+                for (int k = 0; k < it.n_tiles; ++k, ++kv) {
+                    const int st = kv % STAGES;
+                    if (kv >= STAGES &&
+                        !mbar_wait(kv_empty + st, ((kv / STAGES) + 1) & 1, abort_flag, ERR_SITE_BWD | 2)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(kv_full + st, STAGE);
+                    const int row = it.s0 + it.kv_lo + k * BN;
+                    uint8_t *sb = smem + OFF_KV + st * STAGE;
+                    for (int c = 0; c < 3; ++c) tma_load_3d(sb + c * KV_CHUNK, &tm_k, kv_full + st, c * 64, it.group, row);
+                    for (int c = 0; c < 2; ++c)
+                        tma_load_3d(sb + K_STAGE + c * KV_CHUNK, &tm_v, kv_full + st, c * 64, it.group, row);
+                    issued = kv + 1;
+                }
+            }
+            if (*abort_flag) {
+                for (int k = max(0, issued - STAGES); k < issued; ++k)
+                    mbar_wait_cycles(kv_full + k % STAGES, (k / STAGES) & 1, 1ll << 22);
+                mbar_wait_cycles(q_full, (n_item & 1) ^ 1, 1ll << 22);
+            }
+        }
+    } else if (warp == MMA_WARP) {
+        // ------------------------------ MMA issuer --------------------------------
+        // Per key tile: S, dP, (dS from the row warps), dQ. The next tile's S and dP
+        // overwrite dS / dP only after this tile's dQ read them (one issuing thread,
+        // executed in order).
+        const uint32_t leader = elect_one_sync();
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, false, false);
+        constexpr uint32_t idesc_q = idesc_bf16_f32(128, DQK, false, true);
+        const uint64_t q_desc0 = desc_sw128(smem_u32(smem + OFF_Q), 16, 1024);
+        const uint64_t dh_desc0 = desc_sw128(smem_u32(smem + OFF_DH), 16, 1024);
+        const uint64_t kv_desc0 = desc_sw128(smem_u32(smem + OFF_KV), 16, 1024);        // K, V as B (keys x dims)
+        const uint64_t kmn_desc0 = desc_sw128(smem_u32(smem + OFF_KV), KV_CHUNK, 1024);  // K as B (dims x keys)
+        int kv = 0, step = 0, n_item = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+            const Item it = item_at(w);
+            if (!__all_sync(0xffffffffu, mbar_wait(q_full, n_item & 1, abort_flag, ERR_SITE_BWD | 3))) break;
+            for (int k = 0; k < it.n_tiles; ++k, ++kv, ++step) {
+                const int st = kv % STAGES;
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(kv_full + st, (kv / STAGES) & 1, abort_flag, ERR_SITE_BWD | 4))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sbase = st * STAGE;
+#pragma unroll
+                for (int kk = 0; kk < DQK / 16; ++kk) {
+                    const uint32_t offq = ((kk >> 2) * Q_CHUNK + (kk & 3) * 32) >> 4;
+                    const uint32_t offk = (sbase + (kk >> 2) * KV_CHUNK + (kk & 3) * 32) >> 4;
+                    umma_ss_leader(tmem + S_COL, q_desc0 + offq, kv_desc0 + offk, idesc_s, kk > 0, leader);
+                }
+#pragma unroll
+                for (int kk = 0; kk < DV / 16; ++kk) {
+                    const uint32_t offd = ((kk >> 2) * Q_CHUNK + (kk & 3) * 32) >> 4;
+                    const uint32_t offv = (sbase + K_STAGE + (kk >> 2) * KV_CHUNK + (kk & 3) * 32) >> 4;
+                    umma_ss_leader(tmem + DP_COL, dh_desc0 + offd, kv_desc0 + offv, idesc_s, kk > 0, leader);
+                }
+                umma_commit_leader(s_full, leader);
+                if (k == it.n_tiles - 1) umma_commit_leader(q_empty, leader);
+                if (!__all_sync(0xffffffffu, mbar_wait(ds_full, step & 1, abort_flag, ERR_SITE_BWD | 5))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk)
+                    umma_ts_leader(tmem + DQ_COL, tmem + S_COL + kk * 8, kmn_desc0 + ((sbase + kk * 2048) >> 4),
+                                   idesc_q, (k > 0 || kk > 0) ? 1u : 0u, leader);
+                umma_commit_leader(kv_empty + st, leader);
+                if (k == it.n_tiles - 1) umma_commit_leader(dq_final, leader);
+            }
+        }
+    } else {
+        // ------------------------------ row warps ---------------------------------
+        const bool is_sig = lane < 24;
+        const int tau = 6 * warp + pb::quarter_token(lane);
+        const int head = pb::quarter_head(lane);
+        const bool pad_row = lane >= 30;
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        int step = 0, n_item = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+            const Item it = item_at(w);
+            const int t = it.t0 + tau;
+            const bool row_ok = !pad_row && t < it.L;
+            const size_t srow = static_cast<size_t>(it.s0 + t) * hkv + it.group;  // (token, group)
+            float lse2 = 0.f, drow = 0.f;
+            if (row_ok) {
+                lse2 = __ldg(stats + srow * kBwdStats + head);
+                drow = __ldg(stats + srow * kBwdStats + 8 + head);
+            }
+            for (int k = 0; k < it.n_tiles; ++k, ++step) {
+                if (!__all_sync(0xffffffffu, mbar_wait(s_full, step & 1, abort_flag, ERR_SITE_BWD | 6))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t sr[64], dr[64];
+                tmem_ld64(lane_base + S_COL, sr);
+                tmem_ld64(lane_base + DP_COL, dr);
+                const int u0 = it.kv_lo + k * BN;
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float ds2[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int u = u0 + 2 * i + e;
+                        const bool vis = row_ok && u <= t && (window <= 0 || u > t - window);
+                        const float p = fast_exp2(__uint_as_float(sr[2 * i + e]) * kScoreLog2 - lse2);
+                        ds2[e] = vis ? p * (__uint_as_float(dr[2 * i + e]) - drow) : 0.f;
+                    }
+                    pk[i] = pack_bf16x2(ds2[0], ds2[1]);
+                }
+                tmem_st32(lane_base + S_COL, pk);
+                tc_fence_before();
+                mbar_arrive(ds_full);
+            }
+            if (!ok) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(dq_final, n_item & 1, abort_flag, ERR_SITE_BWD | 7))) break;
+            tc_fence_after();
+            __nv_bfloat16 *dst = is_sig ? dq_sig + ((static_cast<size_t>(it.s0 + t) * hs + 4 * it.group + head) * DQK)
+                                        : dq_noise + srow * DQK;
+#pragma unroll 1
+            for (int ch = 0; ch < DQK / 32; ++ch) {
+                uint32_t o[32];
+                tmem_ld32(lane_base + DQ_COL + ch * 32, o);
+                if (row_ok) {
+                    uint32_t wds[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        wds[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * kInvRoot, __uint_as_float(o[2 * i + 1]) * kInvRoot);
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dst + ch * 32);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) d4[i] = make_uint4(wds[4 * i], wds[4 * i + 1], wds[4 * i + 2], wds[4 * i + 3]);
+                }
+            }
+            // dQ is read before the next item's first dQ product overwrites it: that
+            // product waits for these warps' ds_full of the next item's first tile.
+            tc_fence_before();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------------------
+// dK, dV
+// ------------------------------------------------------------------------------
+namespace pbk {
+using namespace pb;
+constexpr int BK = 128;                    // keys per item
+constexpr int HT = 12;                     // tokens per step (half a q tile: 64 rows)
+constexpr int STAGES = 3;
+constexpr int K_CHUNK = BK * 128;          // 128 keys x 64 dims: 16 KB
+constexpr int K_BYTES = 3 * K_CHUNK;
+constexpr int V_BYTES = 2 * K_CHUNK;
+constexpr int H_CHUNK = 64 * 128;          // 64 rows x 64 dims: 8 KB
+constexpr int QH_BYTES = 3 * H_CHUNK;
+constexpr int DHH_BYTES = 2 * H_CHUNK;
+constexpr int STATS_BYTES = HT * kBwdStats * 4;  // 768 B
+constexpr int STAGE = QH_BYTES + DHH_BYTES + 1024;  // 41 KB (stats in the last 1 KB)
+constexpr int OFF_K = 0;
+constexpr int OFF_V = OFF_K + K_BYTES;
+constexpr int OFF_ST = OFF_V + V_BYTES;
+constexpr int OFF_BAR = OFF_ST + STAGES * STAGE;
+constexpr int OFF_MISC = OFF_BAR + 16 * 8;
+constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
+constexpr uint32_t KV_TX = K_BYTES + V_BYTES;
+constexpr uint32_t STEP_TX = (3 + 2) * 2 * QBOX_TX + STATS_BYTES;
+constexpr uint32_t DK_COL = 0, DV_COL = 192, ST_COL = 320, DPT_COL = 384;
+constexpr uint32_t TMEM_COLS = 512;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+}  // namespace pbk
+
+template <class Plan>
+__global__ void __launch_bounds__(pb::NUM_THREADS, 1)
+gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_qn,
+                    const __grid_constant__ CUtensorMap tm_dhs, const __grid_constant__ CUtensorMap tm_dhn,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_stats, __nv_bfloat16 *__restrict__ dk,
+                    __nv_bfloat16 *__restrict__ dv, const __grid_constant__ Plan plan) {
+    using namespace pbk;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint64_t *kv_full = bars + 0;    // one phase per item: the K and V tiles landed
+    uint64_t *kv_empty = bars + 1;   // one phase per item: its last products are done
+    uint64_t *st_full = bars + 2;    // [stage]: Q, dH halves and row statistics of a step
+    uint64_t *st_empty = bars + 5;   // [stage]
+    uint64_t *s_full = bars + 8;     // one phase per step: S^T and dP^T in TMEM
+    uint64_t *pds_full = bars + 9;   // one phase per step: P^T and dS^T in TMEM (128 arrivals)
+    uint64_t *dkv_final = bars + 10; // one phase per item
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int hkv = plan.hkv, window = plan.window;
+    const int n_work = plan.n_items * hkv;
+
+    // Item: keys u0..u0+127 of one sequence; steps: 12-token halves from u0 to the
+    // last token that sees one of the keys.
+    struct Item {
+        int group, s0, L, u0, n_steps;
+    };
+    auto item_at = [&](int w) {
+        Item it;
+        it.group = w % hkv;
+        const uint32_t code = plan.items[w / hkv];
+        const int seq = static_cast<int>(code >> kItemSeqShift);
+        it.s0 = plan.seq_start[seq];
+        it.L = plan.seq_len[seq];
+        it.u0 = static_cast<int>(code & kItemTileMask) * BK;
+        const int t_end = (window > 0) ? min(it.L, it.u0 + BK - 1 + window) : it.L;
+        it.n_steps = max(1, (t_end - it.u0 + HT - 1) / HT);
+        return it;
+    };
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        mbar_init(kv_empty, 1);
+        for (int i = 0; i < STAGES; ++i) {
+            mbar_init(st_full + i, 1);
+            mbar_init(st_empty + i, 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(pds_full, 128);
+        mbar_init(dkv_final, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == PRODUCER_WARP) {
+        // rows 32q+30, 32q+31 of every stage's Q and dH halves are never loaded: zero them once
+        for (int st = 0; st < STAGES; ++st)
+            for (int c = 0; c < 5; ++c)
+                for (int i = lane; i < 2 * 2 * 8; i += 32) {
+                    const int row = 32 * (i >> 4) + 30 + ((i >> 3) & 1);
+                    reinterpret_cast<uint4 *>(smem + OFF_ST + st * STAGE + c * H_CHUNK + row * 128)[i & 7] =
+                        make_uint4(0, 0, 0, 0);
+                }
+        fence_proxy_async_smem();
+    }
+    if (warp == MMA_WARP) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == PRODUCER_WARP) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            int g = 0, issued = 0, n_item = 0;
+            bool ok = true;
+            for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+                const Item it = item_at(w);
+                if (n_item > 0 && !mbar_wait(kv_empty, (n_item - 1) & 1, abort_flag, ERR_SITE_BWD | 11)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(kv_full, KV_TX);
+                for (int c = 0; c < 3; ++c)
+                    tma_load_3d(smem + OFF_K + c * K_CHUNK, &tm_k, kv_full, c * 64, it.group, it.s0 + it.u0);
+                for (int c = 0; c < 2; ++c)
+                    tma_load_3d(smem + OFF_V + c * K_CHUNK, &tm_v, kv_full, c * 64, it.group, it.s0 + it.u0);
+                for (int s = 0; s < it.n_steps; ++s, ++g) {
+                    const int st = g % STAGES;
+                    if (g >= STAGES && !mbar_wait(st_empty + st, ((g / STAGES) + 1) & 1, abort_flag, ERR_SITE_BWD | 12)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(st_full + st, STEP_TX);
+                    uint8_t *sb = smem + OFF_ST + st * STAGE;
+                    const int th = it.s0 + it.u0 + s * HT;
+                    for (int q = 0; q < 2; ++q) {
+                        for (int c = 0; c < 3; ++c) {
+                            uint8_t *dst = sb + c * H_CHUNK + 32 * q * 128;
+                            tma_load_3d(dst, &tm_qs, st_full + st, c * 64, 4 * it.group, th + 6 * q);
+                            tma_load_3d(dst + 24 * 128, &tm_qn, st_full + st, c * 64, it.group, th + 6 * q);
+                        }
+                        for (int c = 0; c < 2; ++c) {
+                            uint8_t *dst = sb + QH_BYTES + c * H_CHUNK + 32 * q * 128;
+                            tma_load_3d(dst, &tm_dhs, st_full + st, c * 64, 4 * it.group, th + 6 * q);
+                            tma_load_3d(dst + 24 * 128, &tm_dhn, st_full + st, c * 64, it.group, th + 6 * q);
+                        }
+                    }
+                    tma_load_3d(sb + QH_BYTES + DHH_BYTES, &tm_stats, st_full + st, 0, it.group, th);
+                    issued = g + 1;
+                }
+            }
+            if (*abort_flag) {
+                for (int k = max(0, issued - STAGES); k < issued; ++k)
+                    mbar_wait_cycles(st_full + k % STAGES, (k / STAGES) & 1, 1ll << 22);
+                mbar_wait_cycles(kv_full, (n_item & 1) ^ 1, 1ll << 22);
+            }
+        }
+    } else if (warp == MMA_WARP) {
+        // ------------------------------ MMA issuer --------------------------------
+        const uint32_t leader = elect_one_sync();
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
+        constexpr uint32_t idesc_v = idesc_bf16_f32(128, DV, false, true);
+        constexpr uint32_t idesc_k = idesc_bf16_f32(128, DQK, false, true);
+        const uint64_t k_desc0 = desc_sw128(smem_u32(smem + OFF_K), 16, 1024);
+        const uint64_t v_desc0 = desc_sw128(smem_u32(smem + OFF_V), 16, 1024);
+        const uint64_t st_desc0 = desc_sw128(smem_u32(smem + OFF_ST), 16, 1024);        // Q, dH halves as B (rows x dims)
+        const uint64_t stmn_desc0 = desc_sw128(smem_u32(smem + OFF_ST), H_CHUNK, 1024);  // as B (dims x rows)
+        int g = 0, n_item = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+            const Item it = item_at(w);
+            if (!__all_sync(0xffffffffu, mbar_wait(kv_full, n_item & 1, abort_flag, ERR_SITE_BWD | 13))) break;
+            for (int s = 0; s < it.n_steps; ++s, ++g) {
+                const int st = g % STAGES;
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(st_full + st, (g / STAGES) & 1, abort_flag, ERR_SITE_BWD | 14))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sbase = st * STAGE;
+#pragma unroll
+                for (int kk = 0; kk < DQK / 16; ++kk) {
+                    const uint32_t offk = ((kk >> 2) * K_CHUNK + (kk & 3) * 32) >> 4;
+                    const uint32_t offq = (sbase + (kk >> 2) * H_CHUNK + (kk & 3) * 32) >> 4;
+                    umma_ss_leader(tmem + ST_COL, k_desc0 + offk, st_desc0 + offq, idesc_s, kk > 0, leader);
+                }
+#pragma unroll
+                for (int kk = 0; kk < DV / 16; ++kk) {
+                    const uint32_t offv = ((kk >> 2) * K_CHUNK + (kk & 3) * 32) >> 4;
+                    const uint32_t offd = (sbase + QH_BYTES + (kk >> 2) * H_CHUNK + (kk & 3) * 32) >> 4;
+                    umma_ss_leader(tmem + DPT_COL, v_desc0 + offv, st_desc0 + offd, idesc_s, kk > 0, leader);
+                }
+                umma_commit_leader(s_full, leader);
+                if (!__all_sync(0xffffffffu, mbar_wait(pds_full, g & 1, abort_flag, ERR_SITE_BWD | 15))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 64 / 16; ++kk) {
+                    const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                    umma_ts_leader(tmem + DV_COL, tmem + ST_COL + kk * 8,
+                                   stmn_desc0 + ((sbase + QH_BYTES + kk * 2048) >> 4), idesc_v, acc, leader);
+                    umma_ts_leader(tmem + DK_COL, tmem + DPT_COL + kk * 8, stmn_desc0 + ((sbase + kk * 2048) >> 4),
+                                   idesc_k, acc, leader);
+                }
+                umma_commit_leader(st_empty + st, leader);
+            }
+            if (!ok) break;
+            umma_commit_leader(kv_empty, leader);
+            umma_commit_leader(dkv_final, leader);
+        }
+    } else {
+        // ------------------------------ key warps ---------------------------------
+        const int kl = warp * 32 + lane;  // key of the tile = TMEM lane
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        int g = 0, n_item = 0;
+        bool ok = true;
+        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+            const Item it = item_at(w);
+            const int u = it.u0 + kl;
+            const bool key_ok = u < it.L;
+            for (int s = 0; s < it.n_steps; ++s, ++g) {
+                const int st = g % STAGES;
+                if (!__all_sync(0xffffffffu, mbar_wait(s_full, g & 1, abort_flag, ERR_SITE_BWD | 16))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t sr[64], dr[64];
+                tmem_ld64(lane_base + ST_COL, sr);
+                tmem_ld64(lane_base + DPT_COL, dr);
+                const float *stat = reinterpret_cast<const float *>(smem + OFF_ST + st * STAGE + QH_BYTES + DHH_BYTES);
+                const int th = it.u0 + s * HT;  // first token of the step
+                uint32_t pk[32], dk2[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float pv[2], dv2[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int r = 2 * i + e;             // row of the 64-row half
+                        const int within = r & 31;
+                        const int tok = 6 * (r >> 5) + pb::quarter_token(within);
+                        const int head = pb::quarter_head(within);
+                        const int t = th + tok;
+                        const bool vis = within < 30 && key_ok && t < it.L && u <= t && (window <= 0 || u > t - window);
+                        const float lse2 = stat[tok * kBwdStats + head];
+                        const float drow = stat[tok * kBwdStats + 8 + head];
+                        const float p = fast_exp2(__uint_as_float(sr[r]) * kScoreLog2 - lse2);
+                        pv[e] = vis ? p : 0.f;
+                        dv2[e] = vis ? p * (__uint_as_float(dr[r]) - drow) : 0.f;
+                    }
+                    pk[i] = pack_bf16x2(pv[0], pv[1]);
+                    dk2[i] = pack_bf16x2(dv2[0], dv2[1]);
+                }
+                tmem_st32(lane_base + ST_COL, pk);
+                tmem_st32(lane_base + DPT_COL, dk2);
+                tc_fence_before();
+                mbar_arrive(pds_full);
+            }
+            if (!ok) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(dkv_final, n_item & 1, abort_flag, ERR_SITE_BWD | 17))) break;
+            tc_fence_after();
+            const size_t krow = static_cast<size_t>(it.s0 + u) * hkv + it.group;
+#pragma unroll 1
+            for (int ch = 0; ch < DQK / 32; ++ch) {
+                uint32_t o[32];
+                tmem_ld32(lane_base + DK_COL + ch * 32, o);
+                if (key_ok) {
+                    uint32_t wd[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        wd[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * kInvRoot, __uint_as_float(o[2 * i + 1]) * kInvRoot);
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dk + krow * DQK + ch * 32);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) d4[i] = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
+                }
+            }
+#pragma unroll 1
+            for (int ch = 0; ch < DV / 32; ++ch) {
+                uint32_t o[32];
+                tmem_ld32(lane_base + DV_COL + ch * 32, o);
+                if (key_ok) {
+                    uint32_t wd[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        wd[i] = pack_bf16x2(__uint_as_float(o[2 * i]), __uint_as_float(o[2 * i + 1]));
+                    uint4 *d4 = reinterpret_cast<uint4 *>(dv + krow * DV + ch * 32);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) d4[i] = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
+                }
+            }
+            tc_fence_before();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------------
+template <class Plan>
+static cudaError_t launch_dq_sized(const BwdLaunch &L, const Plan &plan, cudaStream_t stream) {
+    static PerContextFlag attr_set;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int num_sms = device_sm_count(dev);
+    if (num_sms <= 0) return cudaErrorInvalidDevice;
+    const unsigned long long ctx = current_context_id();
+    if (!attr_set.is_set(dev, ctx)) {
+        e = cudaFuncSetAttribute(gdla_bwd_dq_kernel<Plan>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 pbq::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set.set(dev, current_context_id());
+    }
+    const long long work = static_cast<long long>(plan.n_items) * plan.hkv;
+    const unsigned grid = static_cast<unsigned>(work < num_sms ? work : num_sms);
+    gdla_bwd_dq_kernel<Plan><<<grid, pb::NUM_THREADS, pbq::SMEM_BYTES, stream>>>(
+        L.tm_qs, L.tm_qn, L.tm_dhs, L.tm_dhn, L.tm_k64, L.tm_v64, L.stats, L.dq_sig, L.dq_noise, plan);
+    return cudaPeekAtLastError();
+}
+
+template <class Plan>
+static cudaError_t launch_dkv_sized(const BwdLaunch &L, const Plan &plan, cudaStream_t stream) {
+    static PerContextFlag attr_set;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int num_sms = device_sm_count(dev);
+    if (num_sms <= 0) return cudaErrorInvalidDevice;
+    const unsigned long long ctx = current_context_id();
+    if (!attr_set.is_set(dev, ctx)) {
+        e = cudaFuncSetAttribute(gdla_bwd_dkv_kernel<Plan>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 pbk::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set.set(dev, current_context_id());
+    }
+    const long long work = static_cast<long long>(plan.n_items) * plan.hkv;
+    const unsigned grid = static_cast<unsigned>(work < num_sms ? work : num_sms);
+    gdla_bwd_dkv_kernel<Plan><<<grid, pb::NUM_THREADS, pbk::SMEM_BYTES, stream>>>(
+        L.tm_qs, L.tm_qn, L.tm_dhs, L.tm_dhn, L.tm_k128, L.tm_v128, L.tm_stats, L.dk, L.dv, plan);
+    return cudaPeekAtLastError();
+}
+
+// The plan in the smallest capacity that holds it (kernel parameters are copied
+// with every launch).
+template <class F>
+static cudaError_t with_sized_plan(const PrefillPlan &plan, F &&launch) {
+    auto shrink = [&](auto &small) {
+        small.n_items = plan.n_items;
+        small.hkv = plan.hkv;
+        small.window = plan.window;
+        small.n_seqs = plan.n_seqs;
+        std::memcpy(small.seq_start, plan.seq_start, sizeof(int) * plan.n_seqs);
+        std::memcpy(small.seq_len, plan.seq_len, sizeof(int) * plan.n_seqs);
+        std::memcpy(small.items, plan.items, sizeof(uint32_t) * plan.n_items);
+    };
+    if (plan.n_items <= PrefillPlanSmall::kMaxItems && plan.n_seqs <= PrefillPlanSmall::kMaxSeqs) {
+        PrefillPlanSmall small;
+        shrink(small);
+        return launch(small);
+    }
+    if (plan.n_items <= PrefillPlanMedium::kMaxItems && plan.n_seqs <= PrefillPlanMedium::kMaxSeqs) {
+        PrefillPlanMedium medium;
+        shrink(medium);
+        return launch(medium);
+    }
+    return launch(plan);
+}
+
+cudaError_t launch_bwd_dq(const BwdLaunch &L, const PrefillPlan &plan, cudaStream_t stream) {
+    return with_sized_plan(plan, [&](const auto &p) { return launch_dq_sized(L, p, stream); });
+}
+
+cudaError_t launch_bwd_dkv(const BwdLaunch &L, const PrefillPlan &plan, cudaStream_t stream) {
+    return with_sized_plan(plan, [&](const auto &p) { return launch_dkv_sized(L, p, stream); });
+}
+
+}  // namespace gdla

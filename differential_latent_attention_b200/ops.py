@@ -20,7 +20,7 @@ MAX_KV_HEADS = 64
 
 STATUS = {0: "GDLA_OK", 1: "GDLA_ERR_INVALID_ARG", 2: "GDLA_ERR_UNSUPPORTED", 3: "GDLA_ERR_WORKSPACE",
           4: "GDLA_ERR_CUDA"}
-EXPORTED = ("gdla_attn_fwd", "gdla_decode_workspace_bytes", "gdla_attn_decode", "gdla_attn_decode_noalloc",
+EXPORTED = ("gdla_attn_fwd", "gdla_attn_bwd_workspace_bytes", "gdla_attn_bwd", "gdla_decode_workspace_bytes", "gdla_attn_decode", "gdla_attn_decode_noalloc",
             "gdla_decode_latent_workspace_bytes", "gdla_attn_decode_latent", "gdla_device_error",
             "gdla_selftest_wait_timeout", "gdla_status_string", "gdla_version")
 DC, DR = 512, 64
@@ -54,6 +54,10 @@ def library():
             p, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
             lib.gdla_attn_fwd.argtypes = [p, p, p, p, p, p, p, i, p, i, i, p]
             lib.gdla_attn_fwd.restype = i
+            lib.gdla_attn_bwd_workspace_bytes.argtypes = [ctypes.c_longlong, i]
+            lib.gdla_attn_bwd_workspace_bytes.restype = sz
+            lib.gdla_attn_bwd.argtypes = [p, p, p, p, p, p, p, p, p, p, p, p, p, i, p, i, i, p, sz, p]
+            lib.gdla_attn_bwd.restype = i
             lib.gdla_decode_workspace_bytes.argtypes = [i, i, i, i]
             lib.gdla_decode_workspace_bytes.restype = sz
             lib.gdla_attn_decode.argtypes = [p, p, p, p, p, i, i, p, p, p, i, i, i, p, sz, p]
@@ -130,6 +134,50 @@ def attn_fwd(q_sig, q_noise, k, v, lam, gate, seqlens, window=0, out=None, strea
     if st != 0:
         raise GDLAError(st, "gdla_attn_fwd")
     return out
+
+
+def attn_bwd_workspace_bytes(total_tokens, num_kv_heads):
+    return int(library().gdla_attn_bwd_workspace_bytes(int(total_tokens), int(num_kv_heads)))
+
+
+def attn_bwd(q_sig, q_noise, k, v, lam, gate, dout, seqlens, window=0, grads=None, workspace=None, stream=None):
+    """Packed varlen GDLA prefill backward (calls ``gdla_attn_bwd``).
+
+    Inputs as ``attn_fwd`` plus dout [N, 4H, 128] bf16 (the gradient of out).
+    Returns a dict of dq_sig, dq_noise, dk, dv, dgate (bf16) and dlambda (fp32),
+    written into ``grads`` when given; ``workspace`` (uint8 CUDA tensor) is
+    allocated here when not given.
+    """
+    lens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32).reshape(-1))
+    n = int(lens.sum(dtype=np.int64))
+    hkv = q_noise.shape[1] if q_noise.dim() == 3 else -1
+    hs = GROUP * hkv
+    _check(q_sig, "q_sig", torch.bfloat16, (n, hs, DQK))
+    _check(q_noise, "q_noise", torch.bfloat16, (n, hkv, DQK))
+    _check(k, "k", torch.bfloat16, (n, hkv, DQK))
+    _check(v, "v", torch.bfloat16, (n, hkv, DV))
+    _check(lam, "lam", torch.float32, (n, hs))
+    _check(gate, "gate", torch.bfloat16, (n, hs, DV))
+    _check(dout, "dout", torch.bfloat16, (n, hs, DV))
+    shapes = {"dq_sig": ((n, hs, DQK), torch.bfloat16), "dq_noise": ((n, hkv, DQK), torch.bfloat16),
+              "dk": ((n, hkv, DQK), torch.bfloat16), "dv": ((n, hkv, DV), torch.bfloat16),
+              "dlambda": ((n, hs), torch.float32), "dgate": ((n, hs, DV), torch.bfloat16)}
+    if grads is None:
+        grads = {name: torch.empty(shape, dtype=dt, device=q_sig.device) for name, (shape, dt) in shapes.items()}
+    for name, (shape, dt) in shapes.items():
+        _check(grads[name], name, dt, shape)
+    need = attn_bwd_workspace_bytes(n, hkv)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q_sig.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = library().gdla_attn_bwd(_ptr(q_sig), _ptr(q_noise), _ptr(k), _ptr(v), _ptr(lam), _ptr(gate), _ptr(dout),
+                                 _ptr(grads["dq_sig"]), _ptr(grads["dq_noise"]), _ptr(grads["dk"]), _ptr(grads["dv"]),
+                                 _ptr(grads["dlambda"]), _ptr(grads["dgate"]), int(lens.shape[0]),
+                                 lens.__array_interface__["data"][0], hkv, int(window), workspace.data_ptr(),
+                                 ws_bytes, _stream(stream))
+    if st != 0:
+        raise GDLAError(st, "gdla_attn_bwd")
+    return grads
 
 
 def decode_workspace_bytes(batch, num_kv_heads, max_seqlen_k, window=0):

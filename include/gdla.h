@@ -100,6 +100,34 @@ GDLA_API gdla_status_t gdla_attn_fwd(const void *q_sig, const void *q_noise, con
                             void *stream);
 
 /*
+ * Prefill backward (the pages train GDLA end to end, aitrends.kr/articles/94908,
+ * context-parallel and training-system paragraphs): the gradients of
+ * sum(dout * out) for the packed varlen forward above, with the forward
+ * recomputed (nothing is kept from it). Same shapes, layouts, seqlens and window
+ * as gdla_attn_fwd, plus:
+ *   dout     bf16 [N, 4*num_kv_heads, 128]   gradient of out (read)
+ *   dq_sig   bf16 [N, 4*num_kv_heads, 192]   written
+ *   dq_noise bf16 [N, num_kv_heads, 192]     written
+ *   dk       bf16 [N, num_kv_heads, 192]     written
+ *   dv       bf16 [N, num_kv_heads, 128]     written
+ *   dlambda  fp32 [N, 4*num_kv_heads]        written
+ *   dgate    bf16 [N, 4*num_kv_heads, 128]   written (gradient of the gate logits)
+ *   workspace caller-owned device memory of gdla_attn_bwd_workspace_bytes(N,
+ *            num_kv_heads) bytes, 256-byte aligned; its contents on entry do
+ *            not matter
+ * Every row of every gradient of a token in a sequence is written; the result
+ * is deterministic (no atomics). Errors as gdla_attn_fwd, plus
+ * GDLA_ERR_WORKSPACE for a missing, small or misaligned workspace. All device
+ * buffers 16-byte aligned.
+ */
+GDLA_API size_t gdla_attn_bwd_workspace_bytes(long long total_tokens, int num_kv_heads);
+GDLA_API gdla_status_t gdla_attn_bwd(const void *q_sig, const void *q_noise, const void *k, const void *v,
+                                     const float *lambda, const void *gate_logits, const void *dout, void *dq_sig,
+                                     void *dq_noise, void *dk, void *dv, float *dlambda, void *dgate, int batch,
+                                     const int32_t *seqlens, int num_kv_heads, int window, void *workspace,
+                                     size_t workspace_bytes, void *stream);
+
+/*
  * Bytes of device workspace gdla_attn_decode needs for these sizes (0 when
  * no split-KV pass is used). Returns 0 for invalid sizes as well; the
  * workspace must be 256-byte aligned.

@@ -1,0 +1,83 @@
+"""GPU parity of gdla_attn_bwd (through the C ABI) against the fp64 backward oracle.
+
+Tolerance (per gradient, over all elements): rel_rms <= 5e-3 (the forward's bar)
+and max_abs <= 2e-2 of the gradient's largest magnitude. The backward multiplies bf16 operands the
+forward does not have - dH (= dout sigma(g)), P and dS = P (dP - rowsum(dH H))
+are each rounded to bf16 before a tensor-core product, and every gradient is
+stored in bf16 - so each gradient carries about three bf16 roundings (2^-9
+relative each, ~1.1e-3 rms) instead of the forward's one or two; dS further
+loses relative precision where dP and rowsum(dH H) nearly cancel.
+"""
+import numpy as np
+import pytest
+import torch
+
+import differential_latent_attention_b200 as gdla
+import gdla_inputs as gi
+import oracle
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("dq_sig", "dq_noise", "dk", "dv", "dlambda", "dgate")
+
+
+def _run(seqlens, hkv, window, seed):
+    t = gi.make_prefill_inputs(seqlens, hkv, seed, device="cuda")
+    dout = gi.make_prefill_grad(seqlens, hkv, seed, device="cuda")
+    g = gdla.attn_bwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"], dout, seqlens, window)
+    torch.cuda.synchronize()
+    assert gdla.device_error() == 0
+    ref = oracle.prefill_bwd(*[gi.bf16_bits(t[n]) for n in ("q_sig", "q_noise", "k", "v")], t["lam"].cpu().numpy(),
+                             gi.bf16_bits(t["gate"]), gi.bf16_bits(dout), seqlens, window)
+    return g, ref
+
+
+def _errors(got, ref):
+    got = got.float().cpu().numpy().astype(np.float64)
+    d = got - ref
+    scale = max(float(np.abs(ref).max()), 1e-30)
+    return float(np.abs(d).max()) / scale, float(np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-30))
+
+
+def check_bwd(seqlens, hkv, window, seed, rel_tol=5e-3, max_tol=2e-2):
+    g, ref = _run(seqlens, hkv, window, seed)
+    report = {}
+    for name in NAMES:
+        mx, rel = _errors(g[name], ref[name])
+        report[name] = (mx, rel)
+        assert np.isfinite(g[name].float().cpu().numpy()).all(), name
+    print(f"bwd seqlens={seqlens} hkv={hkv} window={window}: " +
+          " ".join(f"{n}=({m:.1e},{r:.1e})" for n, (m, r) in report.items()))
+    for name, (mx, rel) in report.items():
+        assert rel <= rel_tol and mx <= max_tol, (name, mx, rel)
+
+
+def test_tiny_full():
+    check_bwd((37,), 1, 0, 1)
+
+
+@pytest.mark.parametrize("window", [0, 4, 128])
+def test_ragged(window):
+    check_bwd((9, 0, 23, 1, 130, 64), 2, window, 2 + window)
+
+
+def test_several_tiles_and_ragged_tail():
+    # 700 tokens: 6 key tiles of 128 (ragged last), 30 q tiles (ragged last), 59 steps of 12 tokens
+    check_bwd((700,), 2, 0, 3)
+    check_bwd((700,), 2, 128, 4)
+
+
+def test_sixteen_groups():
+    check_bwd((300, 77), 16, 0, 5)
+
+
+def test_deterministic():
+    seqlens, hkv = (200, 61), 2
+    t = gi.make_prefill_inputs(seqlens, hkv, 9, device="cuda")
+    dout = gi.make_prefill_grad(seqlens, hkv, 9, device="cuda")
+    a = gdla.attn_bwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"], dout, seqlens, 0)
+    ws = torch.full((gdla.attn_bwd_workspace_bytes(sum(seqlens), hkv),), 0xFF, dtype=torch.uint8, device="cuda")
+    b = gdla.attn_bwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"], dout, seqlens, 0, workspace=ws)
+    torch.cuda.synchronize()
+    for name in NAMES:
+        assert torch.equal(a[name], b[name]), name

@@ -59,6 +59,19 @@ def prefill_bytes(w: gi.PrefillWorkload) -> float:
     return float(w.tokens) * per_token
 
 
+# Backward: per visible (query, key) pair and head the recomputed forward (S 2*192,
+# H = PV 2*128: the forward keeps no residuals, and the gate / lambda gradients
+# need H) and the gradient products dP (2*128), dQ (2*192), dK (2*192), dV (2*128).
+BWD_FLOPS_FACTOR = 3.0
+
+
+def prefill_bwd_bytes(w: gi.PrefillWorkload) -> float:
+    """Inputs (q_sig, q_noise, k, v, lambda, gate, dout) read once, gradients written once."""
+    hkv, hs = w.num_kv_heads, 4 * w.num_kv_heads
+    per_token = 2 * 2 * (hs * 192 + hkv * 192 + hkv * 192 + hkv * 128 + hs * 128) + 2 * hs * 128 + 2 * 4 * hs
+    return float(w.tokens) * per_token
+
+
 def decode_bytes(lengths, hkv, window) -> float:
     hs = 4 * hkv
     keys = sum(min(int(l), window) if window > 0 else int(l) for l in lengths)
@@ -547,7 +560,62 @@ def extra_workloads(gdla, dev, flush, args, world, rank, peaks):
         res.append(entry)
         del sets, ws
     res.extend(latent_workloads(gdla, dev, flush, steps, world, rank, peaks, cpu))
+    res.extend(backward_workloads(gdla, dev, flush, steps, world, rank, peaks, cpu))
     return res
+
+
+def backward_workloads(gdla, dev, flush, steps, world, rank, peaks, cpu):
+    """The prefill backward (gdla_attn_bwd: forward recompute, dQ, dK/dV) on the
+    headline shape (T = 4096, full causal) and the SWA-128 shape (B = 2 x 32768),
+    L2 flushed before every timed step."""
+    res = []
+    for w in (gi.PREFILL_FULL, gi.SWA):
+        t = gi.make_prefill_inputs(w.seqlens, w.num_kv_heads, w.seed + 1000 * rank, device=dev)
+        dout = gi.make_prefill_grad(w.seqlens, w.num_kv_heads, w.seed + 1000 * rank, device=dev)
+        hkv, hs, n = w.num_kv_heads, 4 * w.num_kv_heads, w.tokens
+        grads = {"dq_sig": torch.empty((n, hs, 192), dtype=torch.bfloat16, device=dev),
+                 "dq_noise": torch.empty((n, hkv, 192), dtype=torch.bfloat16, device=dev),
+                 "dk": torch.empty((n, hkv, 192), dtype=torch.bfloat16, device=dev),
+                 "dv": torch.empty((n, hkv, 128), dtype=torch.bfloat16, device=dev),
+                 "dlambda": torch.empty((n, hs), dtype=torch.float32, device=dev),
+                 "dgate": torch.empty((n, hs, 128), dtype=torch.bfloat16, device=dev)}
+        ws = torch.empty(gdla.attn_bwd_workspace_bytes(n, hkv), dtype=torch.uint8, device=dev)
+        per = time_steps(lambda: gdla.attn_bwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"], dout,
+                                               w.seqlens, w.window, grads=grads, workspace=ws), steps, 3, flush, world)
+        ms = reduce_max(statistics.median(per), world, dev)
+        flops = BWD_FLOPS_FACTOR * prefill_flops(w)
+        tflops = flops / (ms * 1e-3) / 1e12
+        entry = {"workload": w.name + "_backward", "metric": "TFLOP/s", "value": round(tflops * world, 3),
+                 "ms": round(ms, 5), "steps": steps, "stat": "median",
+                 "l2": "flushed (512 MiB write) before every timed step",
+                 "flops_per_step": flops, "flops_note": "3x the forward's: recomputed S and PV, then dP, dQ, dK, dV",
+                 "roofline": {"bound": "tensor", "achieved": round(tflops, 3), "peak": peaks["bf16_tflops"],
+                              "unit": "TFLOP/s", "frac": round(tflops / peaks["bf16_tflops"], 4)},
+                 "hbm": hbm_roofline(prefill_bwd_bytes(w), ms, peaks["hbm_gbs"])}
+        if cpu and w.window <= 0:
+            entry["cpu_baseline"] = oracle_bwd_sample(t, dout, w)
+        res.append(entry)
+        del t, dout, grads, ws
+    return res
+
+
+def oracle_bwd_sample(t, dout, w, sample_tokens=1024):
+    """The fp64 backward oracle, as it stands, on the first sample_tokens tokens of
+    the (single-sequence, full-causal) workload, all KV groups; value in TFLOP/s by
+    the same flop count."""
+    import oracle
+    s = slice(0, sample_tokens)
+    host = [gi.bf16_bits(t[k][s]) for k in ("q_sig", "q_noise", "k", "v")]
+    cores = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.prefill_bwd(*host, t["lam"][s].cpu().numpy(), gi.bf16_bits(t["gate"][s]), gi.bf16_bits(dout[s]),
+                       (sample_tokens,), 0, num_threads=cores)
+    dt = time.perf_counter() - t0
+    pairs = sample_tokens * (sample_tokens + 1) / 2
+    flops = BWD_FLOPS_FACTOR * pairs * 5 * w.num_kv_heads * FLOPS_PER_PAIR_HEAD
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {sample_tokens} tokens (all {w.num_kv_heads} groups) of {w.name}",
+            "seconds": round(dt, 2)}
 
 
 def latent_rotation_sets(wd, lengths, n_sets, shift, dev, rank):
@@ -721,7 +789,7 @@ def run_reference(args):
     }), flush=True)
 
 
-PROFILE_CASES = ("prefill_T4096_full", "swa128_B2_T8192", "decode_B64_L1024_4096", "decode_B64_L1024_4096_w128",
+PROFILE_CASES = ("prefill_T4096_full", "prefill_T4096_full_backward", "swa128_B2_T8192", "decode_B64_L1024_4096", "decode_B64_L1024_4096_w128",
                  "latent_decode_B64_L1024_4096", "latent_decode_B64_L1024_4096_w128")
 
 
@@ -744,6 +812,12 @@ def run_profile_case(args):
         d = gi.make_decode_inputs(lengths, 16, wd.seed, device=dev)
         fn = lambda: gdla.attn_decode(d["q_sig"], d["q_noise"], d["k_cache"], d["v_cache"], d["cu_seqlens_k"],
                                       4096, d["lam"], d["gate"], wd.window)
+    elif name.endswith("backward"):
+        w = gi.PREFILL_FULL
+        t = gi.make_prefill_inputs(w.seqlens, w.num_kv_heads, w.seed, device=dev)
+        dout = gi.make_prefill_grad(w.seqlens, w.num_kv_heads, w.seed, device=dev)
+        fn = lambda: gdla.attn_bwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"], dout, w.seqlens,
+                                   w.window)
     else:
         w = gi.PREFILL_FULL if name.startswith("prefill") else gi.PrefillWorkload(name, (8192, 8192), 16, 128, 2)
         t = gi.make_prefill_inputs(w.seqlens, w.num_kv_heads, w.seed, device=dev)

@@ -72,7 +72,9 @@ constexpr int OFF_BAR = OFF_KV + STAGES * STAGE;
 constexpr int OFF_MISC = OFF_BAR + 16 * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
 constexpr uint32_t QD_TX = (3 + 2) * 4 * QBOX_TX;  // Q and dH tiles of one item
-constexpr uint32_t DQ_COL = 0, S_COL = 192, DP_COL = 256;
+// dQ, then two buffers of (S, dP): the next key tile's products run while the
+// row warps turn this tile's into dS (written over its S).
+constexpr uint32_t DQ_COL = 0, S_COL0 = 192, DP_COL0 = 256, BUF_COLS = 128;
 constexpr uint32_t TMEM_COLS = 512;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace pbq
@@ -92,9 +94,9 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
     uint64_t *q_empty = bars + 1;   // one phase per item: its last S / dP products are done
     uint64_t *kv_full = bars + 2;   // [stage]
     uint64_t *kv_empty = bars + 4;  // [stage]
-    uint64_t *s_full = bars + 6;    // one phase per key tile: S and dP in TMEM
-    uint64_t *ds_full = bars + 7;   // one phase per key tile: dS in TMEM (128 arrivals)
-    uint64_t *dq_final = bars + 8;  // one phase per item: its last dQ product is done
+    uint64_t *s_full = bars + 6;    // [buffer]: S and dP of a key tile in TMEM
+    uint64_t *ds_full = bars + 8;   // [buffer]: its dS in TMEM (128 arrivals)
+    uint64_t *dq_final = bars + 10; // one phase per item: its last dQ product is done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
 
@@ -125,8 +127,10 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
             mbar_init(kv_full + i, 1);
             mbar_init(kv_empty + i, 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(ds_full, 128);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(s_full + b, 1);
+            mbar_init(ds_full + b, 128);
+        }
         mbar_init(dq_final, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -198,9 +202,9 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
         }
     } else if (warp == MMA_WARP) {
         // ------------------------------ MMA issuer --------------------------------
-        // Per key tile: S, dP, (dS from the row warps), dQ. The next tile's S and dP
-        // overwrite dS / dP only after this tile's dQ read them (one issuing thread,
-        // executed in order).
+        // Order: S(0), dP(0); then per key tile k: S(k+1), dP(k+1) into the other
+        // buffer, (dS(k) from the row warps), dQ(k). S(k+2) overwrites dS(k) only
+        // after dQ(k) read it (one issuing thread, executed in order).
         const uint32_t leader = elect_one_sync();
         constexpr uint32_t idesc_s = idesc_bf16_f32(128, BN, false, false);
         constexpr uint32_t idesc_q = idesc_bf16_f32(128, DQK, false, true);
@@ -213,41 +217,55 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
         for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
             const Item it = item_at(w);
             if (!__all_sync(0xffffffffu, mbar_wait(q_full, n_item & 1, abort_flag, ERR_SITE_BWD | 3))) break;
-            for (int k = 0; k < it.n_tiles; ++k, ++kv, ++step) {
-                const int st = kv % STAGES;
+            // S and dP of key tile k (global tile index kv + k, global step step + k)
+            auto issue_sdp = [&](int k) {
+                const int st = (kv + k) % STAGES;
                 if (!__all_sync(0xffffffffu,
-                                mbar_wait(kv_full + st, (kv / STAGES) & 1, abort_flag, ERR_SITE_BWD | 4))) {
-                    ok = false;
-                    break;
-                }
+                                mbar_wait(kv_full + st, ((kv + k) / STAGES) & 1, abort_flag, ERR_SITE_BWD | 4)))
+                    return false;
                 tc_fence_after();
                 const uint32_t sbase = st * STAGE;
+                const uint32_t buf = ((step + k) & 1) * BUF_COLS;
 #pragma unroll
                 for (int kk = 0; kk < DQK / 16; ++kk) {
                     const uint32_t offq = ((kk >> 2) * Q_CHUNK + (kk & 3) * 32) >> 4;
                     const uint32_t offk = (sbase + (kk >> 2) * KV_CHUNK + (kk & 3) * 32) >> 4;
-                    umma_ss_leader(tmem + S_COL, q_desc0 + offq, kv_desc0 + offk, idesc_s, kk > 0, leader);
+                    umma_ss_leader(tmem + S_COL0 + buf, q_desc0 + offq, kv_desc0 + offk, idesc_s, kk > 0, leader);
                 }
 #pragma unroll
                 for (int kk = 0; kk < DV / 16; ++kk) {
                     const uint32_t offd = ((kk >> 2) * Q_CHUNK + (kk & 3) * 32) >> 4;
                     const uint32_t offv = (sbase + K_STAGE + (kk >> 2) * KV_CHUNK + (kk & 3) * 32) >> 4;
-                    umma_ss_leader(tmem + DP_COL, dh_desc0 + offd, kv_desc0 + offv, idesc_s, kk > 0, leader);
+                    umma_ss_leader(tmem + DP_COL0 + buf, dh_desc0 + offd, kv_desc0 + offv, idesc_s, kk > 0, leader);
                 }
-                umma_commit_leader(s_full, leader);
+                umma_commit_leader(s_full + ((step + k) & 1), leader);
                 if (k == it.n_tiles - 1) umma_commit_leader(q_empty, leader);
-                if (!__all_sync(0xffffffffu, mbar_wait(ds_full, step & 1, abort_flag, ERR_SITE_BWD | 5))) {
+                return true;
+            };
+            ok = issue_sdp(0);
+            for (int k = 0; ok && k < it.n_tiles; ++k) {
+                if (k + 1 < it.n_tiles && !issue_sdp(k + 1)) {
+                    ok = false;
+                    break;
+                }
+                const int st = (kv + k) % STAGES;
+                const int sk = step + k;
+                if (!__all_sync(0xffffffffu, mbar_wait(ds_full + (sk & 1), (sk >> 1) & 1, abort_flag, ERR_SITE_BWD | 5))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t sbase = st * STAGE;
+                const uint32_t buf = (sk & 1) * BUF_COLS;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    umma_ts_leader(tmem + DQ_COL, tmem + S_COL + kk * 8, kmn_desc0 + ((sbase + kk * 2048) >> 4),
+                    umma_ts_leader(tmem + DQ_COL, tmem + S_COL0 + buf + kk * 8, kmn_desc0 + ((sbase + kk * 2048) >> 4),
                                    idesc_q, (k > 0 || kk > 0) ? 1u : 0u, leader);
                 umma_commit_leader(kv_empty + st, leader);
                 if (k == it.n_tiles - 1) umma_commit_leader(dq_final, leader);
             }
+            kv += it.n_tiles;
+            step += it.n_tiles;
         }
     } else {
         // ------------------------------ row warps ---------------------------------
@@ -269,14 +287,16 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
                 drow = __ldg(stats + srow * kBwdStats + 8 + head);
             }
             for (int k = 0; k < it.n_tiles; ++k, ++step) {
-                if (!__all_sync(0xffffffffu, mbar_wait(s_full, step & 1, abort_flag, ERR_SITE_BWD | 6))) {
+                const int b = step & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(s_full + b, (step >> 1) & 1, abort_flag, ERR_SITE_BWD | 6))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t s_addr = lane_base + S_COL0 + b * BUF_COLS;
                 uint32_t sr[64], dr[64];
-                tmem_ld64(lane_base + S_COL, sr);
-                tmem_ld64(lane_base + DP_COL, dr);
+                tmem_ld64(s_addr, sr);
+                tmem_ld64(lane_base + DP_COL0 + b * BUF_COLS, dr);
                 const int u0 = it.kv_lo + k * BN;
                 uint32_t pk[32];
 #pragma unroll
@@ -291,9 +311,9 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
                     }
                     pk[i] = pack_bf16x2(ds2[0], ds2[1]);
                 }
-                tmem_st32(lane_base + S_COL, pk);
+                tmem_st32(s_addr, pk);
                 tc_fence_before();
-                mbar_arrive(ds_full);
+                mbar_arrive(ds_full + b);
             }
             if (!ok) break;
             if (!__all_sync(0xffffffffu, mbar_wait(dq_final, n_item & 1, abort_flag, ERR_SITE_BWD | 7))) break;
@@ -351,7 +371,10 @@ constexpr int OFF_MISC = OFF_BAR + 16 * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
 constexpr uint32_t KV_TX = K_BYTES + V_BYTES;
 constexpr uint32_t STEP_TX = (3 + 2) * 2 * QBOX_TX + STATS_BYTES;
-constexpr uint32_t DK_COL = 0, DV_COL = 192, ST_COL = 320, DPT_COL = 384;
+// dK, dV, two S^T buffers (each later holding P^T in its first 32 columns and
+// dS^T in the next 32), one dP^T buffer (free again once the key warps have
+// loaded it): step s+1's products run while the key warps work on step s.
+constexpr uint32_t DK_COL = 0, DV_COL = 192, ST_COL0 = 320, DPT_COL = 448;
 constexpr uint32_t TMEM_COLS = 512;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace pbk
@@ -371,9 +394,10 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
     uint64_t *kv_empty = bars + 1;   // one phase per item: its last products are done
     uint64_t *st_full = bars + 2;    // [stage]: Q, dH halves and row statistics of a step
     uint64_t *st_empty = bars + 5;   // [stage]
-    uint64_t *s_full = bars + 8;     // one phase per step: S^T and dP^T in TMEM
-    uint64_t *pds_full = bars + 9;   // one phase per step: P^T and dS^T in TMEM (128 arrivals)
-    uint64_t *dkv_final = bars + 10; // one phase per item
+    uint64_t *s_full = bars + 8;     // [buffer]: S^T and dP^T of a step in TMEM
+    uint64_t *dpt_free = bars + 10;  // one phase per step: its dP^T has been loaded (128 arrivals)
+    uint64_t *pds_full = bars + 11;  // [buffer]: P^T and dS^T in TMEM (128 arrivals)
+    uint64_t *dkv_final = bars + 13; // one phase per item
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
 
@@ -406,8 +430,11 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
             mbar_init(st_full + i, 1);
             mbar_init(st_empty + i, 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(pds_full, 128);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(s_full + b, 1);
+            mbar_init(pds_full + b, 128);
+        }
+        mbar_init(dpt_free, 128);
         mbar_init(dkv_final, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -489,49 +516,74 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         const uint64_t v_desc0 = desc_sw128(smem_u32(smem + OFF_V), 16, 1024);
         const uint64_t st_desc0 = desc_sw128(smem_u32(smem + OFF_ST), 16, 1024);        // Q, dH halves as B (rows x dims)
         const uint64_t stmn_desc0 = desc_sw128(smem_u32(smem + OFF_ST), H_CHUNK, 1024);  // as B (dims x rows)
+        // Order: S^T(0), dP^T(0); then per step s: S^T(s+1) into the other buffer,
+        // (dP^T(s) loaded by the key warps) dP^T(s+1), (P^T(s), dS^T(s) written)
+        // dV(s), dK(s). S^T(s+2) overwrites step s's P^T / dS^T only after dV(s) and
+        // dK(s) read them (one issuing thread, executed in order).
         int g = 0, n_item = 0;
         bool ok = true;
         for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
             const Item it = item_at(w);
             if (!__all_sync(0xffffffffu, mbar_wait(kv_full, n_item & 1, abort_flag, ERR_SITE_BWD | 13))) break;
-            for (int s = 0; s < it.n_steps; ++s, ++g) {
-                const int st = g % STAGES;
-                if (!__all_sync(0xffffffffu,
-                                mbar_wait(st_full + st, (g / STAGES) & 1, abort_flag, ERR_SITE_BWD | 14))) {
-                    ok = false;
-                    break;
-                }
+            auto issue_st = [&](int s) {  // S^T of step s (global step g + s), after its stage landed
+                const int gs = g + s, st = gs % STAGES;
+                if (!__all_sync(0xffffffffu, mbar_wait(st_full + st, (gs / STAGES) & 1, abort_flag, ERR_SITE_BWD | 14)))
+                    return false;
                 tc_fence_after();
                 const uint32_t sbase = st * STAGE;
 #pragma unroll
                 for (int kk = 0; kk < DQK / 16; ++kk) {
                     const uint32_t offk = ((kk >> 2) * K_CHUNK + (kk & 3) * 32) >> 4;
                     const uint32_t offq = (sbase + (kk >> 2) * H_CHUNK + (kk & 3) * 32) >> 4;
-                    umma_ss_leader(tmem + ST_COL, k_desc0 + offk, st_desc0 + offq, idesc_s, kk > 0, leader);
+                    umma_ss_leader(tmem + ST_COL0 + (gs & 1) * 64, k_desc0 + offk, st_desc0 + offq, idesc_s, kk > 0,
+                                   leader);
                 }
+                return true;
+            };
+            auto issue_dpt = [&](int s) {  // dP^T of step s, then signal both products
+                const int gs = g + s, st = gs % STAGES;
+                const uint32_t sbase = st * STAGE;
 #pragma unroll
                 for (int kk = 0; kk < DV / 16; ++kk) {
                     const uint32_t offv = ((kk >> 2) * K_CHUNK + (kk & 3) * 32) >> 4;
                     const uint32_t offd = (sbase + QH_BYTES + (kk >> 2) * H_CHUNK + (kk & 3) * 32) >> 4;
                     umma_ss_leader(tmem + DPT_COL, v_desc0 + offv, st_desc0 + offd, idesc_s, kk > 0, leader);
                 }
-                umma_commit_leader(s_full, leader);
-                if (!__all_sync(0xffffffffu, mbar_wait(pds_full, g & 1, abort_flag, ERR_SITE_BWD | 15))) {
+                umma_commit_leader(s_full + (gs & 1), leader);
+            };
+            ok = issue_st(0);
+            if (ok) issue_dpt(0);
+            for (int s = 0; ok && s < it.n_steps; ++s) {
+                const int gs = g + s, st = gs % STAGES;
+                if (s + 1 < it.n_steps) {
+                    if (!issue_st(s + 1) ||
+                        !__all_sync(0xffffffffu, mbar_wait(dpt_free, gs & 1, abort_flag, ERR_SITE_BWD | 18))) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    issue_dpt(s + 1);
+                }
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(pds_full + (gs & 1), (gs >> 1) & 1, abort_flag, ERR_SITE_BWD | 15))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t sbase = st * STAGE;
+                const uint32_t pcol = ST_COL0 + (gs & 1) * 64;
 #pragma unroll
                 for (int kk = 0; kk < 64 / 16; ++kk) {
                     const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                    umma_ts_leader(tmem + DV_COL, tmem + ST_COL + kk * 8,
+                    umma_ts_leader(tmem + DV_COL, tmem + pcol + kk * 8,
                                    stmn_desc0 + ((sbase + QH_BYTES + kk * 2048) >> 4), idesc_v, acc, leader);
-                    umma_ts_leader(tmem + DK_COL, tmem + DPT_COL + kk * 8, stmn_desc0 + ((sbase + kk * 2048) >> 4),
+                    umma_ts_leader(tmem + DK_COL, tmem + pcol + 32 + kk * 8, stmn_desc0 + ((sbase + kk * 2048) >> 4),
                                    idesc_k, acc, leader);
                 }
                 umma_commit_leader(st_empty + st, leader);
             }
             if (!ok) break;
+            g += it.n_steps;
             umma_commit_leader(kv_empty, leader);
             umma_commit_leader(dkv_final, leader);
         }
@@ -546,15 +598,18 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
             const int u = it.u0 + kl;
             const bool key_ok = u < it.L;
             for (int s = 0; s < it.n_steps; ++s, ++g) {
-                const int st = g % STAGES;
-                if (!__all_sync(0xffffffffu, mbar_wait(s_full, g & 1, abort_flag, ERR_SITE_BWD | 16))) {
+                const int st = g % STAGES, b = g & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(s_full + b, (g >> 1) & 1, abort_flag, ERR_SITE_BWD | 16))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t s_addr = lane_base + ST_COL0 + b * 64;
                 uint32_t sr[64], dr[64];
-                tmem_ld64(lane_base + ST_COL, sr);
+                tmem_ld64(s_addr, sr);
                 tmem_ld64(lane_base + DPT_COL, dr);
+                tc_fence_before();
+                mbar_arrive(dpt_free);  // dP^T is in registers: the next step's may overwrite it
                 const float *stat = reinterpret_cast<const float *>(smem + OFF_ST + st * STAGE + QH_BYTES + DHH_BYTES);
                 const int th = it.u0 + s * HT;  // first token of the step
                 uint32_t pk[32], dk2[32];
@@ -578,10 +633,10 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                     pk[i] = pack_bf16x2(pv[0], pv[1]);
                     dk2[i] = pack_bf16x2(dv2[0], dv2[1]);
                 }
-                tmem_st32(lane_base + ST_COL, pk);
-                tmem_st32(lane_base + DPT_COL, dk2);
+                tmem_st32(s_addr, pk);
+                tmem_st32(s_addr + 32, dk2);
                 tc_fence_before();
-                mbar_arrive(pds_full);
+                mbar_arrive(pds_full + b);
             }
             if (!ok) break;
             if (!__all_sync(0xffffffffu, mbar_wait(dkv_final, n_item & 1, abort_flag, ERR_SITE_BWD | 17))) break;

@@ -27,6 +27,15 @@ constexpr int kPlanMaxItems = 6144;  // q-tiles per launch
 constexpr int kItemSeqShift = 20;
 constexpr uint32_t kItemTileMask = (1u << kItemSeqShift) - 1u;
 
+// Work item of a persistent CTA in its round r (0, 1, ...): the CTAs take the
+// list round-robin, in reverse order on odd rounds, so that over a list sorted
+// heaviest first every CTA gets a similar total (plain round-robin hands CTA 0
+// the heaviest item of every round).
+__device__ __forceinline__ int snake_item(int r) {
+    const int g = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+    return r * g + ((r & 1) ? g - 1 - c : c);
+}
+
 // Passed by value (kernel parameters): the q-tiles of one launch, heaviest
 // first. The host builds the largest form and launches the smallest capacity
 // that holds the plan, so a launch carries ~3.3 KB, ~8.7 KB or ~26.6 KB.

@@ -6,8 +6,8 @@
 // and out_i = sigmoid(gate_i) * D_i.
 //
 // Work. A work item is (KV group, block of TILES x 24 consecutive tokens of
-// one sequence). CTAs are persistent (one per SM) and take items round-robin
-// from a list sorted heaviest first.
+// one sequence). CTAs are persistent (one per SM) and take items from a list
+// sorted heaviest first, round-robin with the direction reversed every round.
 //
 // Tiling. In each 24-token tile the 5 query heads fill the M = 128 rows of one
 // tensor-core MMA, laid out per TMEM lane quarter (one warp) so that every
@@ -451,7 +451,7 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
             int gate_items = 0;         // items whose gate/lambda loads were issued
             int n_item = 0;
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+            for (int w = snake_item(0); ok && w < n_work; w = snake_item(n_item + 1), ++n_item) {
                 const Item it = item_at(w);
                 for (int x = 0; x < TILES; ++x) {
                     // the previous item's last QK^T must be done before Q_x is overwritten
@@ -551,7 +551,7 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         int sx[TILES] = {};  // S/P steps of each q tile so far (buffer and phase)
         int n_item = 0;
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+        for (int w = snake_item(0); ok && w < n_work; w = snake_item(n_item + 1), ++n_item) {
             const Item it = item_at(w);
             const int n_last = it.n_tiles[TILES - 1];
 #pragma unroll
@@ -648,7 +648,7 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         int pv = 0;   // PV products of this q tile so far (o_done phases)
         int n_item = 0;
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+        for (int w = snake_item(0); ok && w < n_work; w = snake_item(n_item + 1), ++n_item) {
             const Item it = item_at(w);
             int nt = it.n_tiles[0];
 #pragma unroll

@@ -158,7 +158,7 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
         if (lane == 0) {
             int kv = 0, issued = 0, n_item = 0;
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+            for (int w = snake_item(0); ok && w < n_work; w = snake_item(n_item + 1), ++n_item) {
                 const Item it = item_at(w);
                 if (n_item > 0 && !mbar_wait(q_empty, (n_item - 1) & 1, abort_flag, ERR_SITE_BWD | 1)) {
                     ok = false;
@@ -214,7 +214,7 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
         const uint64_t kmn_desc0 = desc_sw128(smem_u32(smem + OFF_KV), KV_CHUNK, 1024);  // K as B (dims x keys)
         int kv = 0, step = 0, n_item = 0;
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+        for (int w = snake_item(0); ok && w < n_work; w = snake_item(n_item + 1), ++n_item) {
             const Item it = item_at(w);
             if (!__all_sync(0xffffffffu, mbar_wait(q_full, n_item & 1, abort_flag, ERR_SITE_BWD | 3))) break;
             // S and dP of key tile k (global tile index kv + k, global step step + k)
@@ -276,7 +276,7 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         int step = 0, n_item = 0;
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+        for (int w = snake_item(0); ok && w < n_work; w = snake_item(n_item + 1), ++n_item) {
             const Item it = item_at(w);
             const int t = it.t0 + tau;
             const bool row_ok = !pad_row && t < it.L;
@@ -464,7 +464,7 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         if (lane == 0) {
             int g = 0, issued = 0, n_item = 0;
             bool ok = true;
-            for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+            for (int w = snake_item(0); ok && w < n_work; w = snake_item(n_item + 1), ++n_item) {
                 const Item it = item_at(w);
                 if (n_item > 0 && !mbar_wait(kv_empty, (n_item - 1) & 1, abort_flag, ERR_SITE_BWD | 11)) {
                     ok = false;
@@ -522,7 +522,7 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         // dK(s) read them (one issuing thread, executed in order).
         int g = 0, n_item = 0;
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+        for (int w = snake_item(0); ok && w < n_work; w = snake_item(n_item + 1), ++n_item) {
             const Item it = item_at(w);
             if (!__all_sync(0xffffffffu, mbar_wait(kv_full, n_item & 1, abort_flag, ERR_SITE_BWD | 13))) break;
             auto issue_st = [&](int s) {  // S^T of step s (global step g + s), after its stage landed
@@ -593,7 +593,7 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         int g = 0, n_item = 0;
         bool ok = true;
-        for (int w = blockIdx.x; ok && w < n_work; w += gridDim.x, ++n_item) {
+        for (int w = snake_item(0); ok && w < n_work; w = snake_item(n_item + 1), ++n_item) {
             const Item it = item_at(w);
             const int u = it.u0 + kl;
             const bool key_ok = u < it.L;

@@ -144,6 +144,8 @@ KERNEL_SOURCES = {
     "gdla_decode_split_kernel": ("gdla_decode.cu", "gdla_ptx.cuh", "gdla_internal.h"),
     "gdla_decode_latent_split_kernel": ("gdla_decode_latent.cu", "gdla_ptx.cuh", "gdla_internal.h"),
     "gdla_decode_latent_combine_kernel": ("gdla_decode_latent.cu", "gdla_ptx.cuh", "gdla_internal.h"),
+    "gdla_bwd_dq_kernel": ("gdla_prefill_bwd.cu", "gdla_ptx.cuh", "gdla_internal.h"),
+    "gdla_bwd_dkv_kernel": ("gdla_prefill_bwd.cu", "gdla_ptx.cuh", "gdla_internal.h"),
 }
 
 

@@ -1,6 +1,7 @@
 /*
- * GDLA forward oracle: plain, slow, fp64 CPU implementation of the Grouped
- * Differential Latent Attention core.
+ * GDLA oracle: plain, slow, fp64 CPU implementation of the Grouped
+ * Differential Latent Attention core (prefill, its backward, decode and decode
+ * over the compressed cache).
  *
  * TEST INFRASTRUCTURE ONLY. Only tests/, __graft_entry__.smoke() and the CPU
  * baseline leg of bench.py may load this library. The CUDA library never calls

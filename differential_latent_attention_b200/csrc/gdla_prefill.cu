@@ -784,25 +784,29 @@ gdla_prefill_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                 const float lam = is_sig ? reinterpret_cast<const float *>(smem + C::OFF_LAM + x * LAM_TILE)[24 * wq + lane]
                                          : 0.f;
                 const uint32_t g_base = smem_u32(smem + C::OFF_G + x * G_TILE) + (24 * wq + lane) * 128;
+                // Each half (dims 0..63, 64..127) leaves by its TMA store as soon as it is
+                // written, so the first half's store overlaps the second half's arithmetic.
 #pragma unroll
-                for (int ch = 0; ch < DV / 32; ++ch) {
-                    uint32_t o[32];
-                    tmem_ld32(o_addr + ch * 32, o);
-                    epi_chunk_staged(o, inv_l, lam, hsrc, is_sig, g_base + (ch >> 1) * G_HALF, lane & 7, ch, warp_full,
-                                     valid && !warp_full, out + row * DV + ch * 32);
-                }
-                if (warp_full) {
-                    fence_proxy_async_smem();  // the generic writes above, before the TMA store reads them
-                    __syncwarp();
-                    if (lane == 0) {
-                        const int row0_w = it.s0 + tx0 + 6 * wq;
-                        for (int h = 0; h < 2; ++h)
+                for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                    for (int c2 = 0; c2 < 2; ++c2) {
+                        const int ch = 2 * h + c2;
+                        uint32_t o[32];
+                        tmem_ld32(o_addr + ch * 32, o);
+                        epi_chunk_staged(o, inv_l, lam, hsrc, is_sig, g_base + h * G_HALF, lane & 7, ch, warp_full,
+                                         valid && !warp_full, out + row * DV + ch * 32);
+                    }
+                    if (warp_full) {
+                        fence_proxy_async_smem();  // the generic writes above, before the TMA store reads them
+                        __syncwarp();
+                        if (lane == 0) {
                             tma_store_3d(&tm_out, smem + C::OFF_G + x * G_TILE + h * G_HALF + wq * G_WARP_BOX, h * 64,
-                                         4 * it.group, row0_w);
-                        bulk_commit_group();
-                        bulk_wait_group_read0();  // the staging buffer may be refilled
+                                         4 * it.group, it.s0 + tx0 + 6 * wq);
+                            bulk_commit_group();
+                        }
                     }
                 }
+                if (warp_full && lane == 0) bulk_wait_group_read0();  // the staging buffer may be refilled
                 __syncwarp();
                 if (lane == 0) mbar_arrive(g_empty + x);
             } else if constexpr (C::EPI == EPI_HALF) {

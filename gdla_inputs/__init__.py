@@ -123,6 +123,38 @@ def make_prefill_grad(seqlens, num_kv_heads, seed, device="cpu"):
     return _normal_bf16((n, GROUP * num_kv_heads, DV), gen, device)
 
 
+HIDDEN = 4096
+Q_RANK = 1024
+
+
+def make_prologue_inputs(seqlens, num_kv_heads, seed, device="cpu"):
+    """Hidden states and projection weights for the prologue: x [N, 4096] bf16 (N(0,1));
+    weights [out, in] bf16, N(0, 1/in) (unit-variance outputs): w_qa [1024, 4096],
+    w_kva [576, 4096], w_qb [5H*192, 1024], w_uk / w_uv [H, 128, 512], w_lambda
+    [4H, 4096], w_gate [4H*128, 4096]; RMSNorm weights gamma_q [1024], gamma_kv [512]
+    fp32 (1 + N(0, 0.1^2))."""
+    n = int(sum(int(s) for s in seqlens))
+    hs = GROUP * num_kv_heads
+    gen = torch.Generator(device=device).manual_seed(int(seed) + 104729)
+
+    def w(shape, fan_in):
+        return (torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+                / float(np.sqrt(fan_in))).to(torch.bfloat16)
+
+    return {
+        "x": _normal_bf16((n, HIDDEN), gen, device),
+        "w_qa": w((Q_RANK, HIDDEN), HIDDEN),
+        "w_kva": w((DC + DR, HIDDEN), HIDDEN),
+        "gamma_q": 1.0 + 0.1 * torch.randn((Q_RANK,), generator=gen, device=device, dtype=torch.float32),
+        "gamma_kv": 1.0 + 0.1 * torch.randn((DC,), generator=gen, device=device, dtype=torch.float32),
+        "w_qb": w(((hs + num_kv_heads) * DQK, Q_RANK), Q_RANK),
+        "w_uk": w((num_kv_heads, DV, DC), DC),
+        "w_uv": w((num_kv_heads, DV, DC), DC),
+        "w_lambda": w((hs, HIDDEN), HIDDEN),
+        "w_gate": w((hs * DV, HIDDEN), HIDDEN),
+    }
+
+
 def make_decode_inputs(kv_lengths, num_kv_heads, seed, device="cpu"):
     """Decode inputs: one query per sequence plus the packed KV cache and cu_seqlens_k (int32)."""
     lengths = np.asarray(kv_lengths, dtype=np.int64)

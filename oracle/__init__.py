@@ -235,3 +235,82 @@ def prefill_bwd(q_sig, q_noise, k, v, lam, gate, dout, seqlens, window, num_thre
     if rc != 0:
         raise ValueError("gdla_oracle_prefill_bwd rejected its arguments")
     return g
+
+
+# ---------------------------------------------------------------------------
+# Prologue: the projections that produce the attention's inputs from the hidden
+# state (aitrends.kr/articles/94908, GDLA query-path paragraph: c^Q = RMSNorm(x W^Q_a)
+# expanded to content and rotary queries; [c^KV; k^R] = x W^KV_a, c^KV RMSNorm'd once
+# and expanded to 16 KV heads, k^R shared by every head; head-configuration paragraph:
+# hidden 4096, query / KV low-rank 1024 / 512, rotary 64 of the 192 query-key dims;
+# group-ratio paragraph: lambda_t = sigmoid(x_t W^lambda)). Readings where the pages
+# are silent: RMSNorm eps 1e-6 with a learned weight; rotary embedding in the
+# rotate-half form over the 64 rotary dims with base 10000, positions counted from
+# 0 in each sequence; the element-wise gate logits are x W^G (one per signal head
+# and value dim); query heads ordered signal 0..4H-1, then noise 0..H-1.
+# Plain numpy fp64; matmul is the library primitive of each projection step.
+# ---------------------------------------------------------------------------
+HIDDEN = 4096
+Q_RANK = 1024
+ROPE = 64
+ROPE_BASE = 10000.0
+RMS_EPS = 1e-6
+
+
+def _f64(a):
+    """bf16 bit patterns (uint16) or float arrays -> float64."""
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def rms_norm(c, gamma):
+    """RMSNorm over the last axis: c / sqrt(mean(c^2) + eps) * gamma."""
+    c = np.asarray(c, dtype=np.float64)
+    return c / np.sqrt(np.mean(c * c, axis=-1, keepdims=True) + RMS_EPS) * np.asarray(gamma, dtype=np.float64)
+
+
+def rope(xr, positions):
+    """Rotary embedding of the last axis (64 dims) in the rotate-half form: the pair
+    (i, i + 32) is rotated by positions * base^(-i / 32)."""
+    xr = np.asarray(xr, dtype=np.float64)
+    half = xr.shape[-1] // 2
+    inv = ROPE_BASE ** (-np.arange(half, dtype=np.float64) / half)
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * inv[None, :]       # [N, 32]
+    shape = (ang.shape[0],) + (1,) * (xr.ndim - 2) + (half,)
+    cos, sin = np.cos(ang).reshape(shape), np.sin(ang).reshape(shape)
+    a, b = xr[..., :half], xr[..., half:]
+    return np.concatenate([a * cos - b * sin, a * sin + b * cos], axis=-1)
+
+
+def positions_of(seqlens):
+    return np.concatenate([np.arange(int(L), dtype=np.int64) for L in seqlens]) if len(seqlens) else np.zeros(0)
+
+
+def prologue(x, w_qa, w_kva, gamma_q, gamma_kv, w_qb, w_uk, w_uv, w_lambda, w_gate, seqlens):
+    """The attention inputs from the hidden state x [N, 4096], in fp64.
+
+    Weights are [out_features, in_features] (bf16 bits or floats): w_qa [1024, 4096],
+    w_kva [576, 4096], w_qb [5H*192, 1024] (per query head [content 128 | rotary 64]),
+    w_uk, w_uv [H, 128, 512], w_lambda [4H, 4096], w_gate [4H*128, 4096]; gamma_q [1024],
+    gamma_kv [512]. Returns dict q_sig [N, 4H, 192], q_noise [N, H, 192], k [N, H, 192],
+    v [N, H, 128], lam [N, 4H], gate [N, 4H, 128] (float64).
+    """
+    x = _f64(x)
+    hkv = np.asarray(w_uk).shape[0]
+    hs = GROUP * hkv
+    pos = positions_of(seqlens)
+    assert pos.shape[0] == x.shape[0]
+    cq = rms_norm(x @ _f64(w_qa).T, gamma_q)                                   # [N, 1024]
+    ckv_full = x @ _f64(w_kva).T                                               # [N, 576]
+    ckv = rms_norm(ckv_full[:, :DC], gamma_kv)                                 # [N, 512]
+    k_rope = rope(ckv_full[:, DC:], pos)                                       # [N, 64]
+    q = (cq @ _f64(w_qb).T).reshape(x.shape[0], hs + hkv, DQK)                 # [N, 5H, 192]
+    q = np.concatenate([q[..., :DQK - ROPE], rope(q[..., DQK - ROPE:], pos)], axis=-1)
+    k_nope = np.einsum("nc,hdc->nhd", ckv, _f64(w_uk))                          # [N, H, 128]
+    v = np.einsum("nc,hdc->nhd", ckv, _f64(w_uv))                               # [N, H, 128]
+    k = np.concatenate([k_nope, np.broadcast_to(k_rope[:, None, :], (x.shape[0], hkv, ROPE))], axis=-1)
+    lam = 1.0 / (1.0 + np.exp(-(x @ _f64(w_lambda).T)))
+    gate = (x @ _f64(w_gate).T).reshape(x.shape[0], hs, DV)
+    return {"q_sig": q[:, :hs], "q_noise": q[:, hs:], "k": k, "v": v, "lam": lam, "gate": gate}

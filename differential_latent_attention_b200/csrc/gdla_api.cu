@@ -404,6 +404,80 @@ gdla_status_t gdla_attn_bwd(const void *q_sig, const void *q_noise, const void *
     return GDLA_OK;
 }
 
+size_t gdla_prologue_workspace_bytes(long long total_tokens) {
+    if (total_tokens < 0 || total_tokens >= (1ll << 31)) return 0;
+    const size_t n = static_cast<size_t>(total_tokens);
+    return align256(n * 1024 * 4) + align256(n * 576 * 4) + align256(n * 1024 * 2) + align256(n * 512 * 2) +
+           align256(n * 64 * 2) + align256(n * 64 * 4);
+}
+
+gdla_status_t gdla_prologue(const void *x, const void *w_qa, const void *w_kva, const float *gamma_q,
+                            const float *gamma_kv, const void *w_qb, const void *w_uk, const void *w_uv,
+                            const void *w_lambda, const void *w_gate, void *q_sig, void *q_noise, void *k, void *v,
+                            float *lambda, void *gate_logits, int batch, const int32_t *seqlens, int num_kv_heads,
+                            void *workspace, size_t workspace_bytes, void *stream) {
+    if (batch < 1 || seqlens == nullptr) return GDLA_ERR_INVALID_ARG;
+    if (batch > kPrologueMaxSeqs) return GDLA_ERR_UNSUPPORTED;
+    if (num_kv_heads < 1 || num_kv_heads > GDLA_MAX_KV_HEADS) return GDLA_ERR_UNSUPPORTED;
+    std::unique_ptr<ProloguePlan> plan(new ProloguePlan);
+    long long n_total = 0;
+    plan->n_seqs = batch;
+    for (int b = 0; b < batch; ++b) {
+        if (seqlens[b] < 0) return GDLA_ERR_INVALID_ARG;
+        plan->starts[b] = static_cast<int>(n_total);
+        n_total += seqlens[b];
+        if (n_total >= (1ll << 31)) return GDLA_ERR_INVALID_ARG;
+    }
+    plan->starts[batch] = static_cast<int>(n_total);
+    if (n_total == 0) return GDLA_OK;
+    const void *bufs[] = {x, w_qa, w_kva, gamma_q, gamma_kv, w_qb, w_uk, w_uv, w_lambda, w_gate,
+                          q_sig, q_noise, k, v, lambda, gate_logits};
+    for (const void *b : bufs)
+        if (!aligned16(b)) return GDLA_ERR_INVALID_ARG;
+    const size_t need = gdla_prologue_workspace_bytes(n_total);
+    if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return GDLA_ERR_WORKSPACE;
+    const int hkv = num_kv_heads;
+    const uint64_t N = static_cast<uint64_t>(n_total);
+    PrologueLaunch L{};
+    uint8_t *w8 = static_cast<uint8_t *>(workspace);
+    const size_t n = static_cast<size_t>(n_total);
+    L.io.cq = reinterpret_cast<float *>(w8);
+    w8 += align256(n * 1024 * 4);
+    L.io.ckv = reinterpret_cast<float *>(w8);
+    w8 += align256(n * 576 * 4);
+    L.io.cq_n = reinterpret_cast<__nv_bfloat16 *>(w8);
+    w8 += align256(n * 1024 * 2);
+    L.io.ckv_n = reinterpret_cast<__nv_bfloat16 *>(w8);
+    w8 += align256(n * 512 * 2);
+    L.io.krope = reinterpret_cast<__nv_bfloat16 *>(w8);
+    w8 += align256(n * 64 * 2);
+    L.io.rot = reinterpret_cast<float *>(w8);
+    L.io.gamma_q = gamma_q;
+    L.io.gamma_kv = gamma_kv;
+    L.io.lambda = lambda;
+    L.io.gate = static_cast<__nv_bfloat16 *>(gate_logits);
+    L.io.q_sig = static_cast<__nv_bfloat16 *>(q_sig);
+    L.io.q_noise = static_cast<__nv_bfloat16 *>(q_noise);
+    L.io.k = static_cast<__nv_bfloat16 *>(k);
+    L.io.v = static_cast<__nv_bfloat16 *>(v);
+    L.io.hkv = hkv;
+    // 2-D bf16 operands as [rows][K] maps with 64-wide K boxes (128-byte swizzle)
+    if (!make_map(&L.tm_x, x, 4096, N, 1, 64, 128, 1) || !make_map(&L.tm_wqa, w_qa, 4096, 1024, 1, 64, 256, 1) ||
+        !make_map(&L.tm_wkva, w_kva, 4096, 576, 1, 64, 192, 1) ||
+        !make_map(&L.tm_wlam, w_lambda, 4096, 4 * hkv, 1, 64, 64, 1) ||
+        !make_map(&L.tm_wgate, w_gate, 4096, 4ull * hkv * 128, 1, 64, 256, 1) ||
+        !make_map(&L.tm_cqn, L.io.cq_n, 1024, N, 1, 64, 128, 1) ||
+        !make_map(&L.tm_wqb, w_qb, 1024, 5ull * hkv * 192, 1, 64, 192, 1) ||
+        !make_map(&L.tm_ckvn, L.io.ckv_n, 512, N, 1, 64, 128, 1) ||
+        !make_map(&L.tm_wuk, w_uk, 512, 128ull * hkv, 1, 64, 128, 1) ||
+        !make_map(&L.tm_wuv, w_uv, 512, 128ull * hkv, 1, 64, 128, 1))
+        return GDLA_ERR_CUDA;
+    if (launch_prologue(L, *plan, static_cast<int>(n_total), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return GDLA_ERR_CUDA;
+    return GDLA_OK;
+}
+
 size_t gdla_decode_workspace_bytes(int batch, int num_kv_heads, int max_seqlen_k, int window) {
     if (batch < 1 || num_kv_heads < 1 || num_kv_heads > GDLA_MAX_KV_HEADS || max_seqlen_k < 1) return 0;
     return decode_workspace_bytes(make_decode_plan(batch, num_kv_heads, max_seqlen_k, window, 1));

@@ -93,6 +93,33 @@ struct BwdLaunch {
     const float *stats;
     __nv_bfloat16 *dq_sig, *dq_noise, *dk, *dv;
 };
+// Prologue (gdla_prologue.cu): the attention's inputs from the hidden state.
+constexpr int kPrologueMaxSeqs = 1024;
+struct ProloguePlan {
+    int n_seqs;
+    int starts[kPrologueMaxSeqs + 1];  // packed row of each sequence's first token; starts[n_seqs] = N
+};
+struct PrologueIO {
+    float *cq, *ckv;                  // workspace: x W^Q_a [N, 1024], x W^KV_a [N, 576] (fp32)
+    __nv_bfloat16 *cq_n, *ckv_n;      // workspace: RMSNorm'd c^Q [N, 1024], c^KV [N, 512] (bf16)
+    __nv_bfloat16 *krope;             // workspace: rotated k^R [N, 64]
+    float *rot;                       // workspace: [N, 64] cos (0..31), sin (32..63) of each row's angles
+    const float *gamma_q, *gamma_kv;  // RMSNorm weights [1024], [512]
+    float *lambda;                    // out: [N, 4H]
+    __nv_bfloat16 *gate;              // out: [N, 4H, 128]
+    __nv_bfloat16 *q_sig, *q_noise, *k, *v;  // out
+    float *f32_out;                   // plain fp32 projection target (per launch)
+    int ld_out, n_out, hkv;
+};
+struct PrologueLaunch {
+    CUtensorMap tm_x, tm_wqa, tm_wkva, tm_wlam, tm_wgate;  // projections of x (K = 4096)
+    CUtensorMap tm_cqn, tm_wqb;                            // query up-projection (K = 1024)
+    CUtensorMap tm_ckvn, tm_wuk, tm_wuv;                   // KV up-projection (K = 512)
+    PrologueIO io;
+};
+cudaError_t launch_prologue(const PrologueLaunch &launch, const ProloguePlan &plan, int total_tokens,
+                            cudaStream_t stream);
+
 cudaError_t launch_bwd_dq(const BwdLaunch &launch, const PrefillPlan &plan, cudaStream_t stream);
 cudaError_t launch_bwd_dkv(const BwdLaunch &launch, const PrefillPlan &plan, cudaStream_t stream);
 

@@ -3,6 +3,7 @@
 #include "gdla_api.cu"
 #include "gdla_prefill.cu"
 #include "gdla_prefill_bwd.cu"
+#include "gdla_prologue.cu"
 #include "gdla_decode.cu"
 #include "gdla_decode_noalloc.cu"
 #include "gdla_decode_latent.cu"

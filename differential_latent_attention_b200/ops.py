@@ -20,7 +20,8 @@ MAX_KV_HEADS = 64
 
 STATUS = {0: "GDLA_OK", 1: "GDLA_ERR_INVALID_ARG", 2: "GDLA_ERR_UNSUPPORTED", 3: "GDLA_ERR_WORKSPACE",
           4: "GDLA_ERR_CUDA"}
-EXPORTED = ("gdla_attn_fwd", "gdla_attn_bwd_workspace_bytes", "gdla_attn_bwd", "gdla_decode_workspace_bytes", "gdla_attn_decode", "gdla_attn_decode_noalloc",
+EXPORTED = ("gdla_attn_fwd", "gdla_attn_bwd_workspace_bytes", "gdla_attn_bwd", "gdla_prologue_workspace_bytes",
+            "gdla_prologue", "gdla_decode_workspace_bytes", "gdla_attn_decode", "gdla_attn_decode_noalloc",
             "gdla_decode_latent_workspace_bytes", "gdla_attn_decode_latent", "gdla_device_error",
             "gdla_selftest_wait_timeout", "gdla_status_string", "gdla_version")
 DC, DR = 512, 64
@@ -58,6 +59,10 @@ def library():
             lib.gdla_attn_bwd_workspace_bytes.restype = sz
             lib.gdla_attn_bwd.argtypes = [p, p, p, p, p, p, p, p, p, p, p, p, p, i, p, i, i, p, sz, p]
             lib.gdla_attn_bwd.restype = i
+            lib.gdla_prologue_workspace_bytes.argtypes = [ctypes.c_longlong]
+            lib.gdla_prologue_workspace_bytes.restype = sz
+            lib.gdla_prologue.argtypes = [p] * 16 + [i, p, i, p, sz, p]
+            lib.gdla_prologue.restype = i
             lib.gdla_decode_workspace_bytes.argtypes = [i, i, i, i]
             lib.gdla_decode_workspace_bytes.restype = sz
             lib.gdla_attn_decode.argtypes = [p, p, p, p, p, i, i, p, p, p, i, i, i, p, sz, p]
@@ -178,6 +183,52 @@ def attn_bwd(q_sig, q_noise, k, v, lam, gate, dout, seqlens, window=0, grads=Non
     if st != 0:
         raise GDLAError(st, "gdla_attn_bwd")
     return grads
+
+
+def prologue_workspace_bytes(total_tokens):
+    return int(library().gdla_prologue_workspace_bytes(int(total_tokens)))
+
+
+def prologue(x, w_qa, w_kva, gamma_q, gamma_kv, w_qb, w_uk, w_uv, w_lambda, w_gate, seqlens, outs=None,
+             workspace=None, stream=None):
+    """The attention inputs from the hidden state (calls ``gdla_prologue``).
+
+    x [N, 4096] bf16; weights [out, in] bf16: w_qa [1024, 4096], w_kva [576, 4096],
+    w_qb [5H*192, 1024], w_uk / w_uv [H, 128, 512], w_lambda [4H, 4096],
+    w_gate [4H*128, 4096]; gamma_q [1024], gamma_kv [512] fp32. Returns a dict
+    q_sig, q_noise, k, v, lam, gate in the layouts ``attn_fwd`` takes.
+    """
+    lens = np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32).reshape(-1))
+    n = int(lens.sum(dtype=np.int64))
+    hkv = w_uk.shape[0] if w_uk.dim() == 3 else -1
+    hs = GROUP * hkv
+    _check(x, "x", torch.bfloat16, (n, 4096))
+    _check(w_qa, "w_qa", torch.bfloat16, (1024, 4096))
+    _check(w_kva, "w_kva", torch.bfloat16, (576, 4096))
+    _check(gamma_q, "gamma_q", torch.float32, (1024,))
+    _check(gamma_kv, "gamma_kv", torch.float32, (512,))
+    _check(w_qb, "w_qb", torch.bfloat16, ((hs + hkv) * DQK, 1024))
+    _check(w_uk, "w_uk", torch.bfloat16, (hkv, DV, 512))
+    _check(w_uv, "w_uv", torch.bfloat16, (hkv, DV, 512))
+    _check(w_lambda, "w_lambda", torch.bfloat16, (hs, 4096))
+    _check(w_gate, "w_gate", torch.bfloat16, (hs * DV, 4096))
+    shapes = {"q_sig": ((n, hs, DQK), torch.bfloat16), "q_noise": ((n, hkv, DQK), torch.bfloat16),
+              "k": ((n, hkv, DQK), torch.bfloat16), "v": ((n, hkv, DV), torch.bfloat16),
+              "lam": ((n, hs), torch.float32), "gate": ((n, hs, DV), torch.bfloat16)}
+    if outs is None:
+        outs = {name: torch.empty(shape, dtype=dt, device=x.device) for name, (shape, dt) in shapes.items()}
+    for name, (shape, dt) in shapes.items():
+        _check(outs[name], name, dt, shape)
+    if workspace is None:
+        workspace = torch.empty(max(prologue_workspace_bytes(n), 1), dtype=torch.uint8, device=x.device)
+    st = library().gdla_prologue(_ptr(x), _ptr(w_qa), _ptr(w_kva), _ptr(gamma_q), _ptr(gamma_kv), _ptr(w_qb),
+                                 _ptr(w_uk), _ptr(w_uv), _ptr(w_lambda), _ptr(w_gate), _ptr(outs["q_sig"]),
+                                 _ptr(outs["q_noise"]), _ptr(outs["k"]), _ptr(outs["v"]), _ptr(outs["lam"]),
+                                 _ptr(outs["gate"]), int(lens.shape[0]), lens.__array_interface__["data"][0], hkv,
+                                 workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream(stream))
+    if st != 0:
+        raise GDLAError(st, "gdla_prologue")
+    return outs
 
 
 def decode_workspace_bytes(batch, num_kv_heads, max_seqlen_k, window=0):

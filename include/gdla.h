@@ -128,6 +128,39 @@ GDLA_API gdla_status_t gdla_attn_bwd(const void *q_sig, const void *q_noise, con
                                      size_t workspace_bytes, void *stream);
 
 /*
+ * Prologue: the attention's inputs from the hidden state (aitrends.kr/articles/94908,
+ * GDLA query-path paragraph: c^Q = RMSNorm(x W^Q_a) expanded to content and rotary
+ * queries; [c^KV; k^R] = x W^KV_a, c^KV RMSNorm'd once and expanded to the KV
+ * heads, k^R rotated and shared by every head; group-ratio paragraph: lambda =
+ * sigmoid(x W^lambda); the element-wise gate's logits x W^G). Readings: RMSNorm eps
+ * 1e-6, rotary embedding of the 64 rotary dims in the rotate-half form (pairs i,
+ * i + 32) with base 10000 and positions from 0 in each sequence; query heads are
+ * ordered signal 0..4H-1 then noise 0..H-1, each [content 128 | rotary 64].
+ * All weights are [out_features, in_features] bf16, row-major:
+ *   x         bf16 [N, 4096]            hidden state of the packed tokens
+ *   w_qa      bf16 [1024, 4096]         W^Q_a
+ *   w_kva     bf16 [576, 4096]          W^KV_a (rows 0..511 -> c^KV, 512..575 -> k^R)
+ *   gamma_q   fp32 [1024], gamma_kv fp32 [512]   RMSNorm weights
+ *   w_qb      bf16 [5H*192, 1024]       W^Q_b, query head h at rows 192h..192h+191
+ *   w_uk      bf16 [H, 128, 512]        per KV head: c^KV -> k_nope
+ *   w_uv      bf16 [H, 128, 512]        per KV head: c^KV -> v
+ *   w_lambda  bf16 [4H, 4096]           W^lambda (one per signal head)
+ *   w_gate    bf16 [4H*128, 4096]       W^G
+ * Outputs, in the layouts gdla_attn_fwd reads: q_sig [N, 4H, 192], q_noise [N, H, 192],
+ * k [N, H, 192] (k_nope | rotated k^R), v [N, H, 128], lambda fp32 [N, 4H],
+ * gate_logits [N, 4H, 128] (all bf16 but lambda). seqlens: HOST, batch <= 1024
+ * sequences (positions restart at 0 in each). workspace: caller-owned, 256-byte
+ * aligned, gdla_prologue_workspace_bytes(N) bytes. Errors as gdla_attn_fwd, plus
+ * GDLA_ERR_WORKSPACE. Every buffer 16-byte aligned.
+ */
+GDLA_API size_t gdla_prologue_workspace_bytes(long long total_tokens);
+GDLA_API gdla_status_t gdla_prologue(const void *x, const void *w_qa, const void *w_kva, const float *gamma_q,
+                                     const float *gamma_kv, const void *w_qb, const void *w_uk, const void *w_uv,
+                                     const void *w_lambda, const void *w_gate, void *q_sig, void *q_noise, void *k,
+                                     void *v, float *lambda, void *gate_logits, int batch, const int32_t *seqlens,
+                                     int num_kv_heads, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Bytes of device workspace gdla_attn_decode needs for these sizes (0 when
  * no split-KV pass is used). Returns 0 for invalid sizes as well; the
  * workspace must be 256-byte aligned.

@@ -146,6 +146,7 @@ KERNEL_SOURCES = {
     "gdla_decode_latent_combine_kernel": ("gdla_decode_latent.cu", "gdla_ptx.cuh", "gdla_internal.h"),
     "gdla_bwd_dq_kernel": ("gdla_prefill_bwd.cu", "gdla_ptx.cuh", "gdla_internal.h"),
     "gdla_bwd_dkv_kernel": ("gdla_prefill_bwd.cu", "gdla_ptx.cuh", "gdla_internal.h"),
+    "gdla_proj_kernel": ("gdla_prologue.cu", "gdla_ptx.cuh", "gdla_internal.h"),
 }
 
 
@@ -563,7 +564,50 @@ def extra_workloads(gdla, dev, flush, args, world, rank, peaks):
         del sets, ws
     res.extend(latent_workloads(gdla, dev, flush, steps, world, rank, peaks, cpu))
     res.extend(backward_workloads(gdla, dev, flush, steps, world, rank, peaks, cpu))
+    res.extend(prologue_workloads(gdla, dev, flush, steps, world, rank, peaks, cpu))
     return res
+
+
+PROLOGUE_WEIGHTS = ("w_qa", "w_kva", "gamma_q", "gamma_kv", "w_qb", "w_uk", "w_uv", "w_lambda", "w_gate")
+
+
+def prologue_flops(n_tokens, hkv) -> float:
+    """2 flop per multiply-add of the projections: x [4096] -> c^Q (1024), [c^KV; k^R] (576),
+    lambda (4H), gate logits (4H x 128); c^Q -> 5H query heads x 192; c^KV -> H x (128 + 128)."""
+    per_token = 4096 * (1024 + 576 + 4 * hkv + 4 * hkv * 128) + 1024 * 5 * hkv * 192 + 512 * hkv * 256
+    return 2.0 * n_tokens * per_token
+
+
+def prologue_workloads(gdla, dev, flush, steps, world, rank, peaks, cpu):
+    """The prologue (gdla_prologue: the attention inputs from the hidden state) on the
+    headline shape (4096 tokens, 16 KV groups), L2 flushed before every timed step."""
+    w = gi.PREFILL_FULL
+    t = gi.make_prologue_inputs(w.seqlens, w.num_kv_heads, w.seed + 1000 * rank, device=dev)
+    ws = torch.empty(gdla.prologue_workspace_bytes(w.tokens), dtype=torch.uint8, device=dev)
+    outs = gdla.prologue(t["x"], *[t[k] for k in PROLOGUE_WEIGHTS], w.seqlens, workspace=ws)
+    per = time_steps(lambda: gdla.prologue(t["x"], *[t[k] for k in PROLOGUE_WEIGHTS], w.seqlens, outs=outs,
+                                           workspace=ws), steps, 3, flush, world)
+    ms = reduce_max(statistics.median(per), world, dev)
+    flops = prologue_flops(w.tokens, w.num_kv_heads)
+    tflops = flops / (ms * 1e-3) / 1e12
+    entry = {"workload": f"prologue_T{w.tokens}_H{w.num_kv_heads}", "metric": "TFLOP/s",
+             "value": round(tflops * world, 3), "ms": round(ms, 5), "steps": steps, "stat": "median",
+             "l2": "flushed (512 MiB write) before every timed step", "flops_per_step": flops,
+             "roofline": {"bound": "tensor", "achieved": round(tflops, 3), "peak": peaks["bf16_tflops"],
+                          "unit": "TFLOP/s", "frac": round(tflops / peaks["bf16_tflops"], 4)}}
+    if cpu:
+        import oracle
+        host = lambda x: gi.bf16_bits(x) if x.dtype == torch.bfloat16 else x.cpu().numpy()
+        sample = 256
+        t0 = time.perf_counter()
+        oracle.prologue(host(t["x"][:sample]), *[host(t[k]) for k in PROLOGUE_WEIGHTS], (sample,))
+        dt = time.perf_counter() - t0
+        entry["cpu_baseline"] = {"value": round(prologue_flops(sample, w.num_kv_heads) / dt / 1e12, 6),
+                                 "unit": "TFLOP/s", "cores": oracle.default_threads(), "kind": "oracle",
+                                 "sample": f"first {sample} tokens of the prologue workload (numpy fp64)",
+                                 "seconds": round(dt, 2)}
+    del t, ws, outs
+    return [entry]
 
 
 def backward_workloads(gdla, dev, flush, steps, world, rank, peaks, cpu):
@@ -791,7 +835,7 @@ def run_reference(args):
     }), flush=True)
 
 
-PROFILE_CASES = ("prefill_T4096_full", "prefill_T4096_full_backward", "swa128_B2_T8192", "decode_B64_L1024_4096", "decode_B64_L1024_4096_w128",
+PROFILE_CASES = ("prefill_T4096_full", "prefill_T4096_full_backward", "prologue_T4096", "swa128_B2_T8192", "decode_B64_L1024_4096", "decode_B64_L1024_4096_w128",
                  "latent_decode_B64_L1024_4096", "latent_decode_B64_L1024_4096_w128")
 
 
@@ -814,6 +858,10 @@ def run_profile_case(args):
         d = gi.make_decode_inputs(lengths, 16, wd.seed, device=dev)
         fn = lambda: gdla.attn_decode(d["q_sig"], d["q_noise"], d["k_cache"], d["v_cache"], d["cu_seqlens_k"],
                                       4096, d["lam"], d["gate"], wd.window)
+    elif name.startswith("prologue"):
+        w = gi.PREFILL_FULL
+        t = gi.make_prologue_inputs(w.seqlens, w.num_kv_heads, w.seed, device=dev)
+        fn = lambda: gdla.prologue(t["x"], *[t[k] for k in PROLOGUE_WEIGHTS], w.seqlens)
     elif name.endswith("backward"):
         w = gi.PREFILL_FULL
         t = gi.make_prefill_inputs(w.seqlens, w.num_kv_heads, w.seed, device=dev)

@@ -407,8 +407,8 @@ gdla_status_t gdla_attn_bwd(const void *q_sig, const void *q_noise, const void *
 size_t gdla_prologue_workspace_bytes(long long total_tokens) {
     if (total_tokens < 0 || total_tokens >= (1ll << 31)) return 0;
     const size_t n = static_cast<size_t>(total_tokens);
-    return align256(n * 1024 * 4) + align256(n * 576 * 4) + align256(n * 1024 * 2) + align256(n * 512 * 2) +
-           align256(n * 64 * 2) + align256(n * 64 * 4);
+    return align256(n * 1024 * 2) + align256(n * 512 * 2) + align256(n * 16 * 4) + align256(n * 64 * 2) +
+           align256(n * 64 * 4);
 }
 
 gdla_status_t gdla_prologue(const void *x, const void *w_qa, const void *w_kva, const float *gamma_q,
@@ -442,14 +442,12 @@ gdla_status_t gdla_prologue(const void *x, const void *w_qa, const void *w_kva, 
     PrologueLaunch L{};
     uint8_t *w8 = static_cast<uint8_t *>(workspace);
     const size_t n = static_cast<size_t>(n_total);
-    L.io.cq = reinterpret_cast<float *>(w8);
-    w8 += align256(n * 1024 * 4);
-    L.io.ckv = reinterpret_cast<float *>(w8);
-    w8 += align256(n * 576 * 4);
-    L.io.cq_n = reinterpret_cast<__nv_bfloat16 *>(w8);
+    L.io.cq_g = reinterpret_cast<__nv_bfloat16 *>(w8);
     w8 += align256(n * 1024 * 2);
-    L.io.ckv_n = reinterpret_cast<__nv_bfloat16 *>(w8);
+    L.io.ckv_g = reinterpret_cast<__nv_bfloat16 *>(w8);
     w8 += align256(n * 512 * 2);
+    L.io.ssq = reinterpret_cast<float *>(w8);
+    w8 += align256(n * 16 * 4);
     L.io.krope = reinterpret_cast<__nv_bfloat16 *>(w8);
     w8 += align256(n * 64 * 2);
     L.io.rot = reinterpret_cast<float *>(w8);
@@ -467,11 +465,14 @@ gdla_status_t gdla_prologue(const void *x, const void *w_qa, const void *w_kva, 
         !make_map(&L.tm_wkva, w_kva, 4096, 576, 1, 64, 192, 1) ||
         !make_map(&L.tm_wlam, w_lambda, 4096, 4 * hkv, 1, 64, 64, 1) ||
         !make_map(&L.tm_wgate, w_gate, 4096, 4ull * hkv * 128, 1, 64, 256, 1) ||
-        !make_map(&L.tm_cqn, L.io.cq_n, 1024, N, 1, 64, 128, 1) ||
+        !make_map(&L.tm_cqn, L.io.cq_g, 1024, N, 1, 64, 128, 1) ||
         !make_map(&L.tm_wqb, w_qb, 1024, 5ull * hkv * 192, 1, 64, 192, 1) ||
-        !make_map(&L.tm_ckvn, L.io.ckv_n, 512, N, 1, 64, 128, 1) ||
+        !make_map(&L.tm_ckvn, L.io.ckv_g, 512, N, 1, 64, 128, 1) ||
         !make_map(&L.tm_wuk, w_uk, 512, 128ull * hkv, 1, 64, 128, 1) ||
-        !make_map(&L.tm_wuv, w_uv, 512, 128ull * hkv, 1, 64, 128, 1))
+        !make_map(&L.tm_wuv, w_uv, 512, 128ull * hkv, 1, 64, 128, 1) ||
+        !make_map(&L.tm_qs_o, q_sig, 192, 4ull * hkv, N, 64, 1, 32) ||
+        !make_map(&L.tm_qn_o, q_noise, 192, hkv, N, 64, 1, 32) || !make_map(&L.tm_k_o, k, 192, hkv, N, 64, 1, 32) ||
+        !make_map(&L.tm_v_o, v, 128, hkv, N, 64, 1, 32))
         return GDLA_ERR_CUDA;
     if (launch_prologue(L, *plan, static_cast<int>(n_total), static_cast<cudaStream_t>(stream)) != cudaSuccess)
         return GDLA_ERR_CUDA;

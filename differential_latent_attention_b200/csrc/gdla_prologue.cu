@@ -10,19 +10,24 @@
 // rotate-half form (pair i, i+32) with base 10000, positions from 0 in each
 // sequence; gate logits = x W^G; query heads ordered signal 0..4H-1, noise 0..H-1.
 //
-// Launches (all weights [out_features, in_features] bf16, K-major):
-//   1-4  projections of x (K = 4096): c^Q and [c^KV; k^R] (fp32, to the workspace),
-//        lambda (sigmoid, fp32 [N, 4H]) and the gate logits (bf16 [N, 4H, 128]);
-//   5    per token: RMSNorm of c^Q and c^KV (bf16, with their weights), the rotary
-//        angle table cos/sin(t base^(-i/32)) (angles in fp64) and the rotated k^R;
-//   6    RMSNorm(c^Q) W^Q_b (K = 1024), one 192-column query head per tile, its
-//        rotary 64 columns rotated in the epilogue -> q_sig [N, 4H, 192], q_noise [N, H, 192];
-//   7    RMSNorm(c^KV) [W^UK_j; W^UV_j] (K = 512), one KV head per 256-column tile ->
-//        k [N, H, 192] = [k_nope | rotated k^R], v [N, H, 128].
-// The GEMM: one CTA per 128-row x NT-column tile; a TMA producer warp streams
-// 64-wide K chunks of A (the rows) and B (the weights' rows) through a 4-stage
-// ring; one elected thread issues tcgen05 MMAs (M = 128, N = NT, fp32 in TMEM);
-// the 4 epilogue warps (one TMEM lane = one row) apply the mode's epilogue.
+// RMSNorm(c) W = rsqrt(mean(c^2) + eps) * ((c * gamma) W): the row scale is one scalar
+// per token, so it moves from the up-projections' operand to their epilogue. Two
+// launches of one persistent grouped GEMM (weights [out_features, in_features] bf16,
+// K-major):
+//   phase 1, A = x (K = 4096): gate logits (bf16 [N, 4H, 128]); c^Q (256-column tiles:
+//            c^Q * gamma_q in bf16 and the tile's partial sums of squares); [c^KV; k^R]
+//            (192-column tiles: c^KV * gamma_kv in bf16 and partial sums of squares; for
+//            the k^R columns the rotary table cos/sin(t base^(-i/32)), angles in fp64, and
+//            the rotated k^R); lambda (sigmoid, fp32 [N, 4H]);
+//   phase 2: (c^Q * gamma_q) W^Q_b (K = 1024, one 192-column query head per tile, scaled
+//            by the row's rsqrt, rotary 64 columns rotated) -> q_sig, q_noise; and
+//            (c^KV * gamma_kv) W^UK_j, (c^KV * gamma_kv) W^UV_j (K = 512, one KV head per
+//            128-column tile, scaled) -> k = [k_nope | rotated k^R], v.
+// The GEMM: one CTA per SM walks its tiles (t = blockIdx.x, + gridDim.x, ...); a TMA
+// producer warp streams 64-wide K chunks of A (128 rows) and B (the weights' rows)
+// through a 4- or 5-stage ring; one elected thread issues tcgen05 MMAs (M = 128, N = nt, fp32)
+// into one of two TMEM accumulators, so 8 epilogue warps (TMEM lane quarter = warp % 4,
+// column half = warp / 4) drain one tile while the next one is multiplied.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -33,7 +38,7 @@
 namespace gdla {
 
 // Epilogue modes of the projection GEMM.
-enum : int { PRO_PLAIN = 0, PRO_LAMBDA = 1, PRO_GATE = 2, PRO_QUP = 3, PRO_KVUP = 4 };
+enum : int { PRO_CQ = 0, PRO_CKV = 1, PRO_LAMBDA = 2, PRO_GATE = 3, PRO_QUP = 4, PRO_KUP = 5, PRO_VUP = 6 };
 
 // 32 fp32 values (as bits) -> 32 bf16 at dst (64 bytes, 16-byte aligned).
 __device__ __forceinline__ void store_bf16_32(__nv_bfloat16 *dst, const uint32_t (&o)[32]) {
@@ -47,23 +52,30 @@ __device__ __forceinline__ void store_bf16_32(__nv_bfloat16 *dst, const uint32_t
 }
 
 namespace pg {
-constexpr int STAGES = 4;
-constexpr int A_CHUNK = 128 * 128;  // 128 rows x 64 K (bf16)
-constexpr int NUM_THREADS = 192;    // epilogue warps 0-3, producer 4, MMA 5
-constexpr int PRODUCER_WARP = 4, MMA_WARP = 5;
-constexpr int ROPE_HALF = 32;
+constexpr int A_BYTES = 128 * 128;             // 128 rows x 64 K (bf16)
+constexpr int EPI_WARPS = 8;
+constexpr int PRODUCER_WARP = 8, MMA_WARP = 9;
+constexpr int NUM_THREADS = 320;
+constexpr uint32_t ACC_COLS = 256;             // column offset of the second accumulator
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int SSQ = 16;                        // partial sums of squares per row
 }  // namespace pg
 
-template <int EPI, int NT>
-struct ProjCfg {
-    static constexpr int B_CHUNK = NT * 128;
-    static constexpr int STAGE = pg::A_CHUNK + B_CHUNK;
-    static constexpr int OFF_BAR = pg::STAGES * STAGE;
+// Shared memory of a phase: a 4-stage ring for B tiles up to 256 rows (phase 1) or
+// 192 rows (phase 2); phase 2 adds two 4 KB output boxes (32 rows x 64 bf16, 128-byte
+// swizzle) per epilogue warp, which its TMA stores read.
+template <int PHASE>
+struct PhaseCfg {
+    static constexpr int STAGES = 4;
+    static constexpr int B_ROWS = PHASE == 1 ? 256 : 192;
+    static constexpr int STAGE = pg::A_BYTES + B_ROWS * 128;
+    static constexpr int OFF_STG = STAGES * STAGE;
+    static constexpr int STG_BYTES = PHASE == 1 ? 0 : pg::EPI_WARPS * 2 * 4096;
+    static constexpr int OFF_BAR = OFF_STG + STG_BYTES;  // full[S], empty[S], acc_full[2], acc_empty[2], drain
     static constexpr int OFF_MISC = OFF_BAR + 16 * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
-    static constexpr uint32_t TMEM_COLS = NT <= 32 ? 32 : (NT <= 64 ? 64 : (NT <= 128 ? 128 : 256));
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    static_assert(NT % 32 == 0 && NT <= 256, "tile width");
+    static_assert(2 * STAGES + 5 <= 16, "barrier slots");
 };
 
 // Position of packed row m in its sequence (starts[] = cumulative sequence starts).
@@ -76,35 +88,262 @@ __device__ __forceinline__ int row_position(const ProloguePlan &p, int m) {
     return m - p.starts[lo];
 }
 
-template <int EPI, int NT>
+struct TileRef {
+    int p, n_tile, m0;
+};
+__device__ __forceinline__ TileRef decode_tile(const ProjGroup &G, int t) {
+    int p = 0;
+    while (p + 1 < G.n_prob && t >= G.prob[p + 1].first) ++p;
+    const int local = t - G.prob[p].first;
+    return {p, local / G.m_blocks, (local % G.m_blocks) * 128};
+}
+
+// ------------------------------ phase 1 epilogues -----------------------------
+// 32 values c -> bf16 (c * gamma) at dst; returns the sum of squares of the c.
+__device__ __forceinline__ float scale_store_32(__nv_bfloat16 *dst, uint32_t (&o)[32], const float *gamma,
+                                                bool row_ok) {
+    const float4 *g4 = reinterpret_cast<const float4 *>(gamma);
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float4 g = __ldg(g4 + i);
+        const float gv[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float x = __uint_as_float(o[4 * i + j]);
+            ss = fmaf(x, x, ss);
+            o[4 * i + j] = __float_as_uint(x * gv[j]);
+        }
+    }
+    if (row_ok) store_bf16_32(dst, o);
+    return ss;
+}
+
+// c^Q tile (256 columns): this half's 128 columns.
+__device__ __forceinline__ void epi_cq(const PrologueIO &io, uint32_t tcol, int m, bool row_ok, int n_tile,
+                                       int hf) {
+    const int c0 = n_tile * 256 + hf * 128;
+    float ss = 0.f;
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(tcol + hf * 128 + ch * 32, o);
+        ss += scale_store_32(io.cq_g + static_cast<size_t>(m) * 1024 + c0 + ch * 32, o, io.gamma_q + c0 + ch * 32,
+                             row_ok);
+    }
+    if (row_ok) io.ssq[static_cast<size_t>(m) * pg::SSQ + n_tile * 2 + hf] = ss;
+}
+
+// [c^KV; k^R] tile (192 columns): this half's 96 columns. Columns 512..575 are k^R:
+// the half that holds them (tile 2, half 1) also writes the row's rotary table and
+// the rotated k^R.
+__device__ __forceinline__ void epi_ckv(const PrologueIO &io, const ProloguePlan &plan, uint32_t tcol, int m,
+                                        bool row_ok, int n_tile, int hf, int lane) {
+    const int c0 = n_tile * 192 + hf * 96;
+    const bool rope_part = (c0 + 96 > 512);
+    const int n_norm = rope_part ? 1 : 3;  // 32-column chunks of c^KV
+    float ss = 0.f;
+#pragma unroll 1
+    for (int ch = 0; ch < n_norm; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(tcol + hf * 96 + ch * 32, o);
+        ss += scale_store_32(io.ckv_g + static_cast<size_t>(m) * 512 + c0 + ch * 32, o, io.gamma_kv + c0 + ch * 32,
+                             row_ok);
+    }
+    if (row_ok) io.ssq[static_cast<size_t>(m) * pg::SSQ + 8 + n_tile * 2 + hf] = ss;
+    if (!rope_part) return;
+    // this lane's inverse frequency base^(-lane/32) in fp64; the lanes share them by shuffle
+    const double inv_lane = exp2(-static_cast<double>(lane) * (13.287712379549449 / 32.0));
+    uint32_t a[32], b[32];
+    tmem_ld32(tcol + hf * 96 + 32, a);  // k^R dims 0..31
+    tmem_ld32(tcol + hf * 96 + 64, b);  // k^R dims 32..63
+    const double pos = row_ok ? static_cast<double>(row_position(plan, m)) : 0.0;
+    float *rot = io.rot + static_cast<size_t>(m) * 64;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const double inv = __shfl_sync(0xffffffffu, inv_lane, i);
+        double s, c;
+        sincos(pos * inv, &s, &c);
+        if (row_ok) {
+            rot[i] = static_cast<float>(c);
+            rot[32 + i] = static_cast<float>(s);
+        }
+        const double x0 = __uint_as_float(a[i]), x1 = __uint_as_float(b[i]);
+        a[i] = __float_as_uint(static_cast<float>(x0 * c - x1 * s));
+        b[i] = __float_as_uint(static_cast<float>(x0 * s + x1 * c));
+    }
+    if (row_ok) {
+        store_bf16_32(io.krope + static_cast<size_t>(m) * 64, a);
+        store_bf16_32(io.krope + static_cast<size_t>(m) * 64 + 32, b);
+    }
+}
+
+// lambda tile (64 columns of 4H): this half's 32 columns, sigmoid.
+__device__ __forceinline__ void epi_lambda(const PrologueIO &io, uint32_t tcol, int m, bool row_ok, int n_tile,
+                                           int hf) {
+    const int n_out = 4 * io.hkv;
+    const int c0 = n_tile * 64 + hf * 32;
+    if (c0 >= n_out) return;
+    uint32_t o[32];
+    tmem_ld32(tcol + hf * 32, o);
+    if (!row_ok) return;
+    float *dst = io.lambda + static_cast<size_t>(m) * n_out + c0;
+    float y[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) y[i] = 1.f / (1.f + __expf(-__uint_as_float(o[i])));
+    if (c0 + 32 <= n_out) {
+        float4 *d4 = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d4[i] = make_float4(y[4 * i], y[4 * i + 1], y[4 * i + 2], y[4 * i + 3]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if (c0 + i < n_out) dst[i] = y[i];
+    }
+}
+
+// gate tile (256 columns of 4H x 128): this half's 128 columns, bf16.
+__device__ __forceinline__ void epi_gate(const PrologueIO &io, uint32_t tcol, int m, bool row_ok, int n_tile,
+                                         int hf) {
+    __nv_bfloat16 *dst = io.gate + static_cast<size_t>(m) * (4 * io.hkv * 128) + n_tile * 256 + hf * 128;
+#pragma unroll 1
+    for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(tcol + hf * 128 + ch * 32, o);
+        if (row_ok) store_bf16_32(dst + ch * 32, o);
+    }
+}
+
+// ------------------------------ phase 2 epilogues -----------------------------
+__device__ __forceinline__ void scale_32(uint32_t (&o)[32], float r) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * r);
+}
+
+// rsqrt(mean of squares + eps) of row m from its partial sums [first, first + count).
+__device__ __forceinline__ float row_rsqrt(const PrologueIO &io, int m, int first, int count, float inv_width) {
+    const float *p = io.ssq + static_cast<size_t>(m) * pg::SSQ + first;
+    float ss = 0.f;
+    for (int i = 0; i < count; ++i) ss += __ldg(p + i);
+    return rsqrtf(ss * inv_width + 1e-6f);
+}
+
+// 32 fp32 values (as bits) x r -> bf16 into 16-byte chunks c0..c0+3 of this lane's
+// 128-byte row of a 128-byte-swizzled output box at shared address `box`.
+__device__ __forceinline__ void stage_32(uint32_t box, int lane, int c0, const uint32_t (&o)[32], float r) {
+    const uint32_t row = box + lane * 128;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t w[4] = {pack_bf16x2(__uint_as_float(o[8 * i]) * r, __uint_as_float(o[8 * i + 1]) * r),
+                               pack_bf16x2(__uint_as_float(o[8 * i + 2]) * r, __uint_as_float(o[8 * i + 3]) * r),
+                               pack_bf16x2(__uint_as_float(o[8 * i + 4]) * r, __uint_as_float(o[8 * i + 5]) * r),
+                               pack_bf16x2(__uint_as_float(o[8 * i + 6]) * r, __uint_as_float(o[8 * i + 7]) * r)};
+        sts128(row + (((c0 + i) ^ (lane & 7)) << 4), w);
+    }
+}
+
+// One query head h (tile n = h) into this warp's output boxes: half 0 the content dims
+// 0..127 (two boxes), half 1 the rotary dims 128..191 (pairs i, i+32) rotated. Returns
+// the number of boxes staged; box b goes to dims col0 + 64 b.
+__device__ __forceinline__ int epi_qup(const PrologueIO &io, uint32_t tcol, int m, bool row_ok, int hf, int lane,
+                                       uint32_t stg, int &col0) {
+    const float r = row_ok ? row_rsqrt(io, m, 0, 8, 1.f / 1024.f) : 0.f;
+    if (hf == 0) {
+#pragma unroll 1
+        for (int ch = 0; ch < 4; ++ch) {
+            uint32_t o[32];
+            tmem_ld32(tcol + ch * 32, o);
+            stage_32(stg + (ch >> 1) * 4096, lane, (ch & 1) * 4, o, r);
+        }
+        col0 = 0;
+        return 2;
+    }
+    uint32_t a[32], b[32];
+    tmem_ld32(tcol + 128, a);
+    tmem_ld32(tcol + 160, b);
+    if (row_ok) {
+        const float4 *rot = reinterpret_cast<const float4 *>(io.rot + static_cast<size_t>(m) * 64);  // cos | sin
+#pragma unroll
+        for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 c4 = __ldg(rot + i4), s4 = __ldg(rot + 8 + i4);
+            const float cv[4] = {c4.x, c4.y, c4.z, c4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = 4 * i4 + j;
+                const float x0 = __uint_as_float(a[i]), x1 = __uint_as_float(b[i]);
+                a[i] = __float_as_uint(x0 * cv[j] - x1 * sv[j]);
+                b[i] = __float_as_uint(x0 * sv[j] + x1 * cv[j]);
+            }
+        }
+    }
+    stage_32(stg, lane, 0, a, r);
+    stage_32(stg, lane, 4, b, r);
+    col0 = 128;
+    return 1;
+}
+
+// One KV head j (tile n = j) of k_nope (PRO_KUP) or v (PRO_VUP), 64 dims per half;
+// half 1 of k_nope also stages the rotated k^R (k's dims 128..191) as its second box.
+__device__ __forceinline__ int epi_kvup(const PrologueIO &io, uint32_t tcol, int m, bool row_ok, int hf, int lane,
+                                        bool is_k, uint32_t stg, int &col0) {
+    const float r = row_ok ? row_rsqrt(io, m, 8, 6, 1.f / 512.f) : 0.f;
+#pragma unroll 1
+    for (int ch = 0; ch < 2; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(tcol + hf * 64 + ch * 32, o);
+        stage_32(stg, lane, ch * 4, o, r);
+    }
+    col0 = hf * 64;
+    if (!(is_k && hf == 1)) return 1;
+    const uint32_t row = stg + 4096 + lane * 128;
+    const uint4 *kr = reinterpret_cast<const uint4 *>(io.krope + static_cast<size_t>(row_ok ? m : 0) * 64);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint4 v = __ldg(kr + i);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        sts128(row + ((i ^ (lane & 7)) << 4), w);
+    }
+    return 2;
+}
+
+// ------------------------------------------------------------------------------
+// The persistent grouped projection GEMM. PHASE 1 runs PRO_GATE, PRO_CQ, PRO_CKV and
+// PRO_LAMBDA problems; PHASE 2 PRO_QUP, PRO_KUP and PRO_VUP.
+// ------------------------------------------------------------------------------
+template <int PHASE>
 __global__ void __launch_bounds__(pg::NUM_THREADS, 1)
-gdla_proj_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                 const __grid_constant__ CUtensorMap tm_b2, const PrologueIO io, int M, int K) {
-    using C = ProjCfg<EPI, NT>;
+gdla_proj_kernel(const __grid_constant__ ProjGroup G, const __grid_constant__ PrologueIO io,
+                 const __grid_constant__ ProloguePlan plan) {
     using namespace pg;
+    using C = PhaseCfg<PHASE>;
+    constexpr int STAGES = C::STAGES, STAGE = C::STAGE;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::OFF_BAR);
-    uint64_t *full = bars;               // [stage]
-    uint64_t *empty = bars + STAGES;     // [stage]
-    uint64_t *mma_done = bars + 2 * STAGES;
+    uint64_t *full = bars;                   // [stage]
+    uint64_t *empty = bars + STAGES;         // [stage]
+    uint64_t *acc_full = bars + 2 * STAGES;  // [accumulator]
+    uint64_t *acc_empty = acc_full + 2;      // [accumulator]
+    uint64_t *drain = acc_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * 128, tile_n = blockIdx.y, n0 = tile_n * NT;
-    const int nk = K / 64;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
             mbar_init(full + i, 1);
             mbar_init(empty + i, 1);
         }
-        mbar_init(mma_done, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(acc_full + i, 1);
+            mbar_init(acc_empty + i, EPI_WARPS);
+        }
+        mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == MMA_WARP) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -114,235 +353,186 @@ gdla_proj_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant
 
     if (warp == PRODUCER_WARP) {
         if (lane == 0) {
-            int issued = 0;
-            for (int kc = 0; kc < nk; ++kc) {
-                const int st = kc % STAGES;
-                if (kc >= STAGES && !mbar_wait(empty + st, ((kc / STAGES) + 1) & 1, abort_flag, ERR_SITE_PROLOGUE | 1))
-                    break;
-                mbar_arrive_expect_tx(full + st, C::STAGE);
-                uint8_t *sb = smem + st * C::STAGE;
-                tma_load_3d(sb, &tm_a, full + st, kc * 64, m0, 0);
-                if (EPI == PRO_KVUP) {  // [W^UK_j; W^UV_j]: two 128-row boxes
-                    tma_load_3d(sb + A_CHUNK, &tm_b, full + st, kc * 64, tile_n * 128, 0);
-                    tma_load_3d(sb + A_CHUNK + 128 * 128, &tm_b2, full + st, kc * 64, tile_n * 128, 0);
-                } else {
-                    tma_load_3d(sb + A_CHUNK, &tm_b, full + st, kc * 64, n0, 0);
+            uint32_t g = 0, issued = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < G.total_tiles; t += gridDim.x) {
+                const TileRef tr = decode_tile(G, t);
+                const ProjProblem &pr = G.prob[tr.p];
+                const uint32_t bytes = A_BYTES + pr.nt * 128;
+                for (int kc = 0; kc < pr.nk; ++kc, ++g) {
+                    const uint32_t st = g % STAGES;
+                    if (g >= STAGES &&
+                        !mbar_wait(empty + st, ((g / STAGES) + 1) & 1, abort_flag, ERR_SITE_PROLOGUE | 1)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(full + st, bytes);
+                    uint8_t *sb = smem + st * STAGE;
+                    tma_load_3d(sb, &G.tm_a[tr.p], full + st, kc * 64, tr.m0, 0);
+                    tma_load_3d(sb + A_BYTES, &G.tm_b[tr.p], full + st, kc * 64, tr.n_tile * pr.nt, 0);
+                    issued = g + 1;
                 }
-                issued = kc + 1;
             }
             if (*abort_flag)
-                for (int k = max(0, issued - STAGES); k < issued; ++k)
+                for (uint32_t k = issued > STAGES ? issued - STAGES : 0; k < issued; ++k)
                     mbar_wait_cycles(full + k % STAGES, (k / STAGES) & 1, 1ll << 22);
         }
     } else if (warp == MMA_WARP) {
         const uint32_t leader = elect_one_sync();
-        constexpr uint32_t idesc = idesc_bf16_f32(128, NT, false, false);
         const uint64_t a_desc0 = desc_sw128(smem_u32(smem), 16, 1024);
-        const uint64_t b_desc0 = desc_sw128(smem_u32(smem + A_CHUNK), 16, 1024);
+        const uint64_t b_desc0 = desc_sw128(smem_u32(smem + A_BYTES), 16, 1024);
+        uint32_t g = 0;
         bool ok = true;
-        for (int kc = 0; kc < nk; ++kc) {
-            const int st = kc % STAGES;
-            if (!__all_sync(0xffffffffu, mbar_wait(full + st, (kc / STAGES) & 1, abort_flag, ERR_SITE_PROLOGUE | 2))) {
+        int i = 0;
+        for (int t = blockIdx.x; ok && t < G.total_tiles; t += gridDim.x, ++i) {
+            const TileRef tr = decode_tile(G, t);
+            const ProjProblem &pr = G.prob[tr.p];
+            const int buf = i & 1, use = i >> 1;
+            if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(acc_empty + buf, (use - 1) & 1, abort_flag,
+                                                               ERR_SITE_PROLOGUE | 2))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t sb = st * C::STAGE;
+            const uint32_t idesc = idesc_bf16_f32(128, pr.nt, false, false);
+            const uint32_t d = tmem + buf * ACC_COLS;
+            for (int kc = 0; kc < pr.nk; ++kc, ++g) {
+                const uint32_t st = g % STAGES;
+                if (!__all_sync(0xffffffffu,
+                                mbar_wait(full + st, (g / STAGES) & 1, abort_flag, ERR_SITE_PROLOGUE | 3))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sb = st * STAGE;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                umma_ss_leader(tmem, a_desc0 + ((sb + kk * 32) >> 4), b_desc0 + ((sb + kk * 32) >> 4), idesc,
-                               (kc > 0 || kk > 0) ? 1u : 0u, leader);
-            umma_commit_leader(empty + st, leader);
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_ss_leader(d, a_desc0 + ((sb + kk * 32) >> 4), b_desc0 + ((sb + kk * 32) >> 4), idesc,
+                                   (kc > 0 || kk > 0) ? 1u : 0u, leader);
+                umma_commit_leader(empty + st, leader);
+            }
+            if (ok) umma_commit_leader(acc_full + buf, leader);
         }
-        if (ok) umma_commit_leader(mma_done, leader);
+        // every MMA this warp issued has finished before the TMEM is released
+        umma_commit_leader(drain, leader);
+        mbar_wait_cycles(drain, 0, 1ll << 22);
     } else {
         // ------------------------------ epilogue ----------------------------------
-        const int m = m0 + warp * 32 + lane;
-        const bool row_ok = m < M;
-        if (__all_sync(0xffffffffu, mbar_wait(mma_done, 0, abort_flag, ERR_SITE_PROLOGUE | 3))) {
+        const int q = warp & 3, hf = warp >> 2;
+        const uint32_t stg = smem_u32(smem + C::OFF_STG + warp * 2 * 4096);  // this warp's two output boxes
+        int i = 0;
+        for (int t = blockIdx.x; t < G.total_tiles; t += gridDim.x, ++i) {
+            const TileRef tr = decode_tile(G, t);
+            const int buf = i & 1, use = i >> 1;
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(acc_full + buf, use & 1, abort_flag, ERR_SITE_PROLOGUE | 4)))
+                break;
             tc_fence_after();
-            const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-            if constexpr (EPI == PRO_PLAIN) {
-                float *dst = io.f32_out + static_cast<size_t>(m) * io.ld_out + n0;
-#pragma unroll 1
-                for (int ch = 0; ch < NT / 32; ++ch) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_base + ch * 32, o);
-                    if (row_ok) {
-                        float4 *d4 = reinterpret_cast<float4 *>(dst + ch * 32);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            d4[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                                __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+            const uint32_t tcol = tmem + buf * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
+            const int m = tr.m0 + q * 32 + lane;
+            const bool row_ok = m < G.M;
+            const int epi = G.prob[tr.p].epi;
+            if constexpr (PHASE == 1) {
+                if (epi == PRO_CQ) epi_cq(io, tcol, m, row_ok, tr.n_tile, hf);
+                else if (epi == PRO_CKV) epi_ckv(io, plan, tcol, m, row_ok, tr.n_tile, hf, lane);
+                else if (epi == PRO_LAMBDA) epi_lambda(io, tcol, m, row_ok, tr.n_tile, hf);
+                else epi_gate(io, tcol, m, row_ok, tr.n_tile, hf);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(acc_empty + buf);
+            } else {
+                // this warp's boxes are free once its previous stores have read them
+                if (lane == 0) bulk_wait_group_read0();
+                __syncwarp();
+                int col0 = 0, n_box;
+                if (epi == PRO_QUP) n_box = epi_qup(io, tcol, m, row_ok, hf, lane, stg, col0);
+                else n_box = epi_kvup(io, tcol, m, row_ok, hf, lane, epi == PRO_KUP, stg, col0);
+                tc_fence_before();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(acc_empty + buf);
+                    const int row0 = tr.m0 + q * 32;
+                    if (row0 < G.M) {  // rows past the last token are clipped by the store
+                        const int hq = 4 * io.hkv;
+                        const CUtensorMap *map = epi == PRO_QUP ? (tr.n_tile < hq ? &G.tm_o[0] : &G.tm_o[1])
+                                                                : (epi == PRO_KUP ? &G.tm_o[2] : &G.tm_o[3]);
+                        const int head = (epi == PRO_QUP && tr.n_tile >= hq) ? tr.n_tile - hq : tr.n_tile;
+                        for (int b = 0; b < n_box; ++b)
+                            tma_store_3d(map, smem + C::OFF_STG + (warp * 2 + b) * 4096, col0 + 64 * b, head, row0);
+                        bulk_commit_group();
                     }
-                }
-            } else if constexpr (EPI == PRO_LAMBDA) {
-#pragma unroll 1
-                for (int ch = 0; ch < NT / 32; ++ch) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_base + ch * 32, o);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int n = n0 + ch * 32 + i;
-                        if (row_ok && n < io.n_out)
-                            io.lambda[static_cast<size_t>(m) * io.n_out + n] =
-                                1.f / (1.f + __expf(-__uint_as_float(o[i])));
-                    }
-                }
-            } else if constexpr (EPI == PRO_GATE) {
-                __nv_bfloat16 *dst = io.gate + static_cast<size_t>(m) * io.n_out + n0;
-#pragma unroll 1
-                for (int ch = 0; ch < NT / 32; ++ch) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_base + ch * 32, o);
-                    if (row_ok) {
-                        uint4 *d4 = reinterpret_cast<uint4 *>(dst + ch * 32);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            d4[i] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * i]), __uint_as_float(o[8 * i + 1])),
-                                               pack_bf16x2(__uint_as_float(o[8 * i + 2]), __uint_as_float(o[8 * i + 3])),
-                                               pack_bf16x2(__uint_as_float(o[8 * i + 4]), __uint_as_float(o[8 * i + 5])),
-                                               pack_bf16x2(__uint_as_float(o[8 * i + 6]), __uint_as_float(o[8 * i + 7])));
-                    }
-                }
-            } else if constexpr (EPI == PRO_QUP) {
-                // one query head: content dims 0..127, rotary dims 128..191 (pairs i, i+32)
-                const int h = tile_n;
-                __nv_bfloat16 *dst = (h < 4 * io.hkv)
-                                         ? io.q_sig + (static_cast<size_t>(m) * 4 * io.hkv + h) * 192
-                                         : io.q_noise + (static_cast<size_t>(m) * io.hkv + (h - 4 * io.hkv)) * 192;
-#pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_base + ch * 32, o);
-                    if (row_ok) store_bf16_32(dst + ch * 32, o);
-                }
-                uint32_t a[32], b[32];
-                tmem_ld32(lane_base + 128, a);
-                tmem_ld32(lane_base + 160, b);
-                if (row_ok) {
-                    const float *rot = io.rot + static_cast<size_t>(m) * 64;  // cos 0..31, sin 32..63
-                    uint32_t ra[32], rb[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float c = __ldg(rot + i), s = __ldg(rot + 32 + i);
-                        const float x0 = __uint_as_float(a[i]), x1 = __uint_as_float(b[i]);
-                        ra[i] = __float_as_uint(x0 * c - x1 * s);
-                        rb[i] = __float_as_uint(x0 * s + x1 * c);
-                    }
-                    store_bf16_32(dst + 128, ra);
-                    store_bf16_32(dst + 160, rb);
-                }
-            } else {  // PRO_KVUP: one KV head j: k_nope (cols 0..127), v (128..255), rotated k^R copied
-                const int j = tile_n;
-                __nv_bfloat16 *kd = io.k + (static_cast<size_t>(m) * io.hkv + j) * 192;
-                __nv_bfloat16 *vd = io.v + (static_cast<size_t>(m) * io.hkv + j) * 128;
-#pragma unroll 1
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t o[32];
-                    tmem_ld32(lane_base + ch * 32, o);
-                    if (row_ok) store_bf16_32(ch < 4 ? kd + ch * 32 : vd + (ch - 4) * 32, o);
-                }
-                if (row_ok) {
-                    const uint4 *kr = reinterpret_cast<const uint4 *>(io.krope + static_cast<size_t>(m) * 64);
-                    uint4 *kdst = reinterpret_cast<uint4 *>(kd + 128);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) kdst[i] = __ldg(kr + i);
                 }
             }
         }
+        if (PHASE == 2 && lane == 0) bulk_wait_group0();
     }
     tc_fence_before();
     __syncthreads();
     if (warp == MMA_WARP) {
         tc_fence_after();
-        tmem_dealloc(tmem, C::TMEM_COLS);
+        tmem_dealloc(tmem, TMEM_COLS);
     }
-}
-
-// Per token (one warp): RMSNorm of c^Q (1024) and c^KV (512) with their weights
-// into bf16 rows, the rotary table cos/sin(t base^(-i/32)) for i < 32 (angles and
-// their sine / cosine in fp64, stored fp32), and k^R rotated (bf16).
-__global__ void __launch_bounds__(256)
-gdla_prologue_norm_kernel(const PrologueIO io, const ProloguePlan plan, int M) {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-    if (warp >= M) return;
-    const int m = warp;
-    const float *cq = io.cq + static_cast<size_t>(m) * 1024;
-    const float *ckv = io.ckv + static_cast<size_t>(m) * 576;
-    float ss = 0.f;
-    for (int i = lane; i < 1024; i += 32) ss = fmaf(cq[i], cq[i], ss);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    const float rq = rsqrtf(ss * (1.f / 1024.f) + 1e-6f);
-    for (int i = lane; i < 1024; i += 32)
-        io.cq_n[static_cast<size_t>(m) * 1024 + i] = __float2bfloat16_rn(cq[i] * rq * io.gamma_q[i]);
-    ss = 0.f;
-    for (int i = lane; i < 512; i += 32) ss = fmaf(ckv[i], ckv[i], ss);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    const float rkv = rsqrtf(ss * (1.f / 512.f) + 1e-6f);
-    for (int i = lane; i < 512; i += 32)
-        io.ckv_n[static_cast<size_t>(m) * 512 + i] = __float2bfloat16_rn(ckv[i] * rkv * io.gamma_kv[i]);
-    // rotary table and k^R (lane = pair i of 32)
-    const double inv = exp2(-static_cast<double>(lane) * (13.287712379549449 / 32.0));  // 10000^(-i/32)
-    double s, c;
-    sincos(static_cast<double>(row_position(plan, m)) * inv, &s, &c);
-    io.rot[static_cast<size_t>(m) * 64 + lane] = static_cast<float>(c);
-    io.rot[static_cast<size_t>(m) * 64 + 32 + lane] = static_cast<float>(s);
-    const float x0 = ckv[512 + lane], x1 = ckv[512 + 32 + lane];
-    io.krope[static_cast<size_t>(m) * 64 + lane] =
-        __float2bfloat16_rn(static_cast<float>(x0 * c - x1 * s));
-    io.krope[static_cast<size_t>(m) * 64 + 32 + lane] =
-        __float2bfloat16_rn(static_cast<float>(x0 * s + x1 * c));
 }
 
 // ------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------
-template <int EPI, int NT>
-static cudaError_t launch_proj(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b2,
-                               const PrologueIO &io, int M, int K, int n_tiles, cudaStream_t stream) {
-    using C = ProjCfg<EPI, NT>;
+static void add_problem(ProjGroup &G, const CUtensorMap &a, const CUtensorMap &b, int epi, int nt, int K,
+                        int n_tiles) {
+    const int p = G.n_prob++;
+    G.tm_a[p] = a;
+    G.tm_b[p] = b;
+    G.prob[p] = ProjProblem{epi, nt, K / 64, n_tiles, G.total_tiles};
+    G.total_tiles += n_tiles * G.m_blocks;
+}
+
+template <int PHASE>
+static cudaError_t launch_group(const ProjGroup &G, const PrologueIO &io, const ProloguePlan &plan,
+                                cudaStream_t stream) {
     static PerContextFlag attr_set;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     const unsigned long long ctx = current_context_id();
     if (!attr_set.is_set(dev, ctx)) {
-        e = cudaFuncSetAttribute(gdla_proj_kernel<EPI, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES);
+        e = cudaFuncSetAttribute(gdla_proj_kernel<PHASE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 PhaseCfg<PHASE>::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set.set(dev, current_context_id());
     }
-    dim3 grid((M + 127) / 128, n_tiles);
-    gdla_proj_kernel<EPI, NT><<<grid, pg::NUM_THREADS, C::SMEM_BYTES, stream>>>(a, b, b2, io, M, K);
+    int sms = device_sm_count(dev);
+    if (sms <= 0) sms = 148;
+    const int grid = G.total_tiles < sms ? G.total_tiles : sms;
+    gdla_proj_kernel<PHASE><<<grid, pg::NUM_THREADS, PhaseCfg<PHASE>::SMEM_BYTES, stream>>>(G, io, plan);
     return cudaPeekAtLastError();
 }
 
 cudaError_t launch_prologue(const PrologueLaunch &L, const ProloguePlan &plan, int M, cudaStream_t stream) {
-    PrologueIO io = L.io;
-    const int hkv = io.hkv;
-    cudaError_t e;
-    // 1-4: projections of x
-    io.f32_out = io.cq, io.ld_out = 1024;
-    if ((e = launch_proj<PRO_PLAIN, 256>(L.tm_x, L.tm_wqa, L.tm_wqa, io, M, 4096, 4, stream)) != cudaSuccess) return e;
-    io.f32_out = io.ckv, io.ld_out = 576;
-    if ((e = launch_proj<PRO_PLAIN, 192>(L.tm_x, L.tm_wkva, L.tm_wkva, io, M, 4096, 3, stream)) != cudaSuccess) return e;
-    io.n_out = 4 * hkv;
-    if ((e = launch_proj<PRO_LAMBDA, 64>(L.tm_x, L.tm_wlam, L.tm_wlam, io, M, 4096, (4 * hkv + 63) / 64, stream)) !=
-        cudaSuccess)
-        return e;
-    io.n_out = 4 * hkv * 128;
-    if ((e = launch_proj<PRO_GATE, 256>(L.tm_x, L.tm_wgate, L.tm_wgate, io, M, 4096, 2 * hkv, stream)) != cudaSuccess)
-        return e;
-    // 5: norms, rotary table, rotated k^R
-    gdla_prologue_norm_kernel<<<(M + 7) / 8, 256, 0, stream>>>(io, plan, M);
-    if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-    // 6-7: up-projections
-    if ((e = launch_proj<PRO_QUP, 192>(L.tm_cqn, L.tm_wqb, L.tm_wqb, io, M, 1024, 5 * hkv, stream)) != cudaSuccess)
-        return e;
-    return launch_proj<PRO_KVUP, 256>(L.tm_ckvn, L.tm_wuk, L.tm_wuv, io, M, 512, hkv, stream);
+    const int hkv = L.io.hkv;
+    const int m_blocks = (M + 127) / 128;
+    // phase 1: the projections of x, widest tiles first (the tail gets the narrow ones)
+    ProjGroup g1{};
+    g1.m_blocks = m_blocks;
+    g1.M = M;
+    add_problem(g1, L.tm_x, L.tm_wgate, PRO_GATE, 256, 4096, 2 * hkv);
+    add_problem(g1, L.tm_x, L.tm_wqa, PRO_CQ, 256, 4096, 4);
+    add_problem(g1, L.tm_x, L.tm_wkva, PRO_CKV, 192, 4096, 3);
+    add_problem(g1, L.tm_x, L.tm_wlam, PRO_LAMBDA, 64, 4096, (4 * hkv + 63) / 64);
+    cudaError_t e = launch_group<1>(g1, L.io, plan, stream);
+    if (e != cudaSuccess) return e;
+    // phase 2: the up-projections
+    ProjGroup g2{};
+    g2.m_blocks = m_blocks;
+    g2.M = M;
+    g2.tm_o[0] = L.tm_qs_o;
+    g2.tm_o[1] = L.tm_qn_o;
+    g2.tm_o[2] = L.tm_k_o;
+    g2.tm_o[3] = L.tm_v_o;
+    add_problem(g2, L.tm_cqn, L.tm_wqb, PRO_QUP, 192, 1024, 5 * hkv);
+    add_problem(g2, L.tm_ckvn, L.tm_wuk, PRO_KUP, 128, 512, hkv);
+    add_problem(g2, L.tm_ckvn, L.tm_wuv, PRO_VUP, 128, 512, hkv);
+    return launch_group<2>(g2, L.io, plan, stream);
 }
 
 }  // namespace gdla

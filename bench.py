@@ -146,7 +146,7 @@ KERNEL_SOURCES = {
     "gdla_decode_latent_combine_kernel": ("gdla_decode_latent.cu", "gdla_ptx.cuh", "gdla_internal.h"),
     "gdla_bwd_dq_kernel": ("gdla_prefill_bwd.cu", "gdla_ptx.cuh", "gdla_internal.h"),
     "gdla_bwd_dkv_kernel": ("gdla_prefill_bwd.cu", "gdla_ptx.cuh", "gdla_internal.h"),
-    "gdla_proj_kernel": ("gdla_prologue.cu", "gdla_ptx.cuh", "gdla_internal.h"),
+    "gdla_proj_kernel": ("gdla_prologue.cu", "gdla_prologue.h", "gdla_pair.cuh", "gdla_ptx.cuh", "gdla_internal.h"),
 }
 
 

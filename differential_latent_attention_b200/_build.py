@@ -17,7 +17,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG, "libgdla.so")
 SOURCES = ["gdla_lib.cu", "gdla_api.cu", "gdla_prefill.cu", "gdla_prefill_bwd.cu", "gdla_prologue.cu", "gdla_decode.cu", "gdla_decode_noalloc.cu",
-           "gdla_decode_latent.cu", "gdla_selftest.cu", "gdla_internal.h", "gdla_ptx.cuh"]
+           "gdla_decode_latent.cu", "gdla_selftest.cu", "gdla_internal.h", "gdla_ptx.cuh", "gdla_prologue.h",
+           "gdla_pair.cuh"]
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -12,6 +12,7 @@
 
 #include "gdla.h"
 #include "gdla_internal.h"
+#include "gdla_prologue.h"
 #include "gdla_ptx.cuh"
 
 namespace gdla {
@@ -460,16 +461,17 @@ gdla_status_t gdla_prologue(const void *x, const void *w_qa, const void *w_kva, 
     L.io.k = static_cast<__nv_bfloat16 *>(k);
     L.io.v = static_cast<__nv_bfloat16 *>(v);
     L.io.hkv = hkv;
-    // 2-D bf16 operands as [rows][K] maps with 64-wide K boxes (128-byte swizzle)
-    if (!make_map(&L.tm_x, x, 4096, N, 1, 64, 128, 1) || !make_map(&L.tm_wqa, w_qa, 4096, 1024, 1, 64, 256, 1) ||
-        !make_map(&L.tm_wkva, w_kva, 4096, 576, 1, 64, 192, 1) ||
-        !make_map(&L.tm_wlam, w_lambda, 4096, 4 * hkv, 1, 64, 64, 1) ||
-        !make_map(&L.tm_wgate, w_gate, 4096, 4ull * hkv * 128, 1, 64, 256, 1) ||
+    // 2-D bf16 operands as [rows][K] maps with 64-wide K boxes (128-byte swizzle); the
+    // weights' boxes are half a tile's columns (each CTA of a pair loads one half)
+    if (!make_map(&L.tm_x, x, 4096, N, 1, 64, 128, 1) || !make_map(&L.tm_wqa, w_qa, 4096, 1024, 1, 64, 128, 1) ||
+        !make_map(&L.tm_wkva, w_kva, 4096, 576, 1, 64, 96, 1) ||
+        !make_map(&L.tm_wlam, w_lambda, 4096, 4 * hkv, 1, 64, 32, 1) ||
+        !make_map(&L.tm_wgate, w_gate, 4096, 4ull * hkv * 128, 1, 64, 128, 1) ||
         !make_map(&L.tm_cqn, L.io.cq_g, 1024, N, 1, 64, 128, 1) ||
-        !make_map(&L.tm_wqb, w_qb, 1024, 5ull * hkv * 192, 1, 64, 192, 1) ||
+        !make_map(&L.tm_wqb, w_qb, 1024, 5ull * hkv * 192, 1, 64, 96, 1) ||
         !make_map(&L.tm_ckvn, L.io.ckv_g, 512, N, 1, 64, 128, 1) ||
-        !make_map(&L.tm_wuk, w_uk, 512, 128ull * hkv, 1, 64, 128, 1) ||
-        !make_map(&L.tm_wuv, w_uv, 512, 128ull * hkv, 1, 64, 128, 1) ||
+        !make_map(&L.tm_wuk, w_uk, 512, 128ull * hkv, 1, 64, 64, 1) ||
+        !make_map(&L.tm_wuv, w_uv, 512, 128ull * hkv, 1, 64, 64, 1) ||
         !make_map(&L.tm_qs_o, q_sig, 192, 4ull * hkv, N, 64, 1, 32) ||
         !make_map(&L.tm_qn_o, q_noise, 192, hkv, N, 64, 1, 32) || !make_map(&L.tm_k_o, k, 192, hkv, N, 64, 1, 32) ||
         !make_map(&L.tm_v_o, v, 128, hkv, N, 64, 1, 32))

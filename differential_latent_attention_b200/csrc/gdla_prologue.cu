@@ -23,16 +23,21 @@
 //            by the row's rsqrt, rotary 64 columns rotated) -> q_sig, q_noise; and
 //            (c^KV * gamma_kv) W^UK_j, (c^KV * gamma_kv) W^UV_j (K = 512, one KV head per
 //            128-column tile, scaled) -> k = [k_nope | rotated k^R], v.
-// The GEMM: one CTA per SM walks its tiles (t = blockIdx.x, + gridDim.x, ...); a TMA
-// producer warp streams 64-wide K chunks of A (128 rows) and B (the weights' rows)
-// through a 4- or 5-stage ring; one elected thread issues tcgen05 MMAs (M = 128, N = nt, fp32)
-// into one of two TMEM accumulators, so 8 epilogue warps (TMEM lane quarter = warp % 4,
-// column half = warp / 4) drain one tile while the next one is multiplied.
+// The GEMM: CTA pairs (clusters of two, one CTA per SM) walk 256-row x nt-column tiles
+// (t = pair, + pairs, ...). In each CTA a TMA producer warp streams 64-wide K chunks of
+// its 128 rows of A and its half of the tile's B rows (the weights' rows) through a
+// 6-stage ring; one elected thread of the even CTA issues the pair's tcgen05 MMAs
+// (cta_group::2, M = 256, N = nt, fp32) into one of two TMEM accumulators, so 8
+// epilogue warps per CTA (TMEM lane quarter = warp % 4, column half = warp / 4) drain
+// one tile while the next one is multiplied. Each SM loads 128 + nt/2 operand rows
+// per K chunk instead of 128 + nt.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "gdla_internal.h"
+#include "gdla_prologue.h"
+#include "gdla_pair.cuh"
 #include "gdla_ptx.cuh"
 
 namespace gdla {
@@ -61,21 +66,23 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int SSQ = 16;                        // partial sums of squares per row
 }  // namespace pg
 
-// Shared memory of a phase: a 4-stage ring for B tiles up to 256 rows (phase 1) or
-// 192 rows (phase 2); phase 2 adds two 4 KB output boxes (32 rows x 64 bf16, 128-byte
-// swizzle) per epilogue warp, which its TMA stores read.
+// Shared memory of a phase: a 6-stage ring of A chunks and half-B chunks (up to 128
+// rows in phase 1, 96 in phase 2: the up-projections' short MMAs per chunk need
+// about as many loads in flight as the long ones); phase 2 adds three 4 KB output
+// boxes (32 rows x 64 bf16, 128-byte swizzle) per TMEM lane quarter, shared by the
+// quarter's two epilogue warps and read by their TMA stores.
 template <int PHASE>
 struct PhaseCfg {
-    static constexpr int STAGES = 4;
-    static constexpr int B_ROWS = PHASE == 1 ? 256 : 192;
+    static constexpr int STAGES = 6;
+    static constexpr int B_ROWS = PHASE == 1 ? 128 : 96;
     static constexpr int STAGE = pg::A_BYTES + B_ROWS * 128;
     static constexpr int OFF_STG = STAGES * STAGE;
-    static constexpr int STG_BYTES = PHASE == 1 ? 0 : pg::EPI_WARPS * 2 * 4096;
+    static constexpr int STG_BYTES = PHASE == 1 ? 0 : 4 * 3 * 4096;
     static constexpr int OFF_BAR = OFF_STG + STG_BYTES;  // full[S], empty[S], acc_full[2], acc_empty[2], drain
-    static constexpr int OFF_MISC = OFF_BAR + 16 * 8;
+    static constexpr int OFF_MISC = OFF_BAR + 32 * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    static_assert(2 * STAGES + 5 <= 16, "barrier slots");
+    static_assert(2 * STAGES + 9 <= 32, "barrier slots");
 };
 
 // Position of packed row m in its sequence (starts[] = cumulative sequence starts).
@@ -91,11 +98,12 @@ __device__ __forceinline__ int row_position(const ProloguePlan &p, int m) {
 struct TileRef {
     int p, n_tile, m0;
 };
+// Tile t: problem p, column tile n_tile, first row m0 of its 256-row pair block.
 __device__ __forceinline__ TileRef decode_tile(const ProjGroup &G, int t) {
     int p = 0;
     while (p + 1 < G.n_prob && t >= G.prob[p + 1].first) ++p;
     const int local = t - G.prob[p].first;
-    return {p, local / G.m_blocks, (local % G.m_blocks) * 128};
+    return {p, local / G.m_pairs, (local % G.m_pairs) * 256};
 }
 
 // ------------------------------ phase 1 epilogues -----------------------------
@@ -220,14 +228,6 @@ __device__ __forceinline__ void scale_32(uint32_t (&o)[32], float r) {
     for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * r);
 }
 
-// rsqrt(mean of squares + eps) of row m from its partial sums [first, first + count).
-__device__ __forceinline__ float row_rsqrt(const PrologueIO &io, int m, int first, int count, float inv_width) {
-    const float *p = io.ssq + static_cast<size_t>(m) * pg::SSQ + first;
-    float ss = 0.f;
-    for (int i = 0; i < count; ++i) ss += __ldg(p + i);
-    return rsqrtf(ss * inv_width + 1e-6f);
-}
-
 // 32 fp32 values (as bits) x r -> bf16 into 16-byte chunks c0..c0+3 of this lane's
 // 128-byte row of a 128-byte-swizzled output box at shared address `box`.
 __device__ __forceinline__ void stage_32(uint32_t box, int lane, int c0, const uint32_t (&o)[32], float r) {
@@ -242,12 +242,42 @@ __device__ __forceinline__ void stage_32(uint32_t box, int lane, int c0, const u
     }
 }
 
-// One query head h (tile n = h) into this warp's output boxes: half 0 the content dims
-// 0..127 (two boxes), half 1 the rotary dims 128..191 (pairs i, i+32) rotated. Returns
-// the number of boxes staged; box b goes to dims col0 + 64 b.
-__device__ __forceinline__ int epi_qup(const PrologueIO &io, uint32_t tcol, int m, bool row_ok, int hf, int lane,
-                                       uint32_t stg, int &col0) {
-    const float r = row_ok ? row_rsqrt(io, m, 0, 8, 1.f / 1024.f) : 0.f;
+// Row data an up-projection epilogue reads besides the accumulator, loaded before
+// the accumulator is waited for: the partial sums of squares and, for half 1, the
+// row's rotary cos | sin (query tiles) or rotated k^R (k_nope tiles).
+struct Epi2Row {
+    float4 ss0, ss1;
+    float4 rot[16];
+};
+__device__ __forceinline__ void epi2_prefetch(const PrologueIO &io, int m, bool row_ok, int epi, int hf,
+                                              Epi2Row &d) {
+    const bool qup = epi == PRO_QUP;
+    const size_t row = static_cast<size_t>(row_ok ? m : 0);
+    const float4 *p = reinterpret_cast<const float4 *>(io.ssq + row * pg::SSQ);
+    d.ss0 = __ldg(p + (qup ? 0 : 2));
+    d.ss1 = __ldg(p + (qup ? 1 : 3));
+    if (hf == 1 && qup) {
+        const float4 *rot = reinterpret_cast<const float4 *>(io.rot + row * 64);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) d.rot[i] = __ldg(rot + i);
+    } else if (hf == 1 && epi == PRO_KUP) {
+        const float4 *kr = reinterpret_cast<const float4 *>(io.krope + row * 64);  // 64 bf16
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d.rot[i] = __ldg(kr + i);
+    }
+}
+// rsqrt(mean of squares + eps): c^Q from partial sums 0..7, c^KV from 8..13.
+__device__ __forceinline__ float epi2_rsqrt(const Epi2Row &d, bool qup, bool row_ok) {
+    if (!row_ok) return 0.f;
+    const float s = (d.ss0.x + d.ss0.y) + (d.ss0.z + d.ss0.w) + (d.ss1.x + d.ss1.y);
+    return qup ? rsqrtf((s + (d.ss1.z + d.ss1.w)) * (1.f / 1024.f) + 1e-6f) : rsqrtf(s * (1.f / 512.f) + 1e-6f);
+}
+
+// One query head (tile n = head) into the quarter's output boxes `stg`: half 0 the
+// content dims 0..127 (boxes 0, 1), half 1 the rotary dims 128..191 (pairs i, i+32)
+// rotated (box 2).
+__device__ __forceinline__ void epi_qup(const Epi2Row &d, float r, uint32_t tcol, bool row_ok, int hf, int lane,
+                                        uint32_t stg) {
     if (hf == 0) {
 #pragma unroll 1
         for (int ch = 0; ch < 4; ++ch) {
@@ -255,17 +285,15 @@ __device__ __forceinline__ int epi_qup(const PrologueIO &io, uint32_t tcol, int 
             tmem_ld32(tcol + ch * 32, o);
             stage_32(stg + (ch >> 1) * 4096, lane, (ch & 1) * 4, o, r);
         }
-        col0 = 0;
-        return 2;
+        return;
     }
     uint32_t a[32], b[32];
     tmem_ld32(tcol + 128, a);
     tmem_ld32(tcol + 160, b);
     if (row_ok) {
-        const float4 *rot = reinterpret_cast<const float4 *>(io.rot + static_cast<size_t>(m) * 64);  // cos | sin
 #pragma unroll
         for (int i4 = 0; i4 < 8; ++i4) {
-            const float4 c4 = __ldg(rot + i4), s4 = __ldg(rot + 8 + i4);
+            const float4 c4 = d.rot[i4], s4 = d.rot[8 + i4];
             const float cv[4] = {c4.x, c4.y, c4.z, c4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -276,34 +304,29 @@ __device__ __forceinline__ int epi_qup(const PrologueIO &io, uint32_t tcol, int 
             }
         }
     }
-    stage_32(stg, lane, 0, a, r);
-    stage_32(stg, lane, 4, b, r);
-    col0 = 128;
-    return 1;
+    stage_32(stg + 2 * 4096, lane, 0, a, r);
+    stage_32(stg + 2 * 4096, lane, 4, b, r);
 }
 
-// One KV head j (tile n = j) of k_nope (PRO_KUP) or v (PRO_VUP), 64 dims per half;
-// half 1 of k_nope also stages the rotated k^R (k's dims 128..191) as its second box.
-__device__ __forceinline__ int epi_kvup(const PrologueIO &io, uint32_t tcol, int m, bool row_ok, int hf, int lane,
-                                        bool is_k, uint32_t stg, int &col0) {
-    const float r = row_ok ? row_rsqrt(io, m, 8, 6, 1.f / 512.f) : 0.f;
+// One KV head j (tile n = j) of k_nope (PRO_KUP) or v (PRO_VUP): half hf stages
+// dims 64 hf .. 64 hf + 63 in box hf; half 1 of k_nope also stages the rotated k^R
+// (k's dims 128..191) in box 2.
+__device__ __forceinline__ void epi_kvup(const Epi2Row &d, float r, uint32_t tcol, bool is_k, int hf, int lane,
+                                         uint32_t stg) {
 #pragma unroll 1
     for (int ch = 0; ch < 2; ++ch) {
         uint32_t o[32];
         tmem_ld32(tcol + hf * 64 + ch * 32, o);
-        stage_32(stg, lane, ch * 4, o, r);
+        stage_32(stg + hf * 4096, lane, ch * 4, o, r);
     }
-    col0 = hf * 64;
-    if (!(is_k && hf == 1)) return 1;
-    const uint32_t row = stg + 4096 + lane * 128;
-    const uint4 *kr = reinterpret_cast<const uint4 *>(io.krope + static_cast<size_t>(row_ok ? m : 0) * 64);
+    if (!(is_k && hf == 1)) return;
+    const uint32_t row = stg + 2 * 4096 + lane * 128;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const uint4 v = __ldg(kr + i);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        const float4 v = d.rot[i];
+        const uint32_t w[4] = {__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z), __float_as_uint(v.w)};
         sts128(row + ((i ^ (lane & 7)) << 4), w);
     }
-    return 2;
 }
 
 // ------------------------------------------------------------------------------
@@ -311,7 +334,7 @@ __device__ __forceinline__ int epi_kvup(const PrologueIO &io, uint32_t tcol, int
 // PRO_LAMBDA problems; PHASE 2 PRO_QUP, PRO_KUP and PRO_VUP.
 // ------------------------------------------------------------------------------
 template <int PHASE>
-__global__ void __launch_bounds__(pg::NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pg::NUM_THREADS, 1)
 gdla_proj_kernel(const __grid_constant__ ProjGroup G, const __grid_constant__ PrologueIO io,
                  const __grid_constant__ ProloguePlan plan) {
     using namespace pg;
@@ -325,9 +348,13 @@ gdla_proj_kernel(const __grid_constant__ ProjGroup G, const __grid_constant__ Pr
     uint64_t *acc_full = bars + 2 * STAGES;  // [accumulator]
     uint64_t *acc_empty = acc_full + 2;      // [accumulator]
     uint64_t *drain = acc_empty + 2;
+    uint64_t *qfree = drain + 1;            // [lane quarter] (phase 2): its output boxes are free
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool even = rank == 0;
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; ++i) {
@@ -336,18 +363,19 @@ gdla_proj_kernel(const __grid_constant__ ProjGroup G, const __grid_constant__ Pr
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(acc_full + i, 1);
-            mbar_init(acc_empty + i, EPI_WARPS);
+            mbar_init(acc_empty + i, 2 * EPI_WARPS);  // both CTAs' epilogue warps (the even CTA's copy)
         }
         mbar_init(drain, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(qfree + i, 2);
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == MMA_WARP) {
-        tmem_alloc(tmem_slot, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // both CTAs' barriers are initialised before either signals the other
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
@@ -355,51 +383,54 @@ gdla_proj_kernel(const __grid_constant__ ProjGroup G, const __grid_constant__ Pr
         if (lane == 0) {
             uint32_t g = 0, issued = 0;
             bool ok = true;
-            for (int t = blockIdx.x; ok && t < G.total_tiles; t += gridDim.x) {
+            for (int t = pair; ok && t < G.total_tiles; t += n_pairs) {
                 const TileRef tr = decode_tile(G, t);
                 const ProjProblem &pr = G.prob[tr.p];
-                const uint32_t bytes = A_BYTES + pr.nt * 128;
+                const int half = pr.nt >> 1;
+                const uint32_t bytes = 2 * (A_BYTES + half * 128);  // both CTAs' loads
                 for (int kc = 0; kc < pr.nk; ++kc, ++g) {
                     const uint32_t st = g % STAGES;
                     if (g >= STAGES &&
-                        !mbar_wait(empty + st, ((g / STAGES) + 1) & 1, abort_flag, ERR_SITE_PROLOGUE | 1)) {
+                        !mbar_wait_cl(empty + st, ((g / STAGES) + 1) & 1, abort_flag, ERR_SITE_PROLOGUE | 1)) {
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(full + st, bytes);
+                    if (even) mbar_arrive_expect_tx(full + st, bytes);
                     uint8_t *sb = smem + st * STAGE;
-                    tma_load_3d(sb, &G.tm_a[tr.p], full + st, kc * 64, tr.m0, 0);
-                    tma_load_3d(sb + A_BYTES, &G.tm_b[tr.p], full + st, kc * 64, tr.n_tile * pr.nt, 0);
+                    tma_load_3d_pair(sb, &G.tm_a[tr.p], full + st, kc * 64, tr.m0 + 128 * rank, 0);
+                    tma_load_3d_pair(sb + A_BYTES, &G.tm_b[tr.p], full + st, kc * 64,
+                                     tr.n_tile * pr.nt + half * rank, 0);
                     issued = g + 1;
                 }
             }
-            if (*abort_flag)
+            if (*abort_flag && even)
                 for (uint32_t k = issued > STAGES ? issued - STAGES : 0; k < issued; ++k)
-                    mbar_wait_cycles(full + k % STAGES, (k / STAGES) & 1, 1ll << 22);
+                    mbar_wait_cl_cycles(full + k % STAGES, (k / STAGES) & 1, 1ll << 22);
         }
     } else if (warp == MMA_WARP) {
+        if (even) {  // the pair's MMAs are issued by the even CTA
         const uint32_t leader = elect_one_sync();
         const uint64_t a_desc0 = desc_sw128(smem_u32(smem), 16, 1024);
         const uint64_t b_desc0 = desc_sw128(smem_u32(smem + A_BYTES), 16, 1024);
         uint32_t g = 0;
         bool ok = true;
         int i = 0;
-        for (int t = blockIdx.x; ok && t < G.total_tiles; t += gridDim.x, ++i) {
+        for (int t = pair; ok && t < G.total_tiles; t += n_pairs, ++i) {
             const TileRef tr = decode_tile(G, t);
             const ProjProblem &pr = G.prob[tr.p];
             const int buf = i & 1, use = i >> 1;
-            if (use > 0 && !__all_sync(0xffffffffu, mbar_wait(acc_empty + buf, (use - 1) & 1, abort_flag,
-                                                               ERR_SITE_PROLOGUE | 2))) {
+            if (use > 0 && !__all_sync(0xffffffffu, mbar_wait_cl(acc_empty + buf, (use - 1) & 1, abort_flag,
+                                                                  ERR_SITE_PROLOGUE | 2))) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t idesc = idesc_bf16_f32(128, pr.nt, false, false);
+            const uint32_t idesc = idesc_bf16_f32(256, pr.nt, false, false);
             const uint32_t d = tmem + buf * ACC_COLS;
             for (int kc = 0; kc < pr.nk; ++kc, ++g) {
                 const uint32_t st = g % STAGES;
                 if (!__all_sync(0xffffffffu,
-                                mbar_wait(full + st, (g / STAGES) & 1, abort_flag, ERR_SITE_PROLOGUE | 3))) {
+                                mbar_wait_cl(full + st, (g / STAGES) & 1, abort_flag, ERR_SITE_PROLOGUE | 3))) {
                     ok = false;
                     break;
                 }
@@ -407,31 +438,36 @@ gdla_proj_kernel(const __grid_constant__ ProjGroup G, const __grid_constant__ Pr
                 const uint32_t sb = st * STAGE;
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
-                    umma_ss_leader(d, a_desc0 + ((sb + kk * 32) >> 4), b_desc0 + ((sb + kk * 32) >> 4), idesc,
-                                   (kc > 0 || kk > 0) ? 1u : 0u, leader);
-                umma_commit_leader(empty + st, leader);
+                    umma_ss_pair_leader(d, a_desc0 + ((sb + kk * 32) >> 4), b_desc0 + ((sb + kk * 32) >> 4), idesc,
+                                        (kc > 0 || kk > 0) ? 1u : 0u, leader);
+                umma_commit_pair_leader(empty + st, leader);
             }
-            if (ok) umma_commit_leader(acc_full + buf, leader);
+            if (ok) umma_commit_pair_leader(acc_full + buf, leader);
         }
         // every MMA this warp issued has finished before the TMEM is released
-        umma_commit_leader(drain, leader);
-        mbar_wait_cycles(drain, 0, 1ll << 22);
+        umma_commit_pair_leader(drain, leader);
+        mbar_wait_cl_cycles(drain, 0, 1ll << 22);
+        }
     } else {
         // ------------------------------ epilogue ----------------------------------
         const int q = warp & 3, hf = warp >> 2;
-        const uint32_t stg = smem_u32(smem + C::OFF_STG + warp * 2 * 4096);  // this warp's two output boxes
+        const uint32_t stg = smem_u32(smem + C::OFF_STG + q * 3 * 4096);  // the quarter's output boxes
+        const uint32_t acc_empty_even = mapa_shared(smem_u32(acc_empty), 0);
         int i = 0;
-        for (int t = blockIdx.x; t < G.total_tiles; t += gridDim.x, ++i) {
-            const TileRef tr = decode_tile(G, t);
+        for (int t = pair; t < G.total_tiles; t += n_pairs, ++i) {
+            TileRef tr = decode_tile(G, t);
+            tr.m0 += 128 * rank;  // this CTA's rows of the pair block
             const int buf = i & 1, use = i >> 1;
-            if (!__all_sync(0xffffffffu,
-                            mbar_wait(acc_full + buf, use & 1, abort_flag, ERR_SITE_PROLOGUE | 4)))
-                break;
-            tc_fence_after();
-            const uint32_t tcol = tmem + buf * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
             const int m = tr.m0 + q * 32 + lane;
             const bool row_ok = m < G.M;
             const int epi = G.prob[tr.p].epi;
+            Epi2Row pre;
+            if constexpr (PHASE == 2) epi2_prefetch(io, m, row_ok, epi, hf, pre);
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait_cl(acc_full + buf, use & 1, abort_flag, ERR_SITE_PROLOGUE | 4)))
+                break;
+            tc_fence_after();
+            const uint32_t tcol = tmem + buf * ACC_COLS + (static_cast<uint32_t>(q * 32) << 16);
             if constexpr (PHASE == 1) {
                 if (epi == PRO_CQ) epi_cq(io, tcol, m, row_ok, tr.n_tile, hf);
                 else if (epi == PRO_CKV) epi_ckv(io, plan, tcol, m, row_ok, tr.n_tile, hf, lane);
@@ -439,27 +475,36 @@ gdla_proj_kernel(const __grid_constant__ ProjGroup G, const __grid_constant__ Pr
                 else epi_gate(io, tcol, m, row_ok, tr.n_tile, hf);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(acc_empty + buf);
+                if (lane == 0) mbar_arrive_cluster(acc_empty_even + buf * 8);
             } else {
-                // this warp's boxes are free once its previous stores have read them
-                if (lane == 0) bulk_wait_group_read0();
-                __syncwarp();
-                int col0 = 0, n_box;
-                if (epi == PRO_QUP) n_box = epi_qup(io, tcol, m, row_ok, hf, lane, stg, col0);
-                else n_box = epi_kvup(io, tcol, m, row_ok, hf, lane, epi == PRO_KUP, stg, col0);
+                // the quarter's boxes are free once both its warps' previous stores have read them
+                if (lane == 0) {
+                    bulk_wait_group_read0();
+                    mbar_arrive(qfree + q);
+                }
+                if (!__all_sync(0xffffffffu, mbar_wait(qfree + q, i & 1, abort_flag, ERR_SITE_PROLOGUE | 5)))
+                    break;
+                const bool qup = epi == PRO_QUP;
+                const float r = epi2_rsqrt(pre, qup, row_ok);
+                if (qup) epi_qup(pre, r, tcol, row_ok, hf, lane, stg);
+                else epi_kvup(pre, r, tcol, epi == PRO_KUP, hf, lane, stg);
                 tc_fence_before();
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(acc_empty + buf);
+                    mbar_arrive_cluster(acc_empty_even + buf * 8);
                     const int row0 = tr.m0 + q * 32;
                     if (row0 < G.M) {  // rows past the last token are clipped by the store
                         const int hq = 4 * io.hkv;
-                        const CUtensorMap *map = epi == PRO_QUP ? (tr.n_tile < hq ? &G.tm_o[0] : &G.tm_o[1])
-                                                                : (epi == PRO_KUP ? &G.tm_o[2] : &G.tm_o[3]);
-                        const int head = (epi == PRO_QUP && tr.n_tile >= hq) ? tr.n_tile - hq : tr.n_tile;
-                        for (int b = 0; b < n_box; ++b)
-                            tma_store_3d(map, smem + C::OFF_STG + (warp * 2 + b) * 4096, col0 + 64 * b, head, row0);
+                        const CUtensorMap *map = qup ? (tr.n_tile < hq ? &G.tm_o[0] : &G.tm_o[1])
+                                                     : (epi == PRO_KUP ? &G.tm_o[2] : &G.tm_o[3]);
+                        const int head = (qup && tr.n_tile >= hq) ? tr.n_tile - hq : tr.n_tile;
+                        // this warp's boxes: query half 0 -> 0, 1; half 1 -> 2; k / v half hf -> hf
+                        // (and k's half 1 -> 2 as well); box b holds dims 64 b .. 64 b + 63
+                        const int b_lo = qup ? (hf ? 2 : 0) : hf;
+                        const int b_hi = qup ? (hf ? 2 : 1) : (epi == PRO_KUP && hf ? 2 : hf);
+                        for (int b = b_lo; b <= b_hi; ++b)
+                            tma_store_3d(map, smem + C::OFF_STG + (q * 3 + b) * 4096, 64 * b, head, row0);
                         bulk_commit_group();
                     }
                 }
@@ -468,23 +513,24 @@ gdla_proj_kernel(const __grid_constant__ ProjGroup G, const __grid_constant__ Pr
         if (PHASE == 2 && lane == 0) bulk_wait_group0();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // no CTA leaves while the pair's MMAs or the peer may still touch it
     if (warp == MMA_WARP) {
         tc_fence_after();
-        tmem_dealloc(tmem, TMEM_COLS);
+        tmem_dealloc_pair(tmem, TMEM_COLS);
     }
 }
 
 // ------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------
+// The tile's nt B rows are rows n_tile nt .. of b; each CTA of a pair loads one half.
 static void add_problem(ProjGroup &G, const CUtensorMap &a, const CUtensorMap &b, int epi, int nt, int K,
                         int n_tiles) {
     const int p = G.n_prob++;
     G.tm_a[p] = a;
     G.tm_b[p] = b;
     G.prob[p] = ProjProblem{epi, nt, K / 64, n_tiles, G.total_tiles};
-    G.total_tiles += n_tiles * G.m_blocks;
+    G.total_tiles += n_tiles * G.m_pairs;
 }
 
 template <int PHASE>
@@ -501,19 +547,40 @@ static cudaError_t launch_group(const ProjGroup &G, const PrologueIO &io, const 
         if (e != cudaSuccess) return e;
         attr_set.set(dev, current_context_id());
     }
-    int sms = device_sm_count(dev);
-    if (sms <= 0) sms = 148;
-    const int grid = G.total_tiles < sms ? G.total_tiles : sms;
-    gdla_proj_kernel<PHASE><<<grid, pg::NUM_THREADS, PhaseCfg<PHASE>::SMEM_BYTES, stream>>>(G, io, plan);
+    // as many pairs as can be resident at once (a cluster's two CTAs need two SMs of
+    // one GPC, so this can be below half the SM count)
+    static std::atomic<int> max_clusters[kMaxCachedDevices];
+    static PerContextFlag clusters_known;
+    int nc = 0;
+    if (dev >= 0 && dev < kMaxCachedDevices && clusters_known.is_set(dev, ctx)) {
+        nc = max_clusters[dev].load(std::memory_order_relaxed);
+    } else {
+        int sms = device_sm_count(dev);
+        if (sms <= 0) sms = 148;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1));
+        cfg.blockDim = dim3(pg::NUM_THREADS);
+        cfg.dynamicSmemBytes = PhaseCfg<PHASE>::SMEM_BYTES;
+        e = cudaOccupancyMaxActiveClusters(&nc, gdla_proj_kernel<PHASE>, &cfg);
+        if (e != cudaSuccess) return e;
+        if (nc <= 0) return cudaErrorInvalidConfiguration;
+        nc = nc < sms / 2 ? nc : sms / 2;
+        if (dev >= 0 && dev < kMaxCachedDevices) {
+            max_clusters[dev].store(nc, std::memory_order_relaxed);
+            clusters_known.set(dev, ctx);
+        }
+    }
+    const int pairs = G.total_tiles < nc ? G.total_tiles : nc;
+    gdla_proj_kernel<PHASE><<<2 * pairs, pg::NUM_THREADS, PhaseCfg<PHASE>::SMEM_BYTES, stream>>>(G, io, plan);
     return cudaPeekAtLastError();
 }
 
 cudaError_t launch_prologue(const PrologueLaunch &L, const ProloguePlan &plan, int M, cudaStream_t stream) {
     const int hkv = L.io.hkv;
-    const int m_blocks = (M + 127) / 128;
+    const int m_pairs = (M + 255) / 256;
     // phase 1: the projections of x, widest tiles first (the tail gets the narrow ones)
     ProjGroup g1{};
-    g1.m_blocks = m_blocks;
+    g1.m_pairs = m_pairs;
     g1.M = M;
     add_problem(g1, L.tm_x, L.tm_wgate, PRO_GATE, 256, 4096, 2 * hkv);
     add_problem(g1, L.tm_x, L.tm_wqa, PRO_CQ, 256, 4096, 4);
@@ -523,7 +590,7 @@ cudaError_t launch_prologue(const PrologueLaunch &L, const ProloguePlan &plan, i
     if (e != cudaSuccess) return e;
     // phase 2: the up-projections
     ProjGroup g2{};
-    g2.m_blocks = m_blocks;
+    g2.m_pairs = m_pairs;
     g2.M = M;
     g2.tm_o[0] = L.tm_qs_o;
     g2.tm_o[1] = L.tm_qn_o;

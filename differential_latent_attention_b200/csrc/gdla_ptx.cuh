@@ -20,7 +20,6 @@ enum : int {
     ERR_SITE_DECODE = 2 << 16,
     ERR_SITE_LATENT = 4 << 16,
     ERR_SITE_BWD = 8 << 16,
-    ERR_SITE_PROLOGUE = 16 << 16,
 };
 
 // About 2^31 SM cycles (~1 s at 1.9 GHz): far above any legitimate wait.

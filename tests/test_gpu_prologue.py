@@ -57,6 +57,16 @@ def test_sixteen_groups():
     check_prologue((300, 77), 16, 4)
 
 
+def test_three_groups():
+    # 4H = 12 lambda columns (one partly filled 64-column tile), 15 query heads
+    check_prologue((129, 258), 3, 6)
+
+
+def test_bench_size():
+    # the bench's prologue workload in full: 4096 tokens, 16 KV groups (every output element)
+    check_prologue((4096,), 16, 1)
+
+
 def test_feeds_attention():
     """The prologue's outputs are accepted by attn_fwd as they are."""
     seqlens = (200,)

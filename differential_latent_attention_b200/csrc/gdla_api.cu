@@ -468,7 +468,7 @@ gdla_status_t gdla_prologue(const void *x, const void *w_qa, const void *w_kva, 
         !make_map(&L.tm_wlam, w_lambda, 4096, 4 * hkv, 1, 64, 32, 1) ||
         !make_map(&L.tm_wgate, w_gate, 4096, 4ull * hkv * 128, 1, 64, 128, 1) ||
         !make_map(&L.tm_cqn, L.io.cq_g, 1024, N, 1, 64, 128, 1) ||
-        !make_map(&L.tm_wqb, w_qb, 1024, 5ull * hkv * 192, 1, 64, 96, 1) ||
+        !make_map(&L.tm_wqb, w_qb, 1024, 5ull * hkv * 192, 1, 64, 128, 1) ||
         !make_map(&L.tm_ckvn, L.io.ckv_g, 512, N, 1, 64, 128, 1) ||
         !make_map(&L.tm_wuk, w_uk, 512, 128ull * hkv, 1, 64, 64, 1) ||
         !make_map(&L.tm_wuv, w_uv, 512, 128ull * hkv, 1, 64, 64, 1) ||

@@ -19,14 +19,15 @@
 //            (192-column tiles: c^KV * gamma_kv in bf16 and partial sums of squares; for
 //            the k^R columns the rotary table cos/sin(t base^(-i/32)), angles in fp64, and
 //            the rotated k^R); lambda (sigmoid, fp32 [N, 4H]);
-//   phase 2: (c^Q * gamma_q) W^Q_b (K = 1024, one 192-column query head per tile, scaled
-//            by the row's rsqrt, rotary 64 columns rotated) -> q_sig, q_noise; and
+//   phase 2: (c^Q * gamma_q) W^Q_b (K = 1024, 256-column tiles of the 5H x 192 query
+//            columns, scaled by the row's rsqrt, each head's rotary 64 columns rotated)
+//            -> q_sig, q_noise; and
 //            (c^KV * gamma_kv) W^UK_j, (c^KV * gamma_kv) W^UV_j (K = 512, one KV head per
 //            128-column tile, scaled) -> k = [k_nope | rotated k^R], v.
 // The GEMM: CTA pairs (clusters of two, one CTA per SM) walk 256-row x nt-column tiles
 // (t = pair, + pairs, ...). In each CTA a TMA producer warp streams 64-wide K chunks of
 // its 128 rows of A and its half of the tile's B rows (the weights' rows) through a
-// 6-stage ring; one elected thread of the even CTA issues the pair's tcgen05 MMAs
+// 5- or 6-stage ring; one elected thread of the even CTA issues the pair's tcgen05 MMAs
 // (cta_group::2, M = 256, N = nt, fp32) into one of two TMEM accumulators, so 8
 // epilogue warps per CTA (TMEM lane quarter = warp % 4, column half = warp / 4) drain
 // one tile while the next one is multiplied. Each SM loads 128 + nt/2 operand rows
@@ -66,18 +67,17 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int SSQ = 16;                        // partial sums of squares per row
 }  // namespace pg
 
-// Shared memory of a phase: a 6-stage ring of A chunks and half-B chunks (up to 128
-// rows in phase 1, 96 in phase 2: the up-projections' short MMAs per chunk need
-// about as many loads in flight as the long ones); phase 2 adds three 4 KB output
-// boxes (32 rows x 64 bf16, 128-byte swizzle) per TMEM lane quarter, shared by the
-// quarter's two epilogue warps and read by their TMA stores.
+// Shared memory of a phase: a ring of A chunks and half-B chunks (up to 128 rows; 6
+// stages in phase 1, 5 in phase 2); phase 2 adds four 4 KB output boxes (32 rows x 64
+// bf16, 128-byte swizzle) per TMEM lane quarter, shared by the quarter's two epilogue
+// warps and read by their TMA stores.
 template <int PHASE>
 struct PhaseCfg {
-    static constexpr int STAGES = 6;
-    static constexpr int B_ROWS = PHASE == 1 ? 128 : 96;
+    static constexpr int STAGES = PHASE == 1 ? 6 : 5;
+    static constexpr int B_ROWS = 128;
     static constexpr int STAGE = pg::A_BYTES + B_ROWS * 128;
     static constexpr int OFF_STG = STAGES * STAGE;
-    static constexpr int STG_BYTES = PHASE == 1 ? 0 : 4 * 3 * 4096;
+    static constexpr int STG_BYTES = PHASE == 1 ? 0 : 4 * 4 * 4096;
     static constexpr int OFF_BAR = OFF_STG + STG_BYTES;  // full[S], empty[S], acc_full[2], acc_empty[2], drain
     static constexpr int OFF_MISC = OFF_BAR + 32 * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
@@ -242,21 +242,26 @@ __device__ __forceinline__ void stage_32(uint32_t box, int lane, int c0, const u
     }
 }
 
+// Query up-projection tiles are 256 columns of the row [q_sig heads | q_noise heads]
+// (192 per head): box b (64 columns) of tile n starts at column 256 n + 64 b, which is
+// dims 0, 64 or 128 of one head (a head's rotary dims 128..191 never straddle a box).
+__device__ __forceinline__ bool qup_box_rotary(int n_tile, int b) { return (256 * n_tile + 64 * b) % 192 == 128; }
+
 // Row data an up-projection epilogue reads besides the accumulator, loaded before
-// the accumulator is waited for: the partial sums of squares and, for half 1, the
-// row's rotary cos | sin (query tiles) or rotated k^R (k_nope tiles).
+// the accumulator is waited for: the partial sums of squares and the row's rotary
+// cos | sin (a query half holding a rotary box) or rotated k^R (k_nope tiles, half 1).
 struct Epi2Row {
     float4 ss0, ss1;
     float4 rot[16];
 };
-__device__ __forceinline__ void epi2_prefetch(const PrologueIO &io, int m, bool row_ok, int epi, int hf,
+__device__ __forceinline__ void epi2_prefetch(const PrologueIO &io, int m, bool row_ok, int epi, int hf, int n_tile,
                                               Epi2Row &d) {
     const bool qup = epi == PRO_QUP;
     const size_t row = static_cast<size_t>(row_ok ? m : 0);
     const float4 *p = reinterpret_cast<const float4 *>(io.ssq + row * pg::SSQ);
     d.ss0 = __ldg(p + (qup ? 0 : 2));
     d.ss1 = __ldg(p + (qup ? 1 : 3));
-    if (hf == 1 && qup) {
+    if (qup && (qup_box_rotary(n_tile, 2 * hf) || qup_box_rotary(n_tile, 2 * hf + 1))) {
         const float4 *rot = reinterpret_cast<const float4 *>(io.rot + row * 64);
 #pragma unroll
         for (int i = 0; i < 16; ++i) d.rot[i] = __ldg(rot + i);
@@ -273,39 +278,35 @@ __device__ __forceinline__ float epi2_rsqrt(const Epi2Row &d, bool qup, bool row
     return qup ? rsqrtf((s + (d.ss1.z + d.ss1.w)) * (1.f / 1024.f) + 1e-6f) : rsqrtf(s * (1.f / 512.f) + 1e-6f);
 }
 
-// One query head (tile n = head) into the quarter's output boxes `stg`: half 0 the
-// content dims 0..127 (boxes 0, 1), half 1 the rotary dims 128..191 (pairs i, i+32)
-// rotated (box 2).
-__device__ __forceinline__ void epi_qup(const Epi2Row &d, float r, uint32_t tcol, bool row_ok, int hf, int lane,
-                                        uint32_t stg) {
-    if (hf == 0) {
+// One 256-column query tile into the quarter's output boxes `stg`: half hf stages boxes
+// 2 hf and 2 hf + 1 (those past the last column are skipped); a box holding a head's
+// rotary dims is rotated (pairs i, i + 32) with the row's cos | sin.
+__device__ __forceinline__ void epi_qup(const Epi2Row &d, float r, uint32_t tcol, bool row_ok, int n_tile, int hf,
+                                        int lane, uint32_t stg, int n_cols) {
 #pragma unroll 1
-        for (int ch = 0; ch < 4; ++ch) {
-            uint32_t o[32];
-            tmem_ld32(tcol + ch * 32, o);
-            stage_32(stg + (ch >> 1) * 4096, lane, (ch & 1) * 4, o, r);
-        }
-        return;
-    }
-    uint32_t a[32], b[32];
-    tmem_ld32(tcol + 128, a);
-    tmem_ld32(tcol + 160, b);
-    if (row_ok) {
+    for (int bb = 0; bb < 2; ++bb) {
+        const int b = 2 * hf + bb;
+        if (256 * n_tile + 64 * b >= n_cols) break;
+        uint32_t a[32], c[32];
+        tmem_ld32(tcol + 64 * b, a);
+        tmem_ld32(tcol + 64 * b + 32, c);
+        if (qup_box_rotary(n_tile, b) && row_ok) {
 #pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-            const float4 c4 = d.rot[i4], s4 = d.rot[8 + i4];
-            const float cv[4] = {c4.x, c4.y, c4.z, c4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
+            for (int i4 = 0; i4 < 8; ++i4) {
+                const float4 c4 = d.rot[i4], s4 = d.rot[8 + i4];
+                const float cv[4] = {c4.x, c4.y, c4.z, c4.w}, sv[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int i = 4 * i4 + j;
-                const float x0 = __uint_as_float(a[i]), x1 = __uint_as_float(b[i]);
-                a[i] = __float_as_uint(x0 * cv[j] - x1 * sv[j]);
-                b[i] = __float_as_uint(x0 * sv[j] + x1 * cv[j]);
+                for (int j = 0; j < 4; ++j) {
+                    const int i = 4 * i4 + j;
+                    const float x0 = __uint_as_float(a[i]), x1 = __uint_as_float(c[i]);
+                    a[i] = __float_as_uint(x0 * cv[j] - x1 * sv[j]);
+                    c[i] = __float_as_uint(x0 * sv[j] + x1 * cv[j]);
+                }
             }
         }
+        stage_32(stg + b * 4096, lane, 0, a, r);
+        stage_32(stg + b * 4096, lane, 4, c, r);
     }
-    stage_32(stg + 2 * 4096, lane, 0, a, r);
-    stage_32(stg + 2 * 4096, lane, 4, b, r);
 }
 
 // One KV head j (tile n = j) of k_nope (PRO_KUP) or v (PRO_VUP): half hf stages
@@ -451,7 +452,7 @@ gdla_proj_kernel(const __grid_constant__ ProjGroup G, const __grid_constant__ Pr
     } else {
         // ------------------------------ epilogue ----------------------------------
         const int q = warp & 3, hf = warp >> 2;
-        const uint32_t stg = smem_u32(smem + C::OFF_STG + q * 3 * 4096);  // the quarter's output boxes
+        const uint32_t stg = smem_u32(smem + C::OFF_STG + q * 4 * 4096);  // the quarter's output boxes
         const uint32_t acc_empty_even = mapa_shared(smem_u32(acc_empty), 0);
         int i = 0;
         for (int t = pair; t < G.total_tiles; t += n_pairs, ++i) {
@@ -462,7 +463,7 @@ gdla_proj_kernel(const __grid_constant__ ProjGroup G, const __grid_constant__ Pr
             const bool row_ok = m < G.M;
             const int epi = G.prob[tr.p].epi;
             Epi2Row pre;
-            if constexpr (PHASE == 2) epi2_prefetch(io, m, row_ok, epi, hf, pre);
+            if constexpr (PHASE == 2) epi2_prefetch(io, m, row_ok, epi, hf, tr.n_tile, pre);
             if (!__all_sync(0xffffffffu,
                             mbar_wait_cl(acc_full + buf, use & 1, abort_flag, ERR_SITE_PROLOGUE | 4)))
                 break;
@@ -486,7 +487,8 @@ gdla_proj_kernel(const __grid_constant__ ProjGroup G, const __grid_constant__ Pr
                     break;
                 const bool qup = epi == PRO_QUP;
                 const float r = epi2_rsqrt(pre, qup, row_ok);
-                if (qup) epi_qup(pre, r, tcol, row_ok, hf, lane, stg);
+                const int n_cols = 5 * io.hkv * 192;  // query up-projection columns
+                if (qup) epi_qup(pre, r, tcol, row_ok, tr.n_tile, hf, lane, stg, n_cols);
                 else epi_kvup(pre, r, tcol, epi == PRO_KUP, hf, lane, stg);
                 tc_fence_before();
                 fence_proxy_async_smem();
@@ -496,15 +498,21 @@ gdla_proj_kernel(const __grid_constant__ ProjGroup G, const __grid_constant__ Pr
                     const int row0 = tr.m0 + q * 32;
                     if (row0 < G.M) {  // rows past the last token are clipped by the store
                         const int hq = 4 * io.hkv;
-                        const CUtensorMap *map = qup ? (tr.n_tile < hq ? &G.tm_o[0] : &G.tm_o[1])
-                                                     : (epi == PRO_KUP ? &G.tm_o[2] : &G.tm_o[3]);
-                        const int head = (qup && tr.n_tile >= hq) ? tr.n_tile - hq : tr.n_tile;
-                        // this warp's boxes: query half 0 -> 0, 1; half 1 -> 2; k / v half hf -> hf
-                        // (and k's half 1 -> 2 as well); box b holds dims 64 b .. 64 b + 63
-                        const int b_lo = qup ? (hf ? 2 : 0) : hf;
-                        const int b_hi = qup ? (hf ? 2 : 1) : (epi == PRO_KUP && hf ? 2 : hf);
-                        for (int b = b_lo; b <= b_hi; ++b)
-                            tma_store_3d(map, smem + C::OFF_STG + (q * 3 + b) * 4096, 64 * b, head, row0);
+                        if (qup) {  // boxes 2 hf, 2 hf + 1: columns 256 n + 64 b = head, dims
+                            for (int b = 2 * hf; b < 2 * hf + 2; ++b) {
+                                const int col = 256 * tr.n_tile + 64 * b;
+                                if (col >= n_cols) break;
+                                const int head = col / 192;
+                                tma_store_3d(head < hq ? &G.tm_o[0] : &G.tm_o[1],
+                                             smem + C::OFF_STG + (q * 4 + b) * 4096, col % 192,
+                                             head < hq ? head : head - hq, row0);
+                            }
+                        } else {  // k / v half hf -> box hf (dims 64 hf ..), k's half 1 also box 2 (k^R)
+                            const CUtensorMap *map = epi == PRO_KUP ? &G.tm_o[2] : &G.tm_o[3];
+                            const int b_hi = (epi == PRO_KUP && hf) ? 2 : hf;
+                            for (int b = hf; b <= b_hi; ++b)
+                                tma_store_3d(map, smem + C::OFF_STG + (q * 4 + b) * 4096, 64 * b, tr.n_tile, row0);
+                        }
                         bulk_commit_group();
                     }
                 }
@@ -596,7 +604,7 @@ cudaError_t launch_prologue(const PrologueLaunch &L, const ProloguePlan &plan, i
     g2.tm_o[1] = L.tm_qn_o;
     g2.tm_o[2] = L.tm_k_o;
     g2.tm_o[3] = L.tm_v_o;
-    add_problem(g2, L.tm_cqn, L.tm_wqb, PRO_QUP, 192, 1024, 5 * hkv);
+    add_problem(g2, L.tm_cqn, L.tm_wqb, PRO_QUP, 256, 1024, (5 * hkv * 192 + 255) / 256);
     add_problem(g2, L.tm_ckvn, L.tm_wuk, PRO_KUP, 128, 512, hkv);
     add_problem(g2, L.tm_ckvn, L.tm_wuv, PRO_VUP, 128, 512, hkv);
     return launch_group<2>(g2, L.io, plan, stream);

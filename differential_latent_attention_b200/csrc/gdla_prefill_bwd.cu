@@ -76,11 +76,16 @@ constexpr uint32_t QD_TX = (3 + 2) * 4 * QBOX_TX;  // Q and dH tiles of one item
 // row warps turn this tile's into dS (written over its S).
 constexpr uint32_t DQ_COL = 0, S_COL0 = 192, DP_COL0 = 256, BUF_COLS = 128;
 constexpr uint32_t TMEM_COLS = 512;
+// 8 row warps: two per TMEM lane quarter (warp % 4), each taking one half (warp / 4)
+// of a key tile's 32 + 32 columns; producer warp 8, MMA warp 9.
+constexpr int ROW_WARPS = 8;
+constexpr int NUM_THREADS = 32 * ROW_WARPS + 64;
+constexpr int PRODUCER_WARP = ROW_WARPS, MMA_WARP = ROW_WARPS + 1;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace pbq
 
 template <class Plan>
-__global__ void __launch_bounds__(pb::NUM_THREADS, 1)
+__global__ void __launch_bounds__(pbq::NUM_THREADS, 1)
 gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_qn,
                    const __grid_constant__ CUtensorMap tm_dhs, const __grid_constant__ CUtensorMap tm_dhn,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -95,7 +100,7 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
     uint64_t *kv_full = bars + 2;   // [stage]
     uint64_t *kv_empty = bars + 4;  // [stage]
     uint64_t *s_full = bars + 6;    // [buffer]: S and dP of a key tile in TMEM
-    uint64_t *ds_full = bars + 8;   // [buffer]: its dS in TMEM (128 arrivals)
+    uint64_t *ds_full = bars + 8;   // [buffer]: its dS in TMEM (one arrival per row-warp thread)
     uint64_t *dq_final = bars + 10; // one phase per item: its last dQ product is done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
@@ -129,13 +134,13 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(s_full + b, 1);
-            mbar_init(ds_full + b, 128);
+            mbar_init(ds_full + b, 32 * ROW_WARPS);
         }
         mbar_init(dq_final, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == PRODUCER_WARP) {
+    if (warp == pbq::PRODUCER_WARP) {
         // rows 32w+30, 32w+31 of the Q and dH tiles are never loaded: zero them once
         for (int c = 0; c < 5; ++c)
             for (int i = lane; i < 4 * 2 * 8; i += 32) {
@@ -144,7 +149,7 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
             }
         fence_proxy_async_smem();
     }
-    if (warp == MMA_WARP) {
+    if (warp == pbq::MMA_WARP) {
         tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
@@ -153,7 +158,7 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == PRODUCER_WARP) {
+    if (warp == pbq::PRODUCER_WARP) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
             int kv = 0, issued = 0, n_item = 0;
@@ -200,7 +205,7 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
                 mbar_wait_cycles(q_full, (n_item & 1) ^ 1, 1ll << 22);
             }
         }
-    } else if (warp == MMA_WARP) {
+    } else if (warp == pbq::MMA_WARP) {
         // ------------------------------ MMA issuer --------------------------------
         // Order: S(0), dP(0); then per key tile k: S(k+1), dP(k+1) into the other
         // buffer, (dS(k) from the row warps), dQ(k). S(k+2) overwrites dS(k) only
@@ -257,10 +262,12 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
                 tc_fence_after();
                 const uint32_t sbase = st * STAGE;
                 const uint32_t buf = (sk & 1) * BUF_COLS;
+                // packed dS of keys 32 h .. 32 h + 31 sits in columns 32 h .. 32 h + 15 of the buffer
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    umma_ts_leader(tmem + DQ_COL, tmem + S_COL0 + buf + kk * 8, kmn_desc0 + ((sbase + kk * 2048) >> 4),
-                                   idesc_q, (k > 0 || kk > 0) ? 1u : 0u, leader);
+                    umma_ts_leader(tmem + DQ_COL, tmem + S_COL0 + buf + (kk >> 1) * 32 + (kk & 1) * 8,
+                                   kmn_desc0 + ((sbase + kk * 2048) >> 4), idesc_q, (k > 0 || kk > 0) ? 1u : 0u,
+                                   leader);
                 umma_commit_leader(kv_empty + st, leader);
                 if (k == it.n_tiles - 1) umma_commit_leader(dq_final, leader);
             }
@@ -269,11 +276,12 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
         }
     } else {
         // ------------------------------ row warps ---------------------------------
+        const int qw = warp & 3, half = warp >> 2;  // TMEM lane quarter, key-column half
         const bool is_sig = lane < 24;
-        const int tau = 6 * warp + pb::quarter_token(lane);
+        const int tau = 6 * qw + pb::quarter_token(lane);
         const int head = pb::quarter_head(lane);
         const bool pad_row = lane >= 30;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(qw * 32) << 16);
         int step = 0, n_item = 0;
         bool ok = true;
         for (int w = snake_item(0); ok && w < n_work; w = snake_item(n_item + 1), ++n_item) {
@@ -293,14 +301,15 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
                     break;
                 }
                 tc_fence_after();
-                const uint32_t s_addr = lane_base + S_COL0 + b * BUF_COLS;
-                uint32_t sr[64], dr[64];
-                tmem_ld64(s_addr, sr);
-                tmem_ld64(lane_base + DP_COL0 + b * BUF_COLS, dr);
-                const int u0 = it.kv_lo + k * BN;
-                uint32_t pk[32];
+                // this half's 32 keys: S and dP columns 32 half ..; packed dS over its first 16 S columns
+                const uint32_t s_addr = lane_base + S_COL0 + b * BUF_COLS + 32 * half;
+                uint32_t sr[32], dr[32];
+                tmem_ld32(s_addr, sr);
+                tmem_ld32(lane_base + DP_COL0 + b * BUF_COLS + 32 * half, dr);
+                const int u0 = it.kv_lo + k * BN + 32 * half;
+                uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < 16; ++i) {
                     float ds2[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
@@ -311,7 +320,7 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
                     }
                     pk[i] = pack_bf16x2(ds2[0], ds2[1]);
                 }
-                tmem_st32(s_addr, pk);
+                tmem_st16(s_addr, pk);
                 tc_fence_before();
                 mbar_arrive(ds_full + b);
             }
@@ -321,7 +330,7 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
             __nv_bfloat16 *dst = is_sig ? dq_sig + ((static_cast<size_t>(it.s0 + t) * hs + 4 * it.group + head) * DQK)
                                         : dq_noise + srow * DQK;
 #pragma unroll 1
-            for (int ch = 0; ch < DQK / 32; ++ch) {
+            for (int ch = 3 * half; ch < 3 * half + 3; ++ch) {  // this half's 96 of dQ's 192 columns
                 uint32_t o[32];
                 tmem_ld32(lane_base + DQ_COL + ch * 32, o);
                 if (row_ok) {
@@ -341,7 +350,7 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == MMA_WARP) {
+    if (warp == pbq::MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
@@ -701,7 +710,7 @@ static cudaError_t launch_dq_sized(const BwdLaunch &L, const Plan &plan, cudaStr
     }
     const long long work = static_cast<long long>(plan.n_items) * plan.hkv;
     const unsigned grid = static_cast<unsigned>(work < num_sms ? work : num_sms);
-    gdla_bwd_dq_kernel<Plan><<<grid, pb::NUM_THREADS, pbq::SMEM_BYTES, stream>>>(
+    gdla_bwd_dq_kernel<Plan><<<grid, pbq::NUM_THREADS, pbq::SMEM_BYTES, stream>>>(
         L.tm_qs, L.tm_qn, L.tm_dhs, L.tm_dhn, L.tm_k64, L.tm_v64, L.stats, L.dq_sig, L.dq_noise, plan);
     return cudaPeekAtLastError();
 }

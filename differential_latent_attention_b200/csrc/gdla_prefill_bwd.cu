@@ -385,11 +385,16 @@ constexpr uint32_t STEP_TX = (3 + 2) * 2 * QBOX_TX + STATS_BYTES;
 // loaded it): step s+1's products run while the key warps work on step s.
 constexpr uint32_t DK_COL = 0, DV_COL = 192, ST_COL0 = 320, DPT_COL = 448;
 constexpr uint32_t TMEM_COLS = 512;
+// 8 key warps: two per TMEM lane quarter (warp % 4), each taking one half (warp / 4)
+// of a step's 64 rows; producer warp 8, MMA warp 9.
+constexpr int KEY_WARPS = 8;
+constexpr int NUM_THREADS = 32 * KEY_WARPS + 64;
+constexpr int PRODUCER_WARP = KEY_WARPS, MMA_WARP = KEY_WARPS + 1;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 }  // namespace pbk
 
 template <class Plan>
-__global__ void __launch_bounds__(pb::NUM_THREADS, 1)
+__global__ void __launch_bounds__(pbk::NUM_THREADS, 1)
 gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_qn,
                     const __grid_constant__ CUtensorMap tm_dhs, const __grid_constant__ CUtensorMap tm_dhn,
                     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -404,8 +409,8 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
     uint64_t *st_full = bars + 2;    // [stage]: Q, dH halves and row statistics of a step
     uint64_t *st_empty = bars + 5;   // [stage]
     uint64_t *s_full = bars + 8;     // [buffer]: S^T and dP^T of a step in TMEM
-    uint64_t *dpt_free = bars + 10;  // one phase per step: its dP^T has been loaded (128 arrivals)
-    uint64_t *pds_full = bars + 11;  // [buffer]: P^T and dS^T in TMEM (128 arrivals)
+    uint64_t *dpt_free = bars + 10;  // one phase per step: its dP^T has been loaded (every key-warp thread)
+    uint64_t *pds_full = bars + 11;  // [buffer]: P^T and dS^T in TMEM (every key-warp thread)
     uint64_t *dkv_final = bars + 13; // one phase per item
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
@@ -441,14 +446,14 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(s_full + b, 1);
-            mbar_init(pds_full + b, 128);
+            mbar_init(pds_full + b, 32 * KEY_WARPS);
         }
-        mbar_init(dpt_free, 128);
+        mbar_init(dpt_free, 32 * KEY_WARPS);
         mbar_init(dkv_final, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == PRODUCER_WARP) {
+    if (warp == pbk::PRODUCER_WARP) {
         // rows 32q+30, 32q+31 of every stage's Q and dH halves are never loaded: zero them once
         for (int st = 0; st < STAGES; ++st)
             for (int c = 0; c < 5; ++c)
@@ -459,7 +464,7 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                 }
         fence_proxy_async_smem();
     }
-    if (warp == MMA_WARP) {
+    if (warp == pbk::MMA_WARP) {
         tmem_alloc(tmem_slot, TMEM_COLS);
         tmem_relinquish();
     }
@@ -468,7 +473,7 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == PRODUCER_WARP) {
+    if (warp == pbk::PRODUCER_WARP) {
         // ------------------------------ TMA producer ------------------------------
         if (lane == 0) {
             int g = 0, issued = 0, n_item = 0;
@@ -515,7 +520,7 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                 mbar_wait_cycles(kv_full, (n_item & 1) ^ 1, 1ll << 22);
             }
         }
-    } else if (warp == MMA_WARP) {
+    } else if (warp == pbk::MMA_WARP) {
         // ------------------------------ MMA issuer --------------------------------
         const uint32_t leader = elect_one_sync();
         constexpr uint32_t idesc_s = idesc_bf16_f32(128, 64, false, false);
@@ -581,13 +586,16 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                 tc_fence_after();
                 const uint32_t sbase = st * STAGE;
                 const uint32_t pcol = ST_COL0 + (gs & 1) * 64;
+                // rows 32 h .. 32 h + 31 of the step: packed P^T in columns 32 h .. 32 h + 15,
+                // packed dS^T in 32 h + 16 .. 32 h + 31
 #pragma unroll
                 for (int kk = 0; kk < 64 / 16; ++kk) {
                     const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                    umma_ts_leader(tmem + DV_COL, tmem + pcol + kk * 8,
-                                   stmn_desc0 + ((sbase + QH_BYTES + kk * 2048) >> 4), idesc_v, acc, leader);
-                    umma_ts_leader(tmem + DK_COL, tmem + pcol + 32 + kk * 8, stmn_desc0 + ((sbase + kk * 2048) >> 4),
-                                   idesc_k, acc, leader);
+                    const uint32_t pc = pcol + (kk >> 1) * 32 + (kk & 1) * 8;
+                    umma_ts_leader(tmem + DV_COL, tmem + pc, stmn_desc0 + ((sbase + QH_BYTES + kk * 2048) >> 4),
+                                   idesc_v, acc, leader);
+                    umma_ts_leader(tmem + DK_COL, tmem + pc + 16, stmn_desc0 + ((sbase + kk * 2048) >> 4), idesc_k,
+                                   acc, leader);
                 }
                 umma_commit_leader(st_empty + st, leader);
             }
@@ -598,8 +606,9 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         }
     } else {
         // ------------------------------ key warps ---------------------------------
-        const int kl = warp * 32 + lane;  // key of the tile = TMEM lane
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const int qw = warp & 3, half = warp >> 2;  // TMEM lane quarter, half of the step's rows
+        const int kl = qw * 32 + lane;              // key of the tile = TMEM lane
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(qw * 32) << 16);
         int g = 0, n_item = 0;
         bool ok = true;
         for (int w = snake_item(0); ok && w < n_work; w = snake_item(n_item + 1), ++n_item) {
@@ -613,23 +622,24 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                     break;
                 }
                 tc_fence_after();
-                const uint32_t s_addr = lane_base + ST_COL0 + b * 64;
-                uint32_t sr[64], dr[64];
-                tmem_ld64(s_addr, sr);
-                tmem_ld64(lane_base + DPT_COL, dr);
+                // this half's 32 rows: S^T and dP^T columns 32 half ..; packed P^T and dS^T over them
+                const uint32_t s_addr = lane_base + ST_COL0 + b * 64 + 32 * half;
+                uint32_t sr[32], dr[32];
+                tmem_ld32(s_addr, sr);
+                tmem_ld32(lane_base + DPT_COL + 32 * half, dr);
                 tc_fence_before();
                 mbar_arrive(dpt_free);  // dP^T is in registers: the next step's may overwrite it
                 const float *stat = reinterpret_cast<const float *>(smem + OFF_ST + st * STAGE + QH_BYTES + DHH_BYTES);
                 const int th = it.u0 + s * HT;  // first token of the step
-                uint32_t pk[32], dk2[32];
+                uint32_t pk[16], dk2[16];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < 16; ++i) {
                     float pv[2], dv2[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int r = 2 * i + e;             // row of the 64-row half
-                        const int within = r & 31;
-                        const int tok = 6 * (r >> 5) + pb::quarter_token(within);
+                        const int r = 2 * i + e;             // row of this 32-row block
+                        const int within = r;
+                        const int tok = 6 * half + pb::quarter_token(within);
                         const int head = pb::quarter_head(within);
                         const int t = th + tok;
                         const bool vis = within < 30 && key_ok && t < it.L && u <= t && (window <= 0 || u > t - window);
@@ -642,8 +652,8 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                     pk[i] = pack_bf16x2(pv[0], pv[1]);
                     dk2[i] = pack_bf16x2(dv2[0], dv2[1]);
                 }
-                tmem_st32(s_addr, pk);
-                tmem_st32(s_addr + 32, dk2);
+                tmem_st16(s_addr, pk);
+                tmem_st16(s_addr + 16, dk2);
                 tc_fence_before();
                 mbar_arrive(pds_full + b);
             }
@@ -651,8 +661,9 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
             if (!__all_sync(0xffffffffu, mbar_wait(dkv_final, n_item & 1, abort_flag, ERR_SITE_BWD | 17))) break;
             tc_fence_after();
             const size_t krow = static_cast<size_t>(it.s0 + u) * hkv + it.group;
+            // dK's 6 and dV's 4 32-column chunks: half 0 takes dK 0..4, half 1 dK 5 and dV 0..3
 #pragma unroll 1
-            for (int ch = 0; ch < DQK / 32; ++ch) {
+            for (int ch = 5 * half; ch < (half ? DQK / 32 : 5); ++ch) {
                 uint32_t o[32];
                 tmem_ld32(lane_base + DK_COL + ch * 32, o);
                 if (key_ok) {
@@ -666,7 +677,7 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                 }
             }
 #pragma unroll 1
-            for (int ch = 0; ch < DV / 32; ++ch) {
+            for (int ch = 0; ch < (half ? DV / 32 : 0); ++ch) {
                 uint32_t o[32];
                 tmem_ld32(lane_base + DV_COL + ch * 32, o);
                 if (key_ok) {
@@ -684,7 +695,7 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == MMA_WARP) {
+    if (warp == pbk::MMA_WARP) {
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
@@ -732,7 +743,7 @@ static cudaError_t launch_dkv_sized(const BwdLaunch &L, const Plan &plan, cudaSt
     }
     const long long work = static_cast<long long>(plan.n_items) * plan.hkv;
     const unsigned grid = static_cast<unsigned>(work < num_sms ? work : num_sms);
-    gdla_bwd_dkv_kernel<Plan><<<grid, pb::NUM_THREADS, pbk::SMEM_BYTES, stream>>>(
+    gdla_bwd_dkv_kernel<Plan><<<grid, pbk::NUM_THREADS, pbk::SMEM_BYTES, stream>>>(
         L.tm_qs, L.tm_qn, L.tm_dhs, L.tm_dhn, L.tm_k128, L.tm_v128, L.tm_stats, L.dk, L.dv, plan);
     return cudaPeekAtLastError();
 }

@@ -51,13 +51,33 @@ __host__ __device__ constexpr int quarter_token(int within) { return within < 24
 __host__ __device__ constexpr int quarter_head(int within) { return within < 24 ? (within & 3) : 4; }
 }  // namespace pb
 
+// Two 32-column TMEM loads (any two column addresses of this warp's lanes) with one wait.
+__device__ __forceinline__ void tmem_ld32x2(uint32_t a0, uint32_t a1, uint32_t (&r0)[32], uint32_t (&r1)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%65];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r0[0]), "=r"(r0[1]), "=r"(r0[2]), "=r"(r0[3]), "=r"(r0[4]), "=r"(r0[5]), "=r"(r0[6]), "=r"(r0[7]), "=r"(r0[8]), "=r"(r0[9]), "=r"(r0[10]), "=r"(r0[11]), "=r"(r0[12]), "=r"(r0[13]), "=r"(r0[14]), "=r"(r0[15]), "=r"(r0[16]), "=r"(r0[17]), "=r"(r0[18]), "=r"(r0[19]), "=r"(r0[20]), "=r"(r0[21]), "=r"(r0[22]), "=r"(r0[23]), "=r"(r0[24]), "=r"(r0[25]), "=r"(r0[26]), "=r"(r0[27]), "=r"(r0[28]), "=r"(r0[29]), "=r"(r0[30]), "=r"(r0[31]), "=r"(r1[0]), "=r"(r1[1]), "=r"(r1[2]), "=r"(r1[3]), "=r"(r1[4]), "=r"(r1[5]), "=r"(r1[6]), "=r"(r1[7]), "=r"(r1[8]), "=r"(r1[9]), "=r"(r1[10]), "=r"(r1[11]), "=r"(r1[12]), "=r"(r1[13]), "=r"(r1[14]), "=r"(r1[15]), "=r"(r1[16]), "=r"(r1[17]), "=r"(r1[18]), "=r"(r1[19]), "=r"(r1[20]), "=r"(r1[21]), "=r"(r1[22]), "=r"(r1[23]), "=r"(r1[24]), "=r"(r1[25]), "=r"(r1[26]), "=r"(r1[27]), "=r"(r1[28]), "=r"(r1[29]), "=r"(r1[30]), "=r"(r1[31])
+        : "r"(a0), "r"(a1)
+        : "memory");
+}
+// Two 16-column TMEM stores with one wait.
+__device__ __forceinline__ void tmem_st16x2(uint32_t a0, const uint32_t (&r0)[16], uint32_t a1,
+                                            const uint32_t (&r1)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17};\n\t"
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%1], {%18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33};\n\t"
+        "tcgen05.wait::st.sync.aligned;" ::"r"(a0), "r"(a1), "r"(r0[0]), "r"(r0[1]), "r"(r0[2]), "r"(r0[3]), "r"(r0[4]), "r"(r0[5]), "r"(r0[6]), "r"(r0[7]), "r"(r0[8]), "r"(r0[9]), "r"(r0[10]), "r"(r0[11]), "r"(r0[12]), "r"(r0[13]), "r"(r0[14]), "r"(r0[15]), "r"(r1[0]), "r"(r1[1]), "r"(r1[2]), "r"(r1[3]), "r"(r1[4]), "r"(r1[5]), "r"(r1[6]), "r"(r1[7]), "r"(r1[8]), "r"(r1[9]), "r"(r1[10]), "r"(r1[11]), "r"(r1[12]), "r"(r1[13]), "r"(r1[14]), "r"(r1[15])
+        : "memory");
+}
+
 // ------------------------------------------------------------------------------
 // dQ
 // ------------------------------------------------------------------------------
 namespace pbq {
 using namespace pb;
 constexpr int BN = 64;                     // keys per tile
-constexpr int STAGES = 2;
+constexpr int STAGES = 3;
 constexpr int Q_CHUNK = 128 * 128;         // 128 rows x 64 dims
 constexpr int Q_BYTES = 3 * Q_CHUNK;       // 48 KB
 constexpr int DH_BYTES = 2 * Q_CHUNK;      // 32 KB
@@ -98,10 +118,10 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
     uint64_t *q_full = bars + 0;    // one phase per item: Q and dH tiles landed
     uint64_t *q_empty = bars + 1;   // one phase per item: its last S / dP products are done
     uint64_t *kv_full = bars + 2;   // [stage]
-    uint64_t *kv_empty = bars + 4;  // [stage]
-    uint64_t *s_full = bars + 6;    // [buffer]: S and dP of a key tile in TMEM
-    uint64_t *ds_full = bars + 8;   // [buffer]: its dS in TMEM (one arrival per row-warp thread)
-    uint64_t *dq_final = bars + 10; // one phase per item: its last dQ product is done
+    uint64_t *kv_empty = bars + 5;  // [stage]
+    uint64_t *s_full = bars + 8;    // [buffer]: S and dP of a key tile in TMEM
+    uint64_t *ds_full = bars + 10;  // [buffer]: its dS in TMEM (one arrival per row-warp thread)
+    uint64_t *dq_final = bars + 12; // one phase per item: its last dQ product is done
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
 
@@ -304,8 +324,7 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
                 // this half's 32 keys: S and dP columns 32 half ..; packed dS over its first 16 S columns
                 const uint32_t s_addr = lane_base + S_COL0 + b * BUF_COLS + 32 * half;
                 uint32_t sr[32], dr[32];
-                tmem_ld32(s_addr, sr);
-                tmem_ld32(lane_base + DP_COL0 + b * BUF_COLS + 32 * half, dr);
+                tmem_ld32x2(s_addr, lane_base + DP_COL0 + b * BUF_COLS + 32 * half, sr, dr);
                 const int u0 = it.kv_lo + k * BN + 32 * half;
                 uint32_t pk[16];
 #pragma unroll
@@ -625,8 +644,7 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                 // this half's 32 rows: S^T and dP^T columns 32 half ..; packed P^T and dS^T over them
                 const uint32_t s_addr = lane_base + ST_COL0 + b * 64 + 32 * half;
                 uint32_t sr[32], dr[32];
-                tmem_ld32(s_addr, sr);
-                tmem_ld32(lane_base + DPT_COL + 32 * half, dr);
+                tmem_ld32x2(s_addr, lane_base + DPT_COL + 32 * half, sr, dr);
                 tc_fence_before();
                 mbar_arrive(dpt_free);  // dP^T is in registers: the next step's may overwrite it
                 const float *stat = reinterpret_cast<const float *>(smem + OFF_ST + st * STAGE + QH_BYTES + DHH_BYTES);
@@ -652,8 +670,7 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                     pk[i] = pack_bf16x2(pv[0], pv[1]);
                     dk2[i] = pack_bf16x2(dv2[0], dv2[1]);
                 }
-                tmem_st16(s_addr, pk);
-                tmem_st16(s_addr + 16, dk2);
+                tmem_st16x2(s_addr, pk, s_addr + 16, dk2);
                 tc_fence_before();
                 mbar_arrive(pds_full + b);
             }

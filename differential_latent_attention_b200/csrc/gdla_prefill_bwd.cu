@@ -326,16 +326,21 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
                 uint32_t sr[32], dr[32];
                 tmem_ld32x2(s_addr, lane_base + DP_COL0 + b * BUF_COLS + 32 * half, sr, dr);
                 const int u0 = it.kv_lo + k * BN + 32 * half;
+                // bit c: key u0 + c is visible to this row (c <= t - u0, and c > t - window - u0)
+                const int hi = min(31, t - u0);
+                const int lo = (window > 0) ? max(0, t - window - u0 + 1) : 0;
+                const uint32_t vm = (!row_ok || hi < lo)
+                                        ? 0u
+                                        : ((hi == 31 ? 0xFFFFFFFFu : ((1u << (hi + 1)) - 1u)) & ~((1u << lo) - 1u));
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     float ds2[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int u = u0 + 2 * i + e;
-                        const bool vis = row_ok && u <= t && (window <= 0 || u > t - window);
-                        const float p = fast_exp2(__uint_as_float(sr[2 * i + e]) * kScoreLog2 - lse2);
-                        ds2[e] = vis ? p * (__uint_as_float(dr[2 * i + e]) - drow) : 0.f;
+                        const int c = 2 * i + e;
+                        const float p = fast_exp2(fmaf(__uint_as_float(sr[c]), kScoreLog2, -lse2));
+                        ds2[e] = ((vm >> c) & 1u) ? p * (__uint_as_float(dr[c]) - drow) : 0.f;
                     }
                     pk[i] = pack_bf16x2(ds2[0], ds2[1]);
                 }
@@ -647,29 +652,55 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                 tmem_ld32x2(s_addr, lane_base + DPT_COL + 32 * half, sr, dr);
                 tc_fence_before();
                 mbar_arrive(dpt_free);  // dP^T is in registers: the next step's may overwrite it
-                const float *stat = reinterpret_cast<const float *>(smem + OFF_ST + st * STAGE + QH_BYTES + DHH_BYTES);
-                const int th = it.u0 + s * HT;  // first token of the step
-                uint32_t pk[16], dk2[16];
+                // this half's 6 tokens: their row statistics, and which of them see this key
+                const float *stat = reinterpret_cast<const float *>(smem + OFF_ST + st * STAGE + QH_BYTES + DHH_BYTES) +
+                                    6 * half * kBwdStats;
+                const int th = it.u0 + s * HT + 6 * half;  // first token of this half
+                uint32_t tm = 0;                           // bit j: token th + j sees key u
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float pv[2], dv2[2];
+                for (int j = 0; j < 6; ++j) {
+                    const int t = th + j;
+                    tm |= (key_ok && u <= t && t < it.L && (window <= 0 || t < u + window)) ? (1u << j) : 0u;
+                }
+                // rows 4j..4j+3 are token j's signal heads, 24 + j its noise head, 30 and 31 padding
+                uint32_t pk[16], dk2[16];
+                float l4[6], d4[6];
+#pragma unroll
+                for (int j = 0; j < 6; ++j) {
+                    const float4 L = *reinterpret_cast<const float4 *>(stat + j * kBwdStats);
+                    const float4 D = *reinterpret_cast<const float4 *>(stat + j * kBwdStats + 8);
+                    l4[j] = stat[j * kBwdStats + 4];
+                    d4[j] = stat[j * kBwdStats + 12];
+                    const bool vj = (tm >> j) & 1u;
+                    const float lv[4] = {L.x, L.y, L.z, L.w}, dv[4] = {D.x, D.y, D.z, D.w};
+                    float pv[4], ds[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const float p = fast_exp2(fmaf(__uint_as_float(sr[4 * j + h]), kScoreLog2, -lv[h]));
+                        pv[h] = vj ? p : 0.f;
+                        ds[h] = vj ? p * (__uint_as_float(dr[4 * j + h]) - dv[h]) : 0.f;
+                    }
+                    pk[2 * j] = pack_bf16x2(pv[0], pv[1]);
+                    pk[2 * j + 1] = pack_bf16x2(pv[2], pv[3]);
+                    dk2[2 * j] = pack_bf16x2(ds[0], ds[1]);
+                    dk2[2 * j + 1] = pack_bf16x2(ds[2], ds[3]);
+                }
+#pragma unroll
+                for (int m = 0; m < 3; ++m) {
+                    float pv[2], ds[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int r = 2 * i + e;             // row of this 32-row block
-                        const int within = r;
-                        const int tok = 6 * half + pb::quarter_token(within);
-                        const int head = pb::quarter_head(within);
-                        const int t = th + tok;
-                        const bool vis = within < 30 && key_ok && t < it.L && u <= t && (window <= 0 || u > t - window);
-                        const float lse2 = stat[tok * kBwdStats + head];
-                        const float drow = stat[tok * kBwdStats + 8 + head];
-                        const float p = fast_exp2(__uint_as_float(sr[r]) * kScoreLog2 - lse2);
-                        pv[e] = vis ? p : 0.f;
-                        dv2[e] = vis ? p * (__uint_as_float(dr[r]) - drow) : 0.f;
+                        const int j = 2 * m + e;
+                        const bool vj = (tm >> j) & 1u;
+                        const float p = fast_exp2(fmaf(__uint_as_float(sr[24 + j]), kScoreLog2, -l4[j]));
+                        pv[e] = vj ? p : 0.f;
+                        ds[e] = vj ? p * (__uint_as_float(dr[24 + j]) - d4[j]) : 0.f;
                     }
-                    pk[i] = pack_bf16x2(pv[0], pv[1]);
-                    dk2[i] = pack_bf16x2(dv2[0], dv2[1]);
+                    pk[12 + m] = pack_bf16x2(pv[0], pv[1]);
+                    dk2[12 + m] = pack_bf16x2(ds[0], ds[1]);
                 }
+                pk[15] = 0u;
+                dk2[15] = 0u;
                 tmem_st16x2(s_addr, pk, s_addr + 16, dk2);
                 tc_fence_before();
                 mbar_arrive(pds_full + b);

@@ -380,6 +380,10 @@ gdla_status_t gdla_attn_bwd(const void *q_sig, const void *q_noise, const void *
     if (!make_map(&B.tm_qs, q_sig, 192, 4 * hkv, N, 64, 4, TQ) || !make_map(&B.tm_qn, q_noise, 192, hkv, N, 64, 1, TQ) ||
         !make_map(&B.tm_dhs, dh_sig, 128, 4 * hkv, N, 64, 4, TQ) ||
         !make_map(&B.tm_dhn, dh_noise, 128, hkv, N, 64, 1, TQ) ||
+        !make_map(&B.tm_qs12, q_sig, 192, 4 * hkv, N, 64, 4, kBwdStepTokens) ||
+        !make_map(&B.tm_qn12, q_noise, 192, hkv, N, 64, 1, kBwdStepTokens) ||
+        !make_map(&B.tm_dhs12, dh_sig, 128, 4 * hkv, N, 64, 4, kBwdStepTokens) ||
+        !make_map(&B.tm_dhn12, dh_noise, 128, hkv, N, 64, 1, kBwdStepTokens) ||
         !make_map(&B.tm_k64, k, 192, hkv, N, 64, 1, kBwdQKeyTile) ||
         !make_map(&B.tm_v64, v, 128, hkv, N, 64, 1, kBwdQKeyTile) ||
         !make_map(&B.tm_k128, k, 192, hkv, N, 64, 1, kBwdKeyTile) ||

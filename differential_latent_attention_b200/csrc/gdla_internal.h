@@ -87,6 +87,8 @@ constexpr int kBwdStepTokens = 12;
 struct BwdLaunch {
     CUtensorMap tm_qs, tm_qn;       // Q boxes of 6 tokens (as the forward)
     CUtensorMap tm_dhs, tm_dhn;     // dH boxes of 6 tokens
+    CUtensorMap tm_qs12, tm_qn12;   // Q boxes of 12 tokens (dkv steps)
+    CUtensorMap tm_dhs12, tm_dhn12; // dH boxes of 12 tokens
     CUtensorMap tm_k64, tm_v64;     // 64-key K / V boxes (dq)
     CUtensorMap tm_k128, tm_v128;   // 128-key K / V boxes (dkv)
     CUtensorMap tm_stats;           // row statistics, 12 tokens of one group

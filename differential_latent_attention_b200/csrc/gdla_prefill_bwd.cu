@@ -403,7 +403,10 @@ constexpr int OFF_BAR = OFF_ST + STAGES * STAGE;
 constexpr int OFF_MISC = OFF_BAR + 16 * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 64 + 1024;
 constexpr uint32_t KV_TX = K_BYTES + V_BYTES;
-constexpr uint32_t STEP_TX = (3 + 2) * 2 * QBOX_TX + STATS_BYTES;
+// A step's 64 rows: signal rows 4 j + h (token j < 12, head h < 4), noise rows 48 + j,
+// padding rows 60..63; one 12-token box per 64-dim chunk and head kind.
+constexpr int STEP_SIG_ROWS = 4 * HT, STEP_NOISE_ROW0 = 4 * HT, STEP_PAD_ROW0 = 5 * HT;
+constexpr uint32_t STEP_TX = (3 + 2) * STEP_PAD_ROW0 * 128 + STATS_BYTES;
 // dK, dV, two S^T buffers (each later holding P^T in its first 32 columns and
 // dS^T in the next 32), one dP^T buffer (free again once the key warps have
 // loaded it): step s+1's products run while the key warps work on step s.
@@ -478,14 +481,12 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
         fence_mbar_init();
     }
     if (warp == pbk::PRODUCER_WARP) {
-        // rows 32q+30, 32q+31 of every stage's Q and dH halves are never loaded: zero them once
+        // rows 60..63 of every stage's Q and dH chunks are never loaded: zero them once
         for (int st = 0; st < STAGES; ++st)
             for (int c = 0; c < 5; ++c)
-                for (int i = lane; i < 2 * 2 * 8; i += 32) {
-                    const int row = 32 * (i >> 4) + 30 + ((i >> 3) & 1);
-                    reinterpret_cast<uint4 *>(smem + OFF_ST + st * STAGE + c * H_CHUNK + row * 128)[i & 7] =
-                        make_uint4(0, 0, 0, 0);
-                }
+                for (int i = lane; i < (64 - STEP_PAD_ROW0) * 8; i += 32)
+                    reinterpret_cast<uint4 *>(smem + OFF_ST + st * STAGE + c * H_CHUNK +
+                                              (STEP_PAD_ROW0 + (i >> 3)) * 128)[i & 7] = make_uint4(0, 0, 0, 0);
         fence_proxy_async_smem();
     }
     if (warp == pbk::MMA_WARP) {
@@ -522,17 +523,15 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                     mbar_arrive_expect_tx(st_full + st, STEP_TX);
                     uint8_t *sb = smem + OFF_ST + st * STAGE;
                     const int th = it.s0 + it.u0 + s * HT;
-                    for (int q = 0; q < 2; ++q) {
-                        for (int c = 0; c < 3; ++c) {
-                            uint8_t *dst = sb + c * H_CHUNK + 32 * q * 128;
-                            tma_load_3d(dst, &tm_qs, st_full + st, c * 64, 4 * it.group, th + 6 * q);
-                            tma_load_3d(dst + 24 * 128, &tm_qn, st_full + st, c * 64, it.group, th + 6 * q);
-                        }
-                        for (int c = 0; c < 2; ++c) {
-                            uint8_t *dst = sb + QH_BYTES + c * H_CHUNK + 32 * q * 128;
-                            tma_load_3d(dst, &tm_dhs, st_full + st, c * 64, 4 * it.group, th + 6 * q);
-                            tma_load_3d(dst + 24 * 128, &tm_dhn, st_full + st, c * 64, it.group, th + 6 * q);
-                        }
+                    for (int c = 0; c < 3; ++c) {
+                        uint8_t *dst = sb + c * H_CHUNK;
+                        tma_load_3d(dst, &tm_qs, st_full + st, c * 64, 4 * it.group, th);
+                        tma_load_3d(dst + STEP_NOISE_ROW0 * 128, &tm_qn, st_full + st, c * 64, it.group, th);
+                    }
+                    for (int c = 0; c < 2; ++c) {
+                        uint8_t *dst = sb + QH_BYTES + c * H_CHUNK;
+                        tma_load_3d(dst, &tm_dhs, st_full + st, c * 64, 4 * it.group, th);
+                        tma_load_3d(dst + STEP_NOISE_ROW0 * 128, &tm_dhn, st_full + st, c * 64, it.group, th);
                     }
                     tma_load_3d(sb + QH_BYTES + DHH_BYTES, &tm_stats, st_full + st, 0, it.group, th);
                     issued = g + 1;
@@ -652,55 +651,62 @@ gdla_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_cons
                 tmem_ld32x2(s_addr, lane_base + DPT_COL + 32 * half, sr, dr);
                 tc_fence_before();
                 mbar_arrive(dpt_free);  // dP^T is in registers: the next step's may overwrite it
-                // this half's 6 tokens: their row statistics, and which of them see this key
-                const float *stat = reinterpret_cast<const float *>(smem + OFF_ST + st * STAGE + QH_BYTES + DHH_BYTES) +
-                                    6 * half * kBwdStats;
-                const int th = it.u0 + s * HT + 6 * half;  // first token of this half
-                uint32_t tm = 0;                           // bit j: token th + j sees key u
+                // the step's 12 tokens: which of them see this key, and their row statistics
+                const float *stat = reinterpret_cast<const float *>(smem + OFF_ST + st * STAGE + QH_BYTES + DHH_BYTES);
+                const int th = it.u0 + s * HT;  // first token of the step
+                uint32_t tm = 0;                // bit j: token th + j sees key u
 #pragma unroll
-                for (int j = 0; j < 6; ++j) {
+                for (int j = 0; j < HT; ++j) {
                     const int t = th + j;
                     tm |= (key_ok && u <= t && t < it.L && (window <= 0 || t < u + window)) ? (1u << j) : 0u;
                 }
-                // rows 4j..4j+3 are token j's signal heads, 24 + j its noise head, 30 and 31 padding
-                uint32_t pk[16], dk2[16];
-                float l4[6], d4[6];
+                // signal rows 4j + h of the tokens j0 .. j0 + nj - 1 (h < 4), packed into pk/dk2 from 2 p0
+                auto signal_rows = [&](int j0, int nj, int r0, int p0, uint32_t (&pk)[16], uint32_t (&dk2)[16]) {
 #pragma unroll
-                for (int j = 0; j < 6; ++j) {
-                    const float4 L = *reinterpret_cast<const float4 *>(stat + j * kBwdStats);
-                    const float4 D = *reinterpret_cast<const float4 *>(stat + j * kBwdStats + 8);
-                    l4[j] = stat[j * kBwdStats + 4];
-                    d4[j] = stat[j * kBwdStats + 12];
-                    const bool vj = (tm >> j) & 1u;
-                    const float lv[4] = {L.x, L.y, L.z, L.w}, dv[4] = {D.x, D.y, D.z, D.w};
-                    float pv[4], ds[4];
-#pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        const float p = fast_exp2(fmaf(__uint_as_float(sr[4 * j + h]), kScoreLog2, -lv[h]));
-                        pv[h] = vj ? p : 0.f;
-                        ds[h] = vj ? p * (__uint_as_float(dr[4 * j + h]) - dv[h]) : 0.f;
-                    }
-                    pk[2 * j] = pack_bf16x2(pv[0], pv[1]);
-                    pk[2 * j + 1] = pack_bf16x2(pv[2], pv[3]);
-                    dk2[2 * j] = pack_bf16x2(ds[0], ds[1]);
-                    dk2[2 * j + 1] = pack_bf16x2(ds[2], ds[3]);
-                }
-#pragma unroll
-                for (int m = 0; m < 3; ++m) {
-                    float pv[2], ds[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int j = 2 * m + e;
+                    for (int jj = 0; jj < nj; ++jj) {
+                        const int j = j0 + jj;
+                        const float4 L = *reinterpret_cast<const float4 *>(stat + j * kBwdStats);
+                        const float4 D = *reinterpret_cast<const float4 *>(stat + j * kBwdStats + 8);
                         const bool vj = (tm >> j) & 1u;
-                        const float p = fast_exp2(fmaf(__uint_as_float(sr[24 + j]), kScoreLog2, -l4[j]));
-                        pv[e] = vj ? p : 0.f;
-                        ds[e] = vj ? p * (__uint_as_float(dr[24 + j]) - d4[j]) : 0.f;
+                        const float lv[4] = {L.x, L.y, L.z, L.w}, dv[4] = {D.x, D.y, D.z, D.w};
+                        float pv[4], ds[4];
+#pragma unroll
+                        for (int h = 0; h < 4; ++h) {
+                            const int r = r0 + 4 * jj + h;
+                            const float p = fast_exp2(fmaf(__uint_as_float(sr[r]), kScoreLog2, -lv[h]));
+                            pv[h] = vj ? p : 0.f;
+                            ds[h] = vj ? p * (__uint_as_float(dr[r]) - dv[h]) : 0.f;
+                        }
+                        pk[p0 + 2 * jj] = pack_bf16x2(pv[0], pv[1]);
+                        pk[p0 + 2 * jj + 1] = pack_bf16x2(pv[2], pv[3]);
+                        dk2[p0 + 2 * jj] = pack_bf16x2(ds[0], ds[1]);
+                        dk2[p0 + 2 * jj + 1] = pack_bf16x2(ds[2], ds[3]);
                     }
-                    pk[12 + m] = pack_bf16x2(pv[0], pv[1]);
-                    dk2[12 + m] = pack_bf16x2(ds[0], ds[1]);
+                };
+                uint32_t pk[16], dk2[16];
+                if (half == 0) {
+                    signal_rows(0, 8, 0, 0, pk, dk2);  // rows 0..31: tokens 0..7
+                } else {
+                    signal_rows(8, 4, 0, 0, pk, dk2);  // rows 32..47: tokens 8..11
+                    // rows 48..59: the noise head of tokens 0..11; rows 60..63 are padding
+#pragma unroll
+                    for (int m = 0; m < 6; ++m) {
+                        float pv[2], ds[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int j = 2 * m + e;
+                            const bool vj = (tm >> j) & 1u;
+                            const float p = fast_exp2(fmaf(__uint_as_float(sr[16 + j]), kScoreLog2,
+                                                           -stat[j * kBwdStats + 4]));
+                            pv[e] = vj ? p : 0.f;
+                            ds[e] = vj ? p * (__uint_as_float(dr[16 + j]) - stat[j * kBwdStats + 12]) : 0.f;
+                        }
+                        pk[8 + m] = pack_bf16x2(pv[0], pv[1]);
+                        dk2[8 + m] = pack_bf16x2(ds[0], ds[1]);
+                    }
+                    pk[14] = pk[15] = 0u;
+                    dk2[14] = dk2[15] = 0u;
                 }
-                pk[15] = 0u;
-                dk2[15] = 0u;
                 tmem_st16x2(s_addr, pk, s_addr + 16, dk2);
                 tc_fence_before();
                 mbar_arrive(pds_full + b);
@@ -792,7 +798,7 @@ static cudaError_t launch_dkv_sized(const BwdLaunch &L, const Plan &plan, cudaSt
     const long long work = static_cast<long long>(plan.n_items) * plan.hkv;
     const unsigned grid = static_cast<unsigned>(work < num_sms ? work : num_sms);
     gdla_bwd_dkv_kernel<Plan><<<grid, pbk::NUM_THREADS, pbk::SMEM_BYTES, stream>>>(
-        L.tm_qs, L.tm_qn, L.tm_dhs, L.tm_dhn, L.tm_k128, L.tm_v128, L.tm_stats, L.dk, L.dv, plan);
+        L.tm_qs12, L.tm_qn12, L.tm_dhs12, L.tm_dhn12, L.tm_k128, L.tm_v128, L.tm_stats, L.dk, L.dv, plan);
     return cudaPeekAtLastError();
 }
 

@@ -296,9 +296,9 @@ __device__ __forceinline__ void epi_backward(uint32_t o_addr, float l_run, float
         for (int i = 0; i < 16; ++i) {
             const float h0 = __uint_as_float(o[2 * i]) * inv_l, h1 = __uint_as_float(o[2 * i + 1]) * inv_l;
             const float hn0 = __shfl_sync(0xffffffffu, h0, hsrc), hn1 = __shfl_sync(0xffffffffu, h1, hsrc);
-            const float g0 = __uint_as_float(g[i] << 16), g1 = __uint_as_float(g[i] & 0xFFFF0000u);
             const float o0 = __uint_as_float(go[i] << 16), o1 = __uint_as_float(go[i] & 0xFFFF0000u);
-            const float s0 = 1.f / (1.f + __expf(-g0)), s1 = 1.f / (1.f + __expf(-g1));
+            float s0, s1;  // sigmoid of the gate pair, one tanh for both
+            f2_unpack(sigmoid2_bf16(g[i]), s0, s1);
             const float d0 = h0 - lam * hn0, d1 = h1 - lam * hn1;
             const float dD0 = o0 * s0, dD1 = o1 * s1;
             w_dgate[i] = pack_bf16x2(o0 * d0 * s0 * (1.f - s0), o1 * d1 * s1 * (1.f - s1));

@@ -354,26 +354,29 @@ gdla_status_t gdla_attn_bwd(const void *q_sig, const void *q_noise, const void *
     const int TQ = kPrefillTileTokens / 4;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    // 1. forward recompute: dgate, dlambda, dH, row statistics (24-token items, 128-key tiles)
+    // 1. forward recompute: dgate, dlambda, dH, row statistics, with the forward's tiling
+    //    (24-token items over 128-key tiles; short windows 48-token items over 64-key tiles)
+    const PrefillGeometry geo = prefill_geometry(window);
     PrefillLaunch F{};
     if (!make_map(&F.tm_qs, q_sig, 192, 4 * hkv, N, 64, 4, TQ) || !make_map(&F.tm_qn, q_noise, 192, hkv, N, 64, 1, TQ) ||
-        !make_map(&F.tm_k, k, 192, hkv, N, 64, 1, 128) || !make_map(&F.tm_v, v, 128, hkv, N, 64, 1, 128))
+        !make_map(&F.tm_k, k, 192, hkv, N, 64, 1, geo.key_tile) ||
+        !make_map(&F.tm_v, v, 128, hkv, N, 64, 1, geo.v_box))
         return GDLA_ERR_CUDA;
     F.lambda = lambda;
     F.gate = static_cast<const __nv_bfloat16 *>(gate_logits);
     F.bwd = {static_cast<const __nv_bfloat16 *>(dout), static_cast<__nv_bfloat16 *>(dgate), dlambda, dh_sig, dh_noise,
              stats};
-    const int T = kPrefillTileTokens;
-    auto q_cost = [&](int key_tile) {
+    auto q_cost = [&](int T, int key_tile) {
         return [=](int L, int qt) {
             const int t0 = qt * T;
             const int lo = (window > 0) ? std::max(0, t0 - window + 1) : 0;
             return (std::min(L, t0 + T) - lo + key_tile - 1) / key_tile;
         };
     };
-    if (!run_plans(batch, seqlens, hkv, window, T, q_cost(128),
+    if (!run_plans(batch, seqlens, hkv, window, geo.cta_tokens, q_cost(geo.cta_tokens, geo.key_tile),
                    [&](const PrefillPlan &P) { return launch_prefill_bwd_recompute(F, P, st) == cudaSuccess; }))
         return GDLA_ERR_CUDA;
+    const int T = kPrefillTileTokens;
 
     // 2. dQ (24-token items over 64-key tiles) and 3. dK, dV (128-key items over 12-token steps)
     BwdLaunch B{};
@@ -395,7 +398,7 @@ gdla_status_t gdla_attn_bwd(const void *q_sig, const void *q_noise, const void *
     B.dq_noise = static_cast<__nv_bfloat16 *>(dq_noise);
     B.dk = static_cast<__nv_bfloat16 *>(dk);
     B.dv = static_cast<__nv_bfloat16 *>(dv);
-    if (!run_plans(batch, seqlens, hkv, window, T, q_cost(kBwdQKeyTile),
+    if (!run_plans(batch, seqlens, hkv, window, T, q_cost(T, kBwdQKeyTile),
                    [&](const PrefillPlan &P) { return launch_bwd_dq(B, P, st) == cudaSuccess; }))
         return GDLA_ERR_CUDA;
     auto kv_cost = [=](int L, int kt) {

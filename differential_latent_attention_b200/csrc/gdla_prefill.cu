@@ -148,7 +148,8 @@ struct Cfg {
     static_assert(STAGES <= 3, "three barriers each for K and V stages");
 };
 using CausalCfg = Cfg<1, 128, 2, EPI_HALF>;
-using BwdRecomputeCfg = Cfg<1, 128, 2, EPI_BWD>;  // every window: the one-tile schedule
+using BwdRecomputeCfg = Cfg<1, 128, 2, EPI_BWD>;         // full causal and long windows: the one-tile schedule
+using BwdRecomputeSlidingCfg = Cfg<2, 64, 2, EPI_BWD>;  // short windows: the forward's sliding schedule
 using SlidingCfg = Cfg<2, 64, 2, EPI_STAGED>;
 
 // ------------------------------- epilogue ----------------------------------
@@ -951,6 +952,8 @@ cudaError_t launch_prefill_bwd_recompute(const PrefillLaunch &L, const PrefillPl
     if (e != cudaSuccess) return e;
     const int num_sms = device_sm_count(dev);
     if (num_sms <= 0) return cudaErrorInvalidDevice;
+    if (plan.window > 0 && plan.window <= kPrefillSlidingMaxWindow)
+        return launch_sized<pf::BwdRecomputeSlidingCfg>(L, plan, dev, num_sms, stream);
     return launch_sized<pf::BwdRecomputeCfg>(L, plan, dev, num_sms, stream);
 }
 

@@ -99,8 +99,8 @@ cudaError_t launch_bwd_dq(const BwdLaunch &launch, const PrefillPlan &plan, cuda
 cudaError_t launch_bwd_dkv(const BwdLaunch &launch, const PrefillPlan &plan, cudaStream_t stream);
 
 cudaError_t launch_prefill(const PrefillLaunch &launch, const PrefillPlan &plan, cudaStream_t stream);
-// Backward, first pass: the forward recomputed with the one-tile schedule (items of
-// kPrefillTileTokens tokens over 128-key tiles, for every window), writing launch.bwd.
+// Backward, first pass: the forward recomputed on the forward's schedule for the
+// plan's window (prefill_geometry), writing launch.bwd instead of the output.
 cudaError_t launch_prefill_bwd_recompute(const PrefillLaunch &launch, const PrefillPlan &plan, cudaStream_t stream);
 
 // SM count of a device, queried once per device and cached (0 on failure).

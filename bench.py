@@ -257,11 +257,19 @@ def time_steps(fn, steps, warmup, flush, world):
     return [s.elapsed_time(e) for s, e in ev]
 
 
+# Device-side spin before each rotating step, outside its events (~50 us at 1.9 GHz):
+# a call of a few tens of microseconds would otherwise be timed from its start event
+# to its end event while the host was still enqueueing its launches.
+HOST_LEAD_CYCLES = 100_000
+
+
 def time_rotating(fns, steps, warmup, world):
     """Per-step device time (ms) with CUDA events, step i running fns[i % len(fns)]
     and no L2 flush: the sets' inputs together exceed twice the L2, so each step's
     inputs have been evicted since their previous use and no dirty flush lines are
-    written back inside the timed region."""
+    written back inside the timed region. A short device-side spin (touching no
+    memory) precedes each step's start event, so the host has enqueued the step's
+    launches before the step's timing starts."""
     for i in range(warmup):
         fns[i % len(fns)]()
     torch.cuda.synchronize()
@@ -269,6 +277,7 @@ def time_rotating(fns, steps, warmup, world):
     stream = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for i, (s, e) in enumerate(ev):
+        torch.cuda._sleep(HOST_LEAD_CYCLES)
         s.record(stream)
         fns[(warmup + i) % len(fns)]()
         e.record(stream)

@@ -67,6 +67,13 @@ def test_several_tiles_and_ragged_tail():
     check_bwd((700,), 2, 128, 4)
 
 
+@pytest.mark.parametrize("window", [200, 256, 300])
+def test_window_schedules(window):
+    # windows up to 256 recompute on the sliding schedule (48-token items, 64-key tiles),
+    # longer ones on the one-tile schedule (24-token items, 128-key tiles)
+    check_bwd((700, 333), 2, window, 10 + window)
+
+
 def test_sixteen_groups():
     check_bwd((300, 77), 16, 0, 5)
 

@@ -141,3 +141,77 @@ def test_latent_workspace_sizes(lib):
     assert lib.gdla_decode_latent_workspace_bytes(1, 16, 1 << 20, 0) == 32 * per        # at most 32 splits
     assert lib.gdla_decode_latent_workspace_bytes(1, 17, 4096, 0) == 0
     assert lib.gdla_decode_latent_workspace_bytes(0, 16, 4096, 0) == 0
+
+
+def _bwd(lib, lens, hkv=1, window=0, ptrs=None, ws=FAKE, ws_bytes=1 << 40):
+    arr = (ctypes.c_int32 * len(lens))(*lens)
+    p = ptrs or [FAKE] * 13
+    return lib.gdla_attn_bwd(*[ctypes.c_void_p(x) for x in p], len(lens), arr, hkv, window, ctypes.c_void_p(ws),
+                             ws_bytes, None)
+
+
+def test_bwd_argument_checks(lib):
+    assert _bwd(lib, [4], hkv=0) == 2
+    assert _bwd(lib, [4], hkv=65) == 2
+    assert _bwd(lib, [4, -1]) == 1
+    assert lib.gdla_attn_bwd(*[ctypes.c_void_p(FAKE)] * 13, 0, None, 1, 0, ctypes.c_void_p(FAKE), 1, None) == 1
+    assert _bwd(lib, [0, 0]) == 0                                                        # nothing to do
+    for i in range(13):
+        p = [FAKE] * 13
+        p[i] = 0
+        assert _bwd(lib, [4], ptrs=p) == 1                                                # null
+        p[i] = FAKE + 8
+        assert _bwd(lib, [4], ptrs=p) == 1                                                # misaligned
+    assert _bwd(lib, [2 ** 30, 2 ** 30]) == 1                                             # N >= 2^31
+    need = lib.gdla_attn_bwd_workspace_bytes(4, 1)
+    assert _bwd(lib, [4], ws=0) == 3
+    assert _bwd(lib, [4], ws_bytes=need - 1) == 3
+    assert _bwd(lib, [4], ws=FAKE + 16) == 3                                              # not 256-byte aligned
+
+
+def test_bwd_workspace_sizes(lib):
+    # dH_S [N, 4H, 128] and dH_N [N, H, 128] bf16, row statistics [N, H, 16] fp32, each 256-byte aligned
+    a = lambda b: (b + 255) // 256 * 256
+    n, h = 4096, 16
+    assert lib.gdla_attn_bwd_workspace_bytes(n, h) == a(n * 4 * h * 256) + a(n * h * 256) + a(n * h * 64)
+    assert lib.gdla_attn_bwd_workspace_bytes(37, 3) == a(37 * 12 * 256) + a(37 * 3 * 256) + a(37 * 3 * 64)
+    assert lib.gdla_attn_bwd_workspace_bytes(-1, 16) == 0
+    assert lib.gdla_attn_bwd_workspace_bytes(4, 0) == 0
+    assert lib.gdla_attn_bwd_workspace_bytes(4, 65) == 0
+
+
+def _pro(lib, lens, hkv=1, ptrs=None, ws=FAKE, ws_bytes=1 << 40):
+    arr = (ctypes.c_int32 * len(lens))(*lens)
+    p = ptrs or [FAKE] * 16
+    return lib.gdla_prologue(*[ctypes.c_void_p(x) for x in p], len(lens), arr, hkv, ctypes.c_void_p(ws), ws_bytes,
+                             None)
+
+
+def test_prologue_argument_checks(lib):
+    assert _pro(lib, [4], hkv=0) == 2
+    assert _pro(lib, [4], hkv=65) == 2
+    assert _pro(lib, [1] * 1025) == 2                                                     # more sequences than a plan holds
+    assert _pro(lib, [4, -1]) == 1
+    assert lib.gdla_prologue(*[ctypes.c_void_p(FAKE)] * 16, 0, None, 1, ctypes.c_void_p(FAKE), 1, None) == 1
+    assert _pro(lib, [0, 0]) == 0                                                         # nothing to do
+    for i in range(16):
+        p = [FAKE] * 16
+        p[i] = 0
+        assert _pro(lib, [4], ptrs=p) == 1                                                # null
+        p[i] = FAKE + 8
+        assert _pro(lib, [4], ptrs=p) == 1                                                # misaligned
+    assert _pro(lib, [2 ** 30, 2 ** 30]) == 1                                             # N >= 2^31
+    need = lib.gdla_prologue_workspace_bytes(4)
+    assert _pro(lib, [4], ws=0) == 3
+    assert _pro(lib, [4], ws_bytes=need - 1) == 3
+    assert _pro(lib, [4], ws=FAKE + 16) == 3
+
+
+def test_prologue_workspace_sizes(lib):
+    # c^Q * gamma and c^KV * gamma (bf16), partial sums of squares [N, 16], rotated k^R [N, 64] bf16,
+    # rotary table [N, 64] fp32, each 256-byte aligned
+    a = lambda b: (b + 255) // 256 * 256
+    for n in (4096, 37):
+        assert lib.gdla_prologue_workspace_bytes(n) == (a(n * 2048) + a(n * 1024) + a(n * 64) + a(n * 128) +
+                                                        a(n * 256))
+    assert lib.gdla_prologue_workspace_bytes(-1) == 0

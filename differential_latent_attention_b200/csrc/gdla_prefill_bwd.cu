@@ -95,7 +95,11 @@ constexpr uint32_t QD_TX = (3 + 2) * 4 * QBOX_TX;  // Q and dH tiles of one item
 // dQ, then two buffers of (S, dP): the next key tile's products run while the
 // row warps turn this tile's into dS (written over its S).
 constexpr uint32_t DQ_COL = 0, S_COL0 = 192, DP_COL0 = 256, BUF_COLS = 128;
+// The item's dH tile, copied from shared memory once per item: dP = dH V^T then reads
+// its A operand from TMEM (only V from shared memory, full rate at N = 64).
+constexpr uint32_t DH_COL = 448;
 constexpr uint32_t TMEM_COLS = 512;
+static_assert(DH_COL + DV / 2 <= TMEM_COLS, "TMEM budget");
 // 8 row warps: two per TMEM lane quarter (warp % 4), each taking one half (warp / 4)
 // of a key tile's 32 + 32 columns; producer warp 8, MMA warp 9.
 constexpr int ROW_WARPS = 8;
@@ -242,6 +246,13 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
         for (int w = snake_item(0); ok && w < n_work; w = snake_item(n_item + 1), ++n_item) {
             const Item it = item_at(w);
             if (!__all_sync(0xffffffffu, mbar_wait(q_full, n_item & 1, abort_flag, ERR_SITE_BWD | 3))) break;
+            // dH (staged in shared memory) -> TMEM, one 16-dim K step per copy; the dP products
+            // below are issued after these copies and run after them
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < DV / 16; ++kk)
+                tmem_cp_128x256b_leader(tmem + DH_COL + kk * 8,
+                                        dh_desc0 + (((kk >> 2) * Q_CHUNK + (kk & 3) * 32) >> 4), leader);
             // S and dP of key tile k (global tile index kv + k, global step step + k)
             auto issue_sdp = [&](int k) {
                 const int st = (kv + k) % STAGES;
@@ -259,9 +270,9 @@ gdla_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
                 }
 #pragma unroll
                 for (int kk = 0; kk < DV / 16; ++kk) {
-                    const uint32_t offd = ((kk >> 2) * Q_CHUNK + (kk & 3) * 32) >> 4;
                     const uint32_t offv = (sbase + K_STAGE + (kk >> 2) * KV_CHUNK + (kk & 3) * 32) >> 4;
-                    umma_ss_leader(tmem + DP_COL0 + buf, dh_desc0 + offd, kv_desc0 + offv, idesc_s, kk > 0, leader);
+                    umma_ts_leader(tmem + DP_COL0 + buf, tmem + DH_COL + kk * 8, kv_desc0 + offv, idesc_s, kk > 0,
+                                   leader);
                 }
                 umma_commit_leader(s_full + ((step + k) & 1), leader);
                 if (k == it.n_tiles - 1) umma_commit_leader(q_empty, leader);

@@ -78,6 +78,30 @@ def test_sixteen_groups():
     check_bwd((300, 77), 16, 0, 5)
 
 
+@pytest.mark.parametrize("w", [gi.PREFILL_FULL, gi.SWA], ids=lambda w: w.name)
+def test_bench_workload_two_groups(w):
+    """The bench's own backward workloads in its launch (T = 4096 full causal, and 2 x 32768 at
+    window 128, all 16 KV groups in one call). A group's gradients depend on its own five heads,
+    K and V only, so the oracle checks the first and the last group, each as a one-group problem."""
+    t = gi.make_prefill_inputs(w.seqlens, w.num_kv_heads, w.seed, device="cuda")
+    dout = gi.make_prefill_grad(w.seqlens, w.num_kv_heads, w.seed, device="cuda")
+    g = gdla.attn_bwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"], dout, w.seqlens, w.window)
+    torch.cuda.synchronize()
+    assert gdla.device_error() == 0
+    for j in (0, w.num_kv_heads - 1):
+        sig, noi = slice(4 * j, 4 * j + 4), slice(j, j + 1)
+        ref = oracle.prefill_bwd(gi.bf16_bits(t["q_sig"][:, sig]), gi.bf16_bits(t["q_noise"][:, noi]),
+                                 gi.bf16_bits(t["k"][:, noi]), gi.bf16_bits(t["v"][:, noi]),
+                                 t["lam"][:, sig].cpu().numpy(), gi.bf16_bits(t["gate"][:, sig]),
+                                 gi.bf16_bits(dout[:, sig]), w.seqlens, w.window)
+        got = {"dq_sig": g["dq_sig"][:, sig], "dq_noise": g["dq_noise"][:, noi], "dk": g["dk"][:, noi],
+               "dv": g["dv"][:, noi], "dlambda": g["dlambda"][:, sig], "dgate": g["dgate"][:, sig]}
+        report = {name: _errors(got[name], ref[name]) for name in NAMES}
+        print(f"bwd {w.name} group {j}: " + " ".join(f"{n}=({m:.1e},{r:.1e})" for n, (m, r) in report.items()))
+        for name, (mx, rel) in report.items():
+            assert rel <= 5e-3 and mx <= 2e-2, (j, name, mx, rel)
+
+
 def test_deterministic():
     seqlens, hkv = (200, 61), 2
     t = gi.make_prefill_inputs(seqlens, hkv, 9, device="cuda")

@@ -6,8 +6,13 @@ K_j = [W^UK_j c | kr], V_j = W^UV_j c. With the query's non-rotary part
 absorbed (q_abs = [W^UK_j^T q_nope | q_rope]) the scores and outputs are the
 same numbers computed in another order. The inputs here are small integers and
 sparse +-1 projections, so every expanded and absorbed tensor is exact in bf16
-and the two independent fp64 computations must agree to rounding.
+and the two independent fp64 computations must agree to rounding. Slips planted in
+copies of the latent oracle's own code must each break that agreement.
 """
+import ctypes
+import os
+import subprocess
+
 import numpy as np
 import pytest
 
@@ -93,3 +98,60 @@ def test_plausible_slips_break_the_equivalence(slip):
     else:
         got = _absorbed(x, 0, drop_rope=True)
     assert np.abs(got - ref).max() > 1e-3
+
+
+# Planted slips inside the latent oracle itself: each is a copy of the oracle source
+# with one plausible mistake in the latent path (scale, rotary dims, value slice,
+# W^UV layout or group, noise-head index, window edge, subtract sign, normalisation),
+# built on the CPU; the expanded decode (untouched code) must then disagree.
+LATENT_MUTANTS = {
+    "scale_dropped": ("for (int e = 0; e < DL; ++e) s += qd[e] * bf16_to_double(r[e]);\n        s = s / root;",
+                      "for (int e = 0; e < DL; ++e) s += qd[e] * bf16_to_double(r[e]);"),
+    "rope_dims_dropped": ("for (int e = 0; e < DL; ++e) s += qd[e] * bf16_to_double(r[e]);",
+                          "for (int e = 0; e < DC; ++e) s += qd[e] * bf16_to_double(r[e]);"),
+    "values_from_wrong_slice": ("for (int e = 0; e < DC; ++e) o[e] += w * bf16_to_double(r[e]);",
+                                "for (int e = 0; e < DC; ++e) o[e] += w * bf16_to_double(r[e + DR]);"),
+    "up_projection_transposed": ("bf16_to_double(w_uv_j[(long)d * DC + e])", "bf16_to_double(w_uv_j[(long)e * DV + d])"),
+    "noise_group_index": ("attend_latent(J->q_noise + (b * J->hkv + j) * DL,",
+                          "attend_latent(J->q_noise + (b * J->hkv + (J->hkv - 1 - j)) * DL,"),
+    "w_uv_group_dropped": ("const uint16_t *w_uv_j = J->w_uv + (long)j * DV * DC;", "const uint16_t *w_uv_j = J->w_uv;"),
+    "window_off_by_one": ("if (J->window > 0 && t - J->window + 1 > 0) lo = t - J->window + 1;\n"
+                          "        const long nkeys = (long)(t - lo + 1);\n        const uint16_t *rows = J->ckv",
+                          "if (J->window > 0 && t - J->window + 2 > 0) lo = t - J->window + 2;\n"
+                          "        const long nkeys = (long)(t - lo + 1);\n        const uint16_t *rows = J->ckv"),
+    "subtract_sign": ("const double dd = hsig[d] - l * hn[d];", "const double dd = hsig[d] + l * hn[d];"),
+    "normalisation_dropped": ("for (int e = 0; e < DC; ++e) o[e] /= den;", ""),
+}
+MUTANT_DIR = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "_build", "oracle_mutants")
+
+
+def _build_latent_mutant(name, old, new):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "gdla_oracle.c")).read()
+    assert src.count(old) == 1, name
+    os.makedirs(MUTANT_DIR, exist_ok=True)
+    c = os.path.join(MUTANT_DIR, f"latent_{name}.c")
+    so = os.path.join(MUTANT_DIR, f"liblatent_{name}.so")
+    with open(c, "w") as f:
+        f.write(src.replace(old, new))
+    subprocess.check_call(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-pthread", "-o", so, c, "-lm"],
+                          env={**os.environ, "TMPDIR": MUTANT_DIR})
+    lib = ctypes.CDLL(so)
+    real = oracle._load()
+    for fn in ("gdla_oracle_decode", "gdla_oracle_decode_latent"):
+        getattr(lib, fn).argtypes = getattr(real, fn).argtypes
+        getattr(lib, fn).restype = getattr(real, fn).restype
+    return lib
+
+
+@pytest.mark.parametrize("name", sorted(LATENT_MUTANTS))
+def test_planted_latent_slip_is_caught(name, monkeypatch):
+    lib = _build_latent_mutant(name, *LATENT_MUTANTS[name])
+    worst = 0.0
+    for window in (0, 16):
+        x = _case(95 + window, (1, 7, 40, 129), 2)
+        ref = _expanded(x, window)               # the unmodified expanded decode
+        monkeypatch.setattr(oracle, "_lib", lib)
+        got = _absorbed(x, window)               # the mutant's latent path
+        monkeypatch.undo()
+        worst = max(worst, float(np.abs(got - ref).max()))
+    assert worst > 1e-6, f"mutant {name} not caught (worst {worst:.2e})"

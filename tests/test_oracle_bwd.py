@@ -121,6 +121,13 @@ BWD_MUTANTS = {
     "dnoise_without_lambda": ("dh[GROUP][d] -= l * ddd;", "dh[GROUP][d] -= ddd;"),
     "dgate_without_sigma_prime": ("go * dd * sg * (1.0 - sg)", "go * dd * sg"),
     "dk_unscaled": ("dkr[d] += ds * bf16_to_double(q[d]) / root;", "dkr[d] += ds * bf16_to_double(q[d]);"),
+    "dq_unscaled": ("dq[d] += ds * bf16_to_double(kr[d]) / root;", "dq[d] += ds * bf16_to_double(kr[d]);"),
+    "window_off_by_one": ("if (J->window > 0 && t - J->window + 1 > 0) lo = t - J->window + 1;\n"
+                          "            const long nkeys = t - lo + 1;",
+                          "if (J->window > 0 && t - J->window + 2 > 0) lo = t - J->window + 2;\n"
+                          "            const long nkeys = t - lo + 1;"),
+    "gate_sign": ("const double sg = 1.0 / (1.0 + exp(-g));", "const double sg = 1.0 / (1.0 + exp(g));"),
+    "dD_without_gate": ("const double ddd = go * sg;", "const double ddd = go;"),
     "dv_from_wrong_head": ("for (int d = 0; d < DV; ++d) dvr[d] += p[u] * dh[d];",
                            "for (int d = 0; d < DV; ++d) dvr[d] += p[u] * dh[d] * (dq == J_unused ? 0 : 1);"),
 }

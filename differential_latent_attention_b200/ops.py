@@ -96,6 +96,31 @@ def _stream(stream):
     return stream.cuda_stream
 
 
+def _on_one_device(stream, named):
+    """Every tensor of a call on one CUDA device, and the launch stream on it too: the
+    library launches on that stream and its kernels dereference every pointer there.
+    ``named`` holds (name, tensor) pairs already checked to be CUDA tensors (None skipped)."""
+    dev = None
+    for name, t in named:
+        if t is None:
+            continue
+        d = t.get_device()
+        if dev is None:
+            dev = d
+        elif d != dev:
+            raise ValueError(f"{name} is on cuda:{d}, the call's other tensors on cuda:{dev}")
+    sdev = stream.device.index if stream is not None else torch.cuda.current_device()
+    if dev is not None and sdev != dev:
+        raise ValueError(f"the tensors are on cuda:{dev} but the launch stream is on cuda:{sdev}")
+
+
+def _check_workspace(ws):
+    if ws is None:
+        return
+    if not isinstance(ws, torch.Tensor) or not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+
+
 def _check(t, name, dtype, shape):
     # common case first: one combined test per call, the detailed ones only to explain a failure
     if type(t) is torch.Tensor and t.dtype is dtype and t.shape == shape and t.is_cuda and t.is_contiguous():
@@ -133,6 +158,8 @@ def attn_fwd(q_sig, q_noise, k, v, lam, gate, seqlens, window=0, out=None, strea
     if out is None:
         out = torch.empty((n, hs, DV), dtype=torch.bfloat16, device=q_sig.device)
     _check(out, "out", torch.bfloat16, (n, hs, DV))
+    _on_one_device(stream, (("q_sig", q_sig), ("q_noise", q_noise), ("k", k), ("v", v), ("lam", lam),
+                            ("gate", gate), ("out", out)))
     st = library().gdla_attn_fwd(_ptr(q_sig), _ptr(q_noise), _ptr(k), _ptr(v), _ptr(lam), _ptr(gate), _ptr(out),
                                  int(lens.shape[0]), lens.__array_interface__["data"][0], hkv, int(window),
                                  _stream(stream))
@@ -174,6 +201,9 @@ def attn_bwd(q_sig, q_noise, k, v, lam, gate, dout, seqlens, window=0, grads=Non
     need = attn_bwd_workspace_bytes(n, hkv)
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q_sig.device)
+    _check_workspace(workspace)
+    _on_one_device(stream, [("q_sig", q_sig), ("q_noise", q_noise), ("k", k), ("v", v), ("lam", lam),
+                            ("gate", gate), ("dout", dout), ("workspace", workspace)] + list(grads.items()))
     ws_bytes = workspace.numel() * workspace.element_size()
     st = library().gdla_attn_bwd(_ptr(q_sig), _ptr(q_noise), _ptr(k), _ptr(v), _ptr(lam), _ptr(gate), _ptr(dout),
                                  _ptr(grads["dq_sig"]), _ptr(grads["dq_noise"]), _ptr(grads["dk"]), _ptr(grads["dv"]),
@@ -221,6 +251,10 @@ def prologue(x, w_qa, w_kva, gamma_q, gamma_kv, w_qb, w_uk, w_uv, w_lambda, w_ga
         _check(outs[name], name, dt, shape)
     if workspace is None:
         workspace = torch.empty(max(prologue_workspace_bytes(n), 1), dtype=torch.uint8, device=x.device)
+    _check_workspace(workspace)
+    _on_one_device(stream, [("x", x), ("w_qa", w_qa), ("w_kva", w_kva), ("gamma_q", gamma_q), ("gamma_kv", gamma_kv),
+                            ("w_qb", w_qb), ("w_uk", w_uk), ("w_uv", w_uv), ("w_lambda", w_lambda),
+                            ("w_gate", w_gate), ("workspace", workspace)] + list(outs.items()))
     st = library().gdla_prologue(_ptr(x), _ptr(w_qa), _ptr(w_kva), _ptr(gamma_q), _ptr(gamma_kv), _ptr(w_qb),
                                  _ptr(w_uk), _ptr(w_uv), _ptr(w_lambda), _ptr(w_gate), _ptr(outs["q_sig"]),
                                  _ptr(outs["q_noise"]), _ptr(outs["k"]), _ptr(outs["v"]), _ptr(outs["lam"]),
@@ -262,6 +296,10 @@ def attn_decode(q_sig, q_noise, k_cache, v_cache, cu_seqlens_k, max_seqlen_k, la
     need = decode_workspace_bytes(b, hkv, max_seqlen_k, window)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q_sig.device)
+    _check_workspace(workspace)
+    _on_one_device(stream, (("q_sig", q_sig), ("q_noise", q_noise), ("k_cache", k_cache), ("v_cache", v_cache),
+                            ("cu_seqlens_k", cu_seqlens_k), ("lam", lam), ("gate", gate), ("out", out),
+                            ("workspace", workspace)))
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = library().gdla_attn_decode(_ptr(q_sig), _ptr(q_noise), _ptr(k_cache), _ptr(v_cache), _ptr(cu_seqlens_k),
                                     int(nk), int(max_seqlen_k), _ptr(lam), _ptr(gate), _ptr(out), int(b), hkv,
@@ -303,6 +341,10 @@ def attn_decode_latent(q_abs_sig, q_abs_noise, ckv, cu_seqlens_k, max_seqlen_k, 
     need = decode_latent_workspace_bytes(b, hkv, max_seqlen_k, window)
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q_abs_sig.device)
+    _check_workspace(workspace)
+    _on_one_device(stream, (("q_abs_sig", q_abs_sig), ("q_abs_noise", q_abs_noise), ("ckv", ckv),
+                            ("cu_seqlens_k", cu_seqlens_k), ("w_uv", w_uv), ("lam", lam), ("gate", gate),
+                            ("out", out), ("workspace", workspace)))
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = library().gdla_attn_decode_latent(_ptr(q_abs_sig), _ptr(q_abs_noise), _ptr(ckv), _ptr(cu_seqlens_k),
                                            int(nk), int(max_seqlen_k), _ptr(w_uv), _ptr(lam), _ptr(gate),

@@ -215,3 +215,34 @@ def test_prologue_workspace_sizes(lib):
         assert lib.gdla_prologue_workspace_bytes(n) == (a(n * 2048) + a(n * 1024) + a(n * 64) + a(n * 128) +
                                                         a(n * 256))
     assert lib.gdla_prologue_workspace_bytes(-1) == 0
+
+
+class _OnDevice:
+    """Stands in for a CUDA tensor's device index (the binding's device check reads only that)."""
+
+    def __init__(self, index):
+        self.index = index
+
+    def get_device(self):
+        return self.index
+
+
+class _StreamOn:
+    def __init__(self, index):
+        import torch
+        self.device = torch.device("cuda", index)
+
+
+def test_binding_wants_one_device_for_tensors_and_stream():
+    ops._on_one_device(_StreamOn(1), [("a", _OnDevice(1)), ("b", None), ("c", _OnDevice(1))])
+    with pytest.raises(ValueError, match="c is on cuda:0"):
+        ops._on_one_device(_StreamOn(1), [("a", _OnDevice(1)), ("c", _OnDevice(0))])
+    with pytest.raises(ValueError, match="launch stream is on cuda:0"):
+        ops._on_one_device(_StreamOn(0), [("a", _OnDevice(1))])
+
+
+def test_binding_rejects_a_host_workspace():
+    import torch
+    ops._check_workspace(None)
+    with pytest.raises(ValueError, match="workspace"):
+        ops._check_workspace(torch.empty(16, dtype=torch.uint8))

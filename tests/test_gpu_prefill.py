@@ -200,3 +200,56 @@ def test_window_at_least_length_equals_full_bitwise():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     assert torch.equal(c.view(torch.int16), d.view(torch.int16))
     check_prefill(short, 2, 256, 24, t=ts)
+
+
+def _closed_form(t, rows, v_rows):
+    """sigma(g) (1 - lambda) v for the given output rows, each with its own value row
+    per KV group (fp64, from the inputs as stored)."""
+    g = t["gate"][rows].double().cpu()                               # [R, 4H, 128]
+    lam = t["lam"][rows].double().cpu()                              # [R, 4H]
+    v = v_rows.double().cpu().repeat_interleave(4, dim=1)            # [R, 4H, 128]
+    return (torch.sigmoid(g) * (1.0 - lam)[..., None] * v).numpy()
+
+
+@pytest.mark.parametrize("window", [1, 0])
+def test_single_visible_key_closed_form(window):
+    """A row that sees one key (every row at window 1; the first row of each sequence
+    otherwise) has H_S = H_N = v_t, so out = sigmoid(g) (1 - lambda) v_t: the GPU output
+    against that closed form in fp64, not against the oracle."""
+    seqlens = (37, 1, 130, 24, 25)
+    t = gi.make_prefill_inputs(seqlens, 2, 31 + window, device="cuda")
+    out = gpu_prefill(t, seqlens, window)
+    torch.cuda.synchronize()
+    starts = np.concatenate([[0], np.cumsum(seqlens)[:-1]])
+    rows = torch.arange(sum(seqlens)) if window == 1 else torch.as_tensor(starts)
+    ref = _closed_form(t, rows, t["v"][rows])
+    assert_close(out[rows.cuda()].float().cpu().numpy(), ref, f"one visible key, window {window}")
+
+
+@pytest.mark.parametrize("window", [0, 128])
+def test_identical_value_rows_closed_form(window):
+    """All value rows of a group equal (v_u = c_j): the softmax weights sum to one, so
+    out = sigmoid(g) (1 - lambda) c_j for every row, whatever the scores."""
+    seqlens = (300, 61)
+    t = gi.make_prefill_inputs(seqlens, 2, 33 + window, device="cuda")
+    t["v"] = t["v"][:1].expand_as(t["v"]).contiguous()
+    out = gpu_prefill(t, seqlens, window)
+    torch.cuda.synchronize()
+    rows = torch.arange(sum(seqlens))
+    ref = _closed_form(t, rows, t["v"])
+    assert_close(out.float().cpu().numpy(), ref, f"identical value rows, window {window}")
+
+
+def test_saturated_gate_gives_the_ungated_difference():
+    """Gate logits 40 and 60 both give sigmoid = 1 to fp32 resolution: the outputs are
+    bit-identical, and equal to the oracle's D = H_S - lambda H_N."""
+    seqlens = (200, 33)
+    t = gi.make_prefill_inputs(seqlens, 2, 35, device="cuda")
+    t["gate"] = torch.full_like(t["gate"], 40.0)
+    a = gpu_prefill(t, seqlens, 0)
+    t60 = dict(t, gate=torch.full_like(t["gate"], 60.0))
+    b = gpu_prefill(t60, seqlens, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    ref = oracle.prefill(*host_args(t), seqlens, 0)
+    assert_close(a.float().cpu().numpy(), ref, "gate logit 40")

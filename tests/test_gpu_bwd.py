@@ -112,3 +112,32 @@ def test_deterministic():
     torch.cuda.synchronize()
     for name in NAMES:
         assert torch.equal(a[name], b[name]), name
+
+
+def test_window_one_closed_form():
+    """Window 1: every token attends only to itself (P = 1), so with s = sigmoid(g),
+    D_i = (1 - lambda_i) v and dD_i = dout_i s_i:
+        dgate_i = dout_i D_i s_i (1 - s_i),  dlambda_i = -sum_d dD_i v,
+        dv = sum_i (1 - lambda_i) dD_i,  and dq, dk vanish (dS = P (dP - rowsum) = 0).
+    The GPU gradients against those closed forms in fp64, not against the oracle."""
+    seqlens = (37, 1, 130, 24)
+    hkv = 2
+    t = gi.make_prefill_inputs(seqlens, hkv, 41, device="cuda")
+    dout = gi.make_prefill_grad(seqlens, hkv, 41, device="cuda")
+    g = gdla.attn_bwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"], dout, seqlens, 1)
+    torch.cuda.synchronize()
+    assert gdla.device_error() == 0
+    s = torch.sigmoid(t["gate"].double().cpu())                              # [N, 4H, 128]
+    lam = t["lam"].double().cpu()[..., None]                                 # [N, 4H, 1]
+    v = t["v"].double().cpu().repeat_interleave(4, dim=1)                    # [N, 4H, 128]
+    go = dout.double().cpu()
+    dd = go * s
+    ref = {"dgate": go * (1.0 - lam) * v * s * (1.0 - s),
+           "dlambda": -(dd * v).sum(-1),
+           "dv": ((1.0 - lam) * dd).reshape(-1, hkv, 4, 128).sum(2)}
+    for name, r in ref.items():
+        mx, rel = _errors(g[name], r.numpy())
+        assert rel <= 5e-3 and mx <= 2e-2, (name, mx, rel)
+    scale = float(g["dv"].float().abs().max())
+    for name in ("dq_sig", "dq_noise", "dk"):
+        assert float(g[name].float().abs().max()) <= 1e-3 * scale, name

@@ -136,3 +136,16 @@ def test_window_at_least_length_equals_full_bitwise():
     torch.cuda.synchronize()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     assert torch.equal(a.view(torch.int16), c.view(torch.int16))
+
+
+def test_window_one_closed_form():
+    """Window 1: each query sees only its own (last) cache row, so out = sigmoid(g)
+    (1 - lambda) v_last of its group: checked in fp64 against that closed form."""
+    lengths = (1, 2, 64, 1025, 300)
+    d = gi.make_decode_inputs(lengths, 2, 61, device="cuda")
+    out = gpu_decode(d, max(lengths), 1)
+    torch.cuda.synchronize()
+    last = d["cu_seqlens_k"][1:].long() - 1
+    v = d["v_cache"][last].double().cpu().repeat_interleave(4, dim=1)      # [B, 4H, 128]
+    ref = torch.sigmoid(d["gate"].double().cpu()) * (1.0 - d["lam"].double().cpu())[..., None] * v
+    assert_close(out.float().cpu().numpy(), ref.numpy(), "decode window 1")

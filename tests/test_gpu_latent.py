@@ -93,3 +93,18 @@ def test_deterministic_and_workspace_contents_do_not_matter():
     b = _gpu(d, 5000, 0, workspace=ws)
     torch.cuda.synchronize()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_window_one_closed_form():
+    """Window 1: each query sees only its last cache row [c | k_rope], so every head of
+    group j gives H = W^UV_j c and out = sigmoid(g) (1 - lambda) W^UV_j c (fp64)."""
+    lengths = (1, 2, 49, 2049, 300)
+    d = gi.make_latent_decode_inputs(lengths, 2, 62, device="cuda")
+    out = _gpu(d, max(lengths), 1)
+    torch.cuda.synchronize()
+    last = d["cu_seqlens_k"][1:].long() - 1
+    c = d["ckv"][last, :512].double().cpu()                                  # [B, 512]
+    h = torch.einsum("jde,be->bjd", d["w_uv"].double().cpu(), c)              # [B, H, 128]
+    h = h.repeat_interleave(4, dim=1)
+    ref = torch.sigmoid(d["gate"].double().cpu()) * (1.0 - d["lam"].double().cpu())[..., None] * h
+    assert_close(out.float().cpu().numpy(), ref.numpy(), "latent decode window 1")

@@ -253,3 +253,28 @@ def test_saturated_gate_gives_the_ungated_difference():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
     ref = oracle.prefill(*host_args(t), seqlens, 0)
     assert_close(a.float().cpu().numpy(), ref, "gate logit 40")
+
+
+@pytest.mark.parametrize("window", [0, 128])
+def test_zero_queries_give_the_running_mean(window):
+    """All queries zero: every visible key scores 0, so each head's H is the plain mean of
+    the visible value rows and out = sigmoid(g) (1 - lambda) mean(v) (fp64 closed form,
+    over sequences spanning several key tiles)."""
+    seqlens = (300, 61)
+    t = gi.make_prefill_inputs(seqlens, 2, 37 + window, device="cuda")
+    t["q_sig"] = torch.zeros_like(t["q_sig"])
+    t["q_noise"] = torch.zeros_like(t["q_noise"])
+    out = gpu_prefill(t, seqlens, window)
+    torch.cuda.synchronize()
+    v = t["v"].double().cpu()
+    means = []
+    s0 = 0
+    for n in seqlens:
+        c = torch.cumsum(v[s0:s0 + n], 0)
+        for i in range(n):
+            lo = 0 if window <= 0 else max(0, i - window + 1)
+            tot = c[i] - (c[lo - 1] if lo > 0 else 0)
+            means.append(tot / (i - lo + 1))
+        s0 += n
+    ref = _closed_form(t, torch.arange(sum(seqlens)), torch.stack(means))
+    assert_close(out.float().cpu().numpy(), ref, f"zero queries, window {window}")

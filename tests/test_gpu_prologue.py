@@ -28,6 +28,11 @@ def check_prologue(seqlens, hkv, seed):
     got = gdla.prologue(t["x"], *[t[w] for w in WEIGHTS], seqlens)
     torch.cuda.synchronize()
     assert gdla.device_error() == 0
+    check_prologue_outputs(t, got, seqlens)
+
+
+def check_prologue_outputs(t, got, seqlens):
+    hkv = t["w_uk"].shape[0]
     ref = oracle.prologue(_host(t["x"]), *[_host(t[w]) for w in WEIGHTS], seqlens)
     report = {}
     for name in NAMES:
@@ -76,3 +81,21 @@ def test_feeds_attention():
     torch.cuda.synchronize()
     assert torch.isfinite(out.float()).all()
     assert gdla.device_error() == 0
+
+
+def test_zero_hidden_state():
+    """x = 0 (tokens 0 and 100 of two sequences zeroed, the rest random): those rows'
+    projections vanish, RMSNorm of a zero vector is zero (no division by zero), the
+    rotary part of zero stays zero, lambda = sigmoid(0) = 1/2, and the gate
+    logits are zero; the other rows still match the oracle."""
+    seqlens = (40, 90)
+    t = gi.make_prologue_inputs(seqlens, 2, 8, device="cuda")
+    zero_rows = [0, 40 + 60]
+    t["x"][zero_rows] = 0
+    o = gdla.prologue(t["x"], *[t[w] for w in WEIGHTS], seqlens)
+    torch.cuda.synchronize()
+    assert gdla.device_error() == 0
+    for name in ("q_sig", "q_noise", "k", "v", "gate"):
+        assert torch.count_nonzero(o[name][zero_rows].float()).item() == 0, name
+    assert float((o["lam"][zero_rows] - 0.5).abs().max()) <= 1e-6
+    check_prologue_outputs(t, o, seqlens)

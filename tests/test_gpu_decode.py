@@ -149,3 +149,22 @@ def test_window_one_closed_form():
     v = d["v_cache"][last].double().cpu().repeat_interleave(4, dim=1)      # [B, 4H, 128]
     ref = torch.sigmoid(d["gate"].double().cpu()) * (1.0 - d["lam"].double().cpu())[..., None] * v
     assert_close(out.float().cpu().numpy(), ref.numpy(), "decode window 1")
+
+
+@pytest.mark.parametrize("window", [0, 128])
+def test_zero_query_gives_the_mean_of_the_visible_values(window):
+    """Zero queries: every visible key scores 0, so out = sigmoid(g) (1 - lambda) times the
+    mean of the visible value rows (fp64 closed form; one- and several-split plans)."""
+    lengths = (1, 129, 1025, 5000, 64)
+    d = gi.make_decode_inputs(lengths, 2, 63 + window, device="cuda")
+    d["q_sig"] = torch.zeros_like(d["q_sig"])
+    d["q_noise"] = torch.zeros_like(d["q_noise"])
+    out = gpu_decode(d, max(lengths), window)
+    torch.cuda.synchronize()
+    cu = d["cu_seqlens_k"].cpu().long()
+    v = d["v_cache"].double().cpu()
+    means = torch.stack([v[max(int(cu[b]), int(cu[b + 1]) - window) if window > 0 else int(cu[b]):int(cu[b + 1])]
+                         .mean(0) for b in range(len(lengths))])                       # [B, H, 128]
+    ref = torch.sigmoid(d["gate"].double().cpu()) * (1.0 - d["lam"].double().cpu())[..., None] * \
+        means.repeat_interleave(4, dim=1)
+    assert_close(out.float().cpu().numpy(), ref.numpy(), f"decode zero queries, window {window}")

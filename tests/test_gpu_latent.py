@@ -108,3 +108,22 @@ def test_window_one_closed_form():
     h = h.repeat_interleave(4, dim=1)
     ref = torch.sigmoid(d["gate"].double().cpu()) * (1.0 - d["lam"].double().cpu())[..., None] * h
     assert_close(out.float().cpu().numpy(), ref.numpy(), "latent decode window 1")
+
+
+@pytest.mark.parametrize("window", [0, 128])
+def test_zero_query_gives_the_projected_mean(window):
+    """Zero absorbed queries: every visible row scores 0, so each head of group j gives
+    H = W^UV_j mean(c) over the visible rows and out = sigmoid(g) (1 - lambda) H (fp64)."""
+    lengths = (1, 129, 2049, 5000, 64)
+    d = gi.make_latent_decode_inputs(lengths, 2, 64 + window, device="cuda")
+    d["q_abs_sig"] = torch.zeros_like(d["q_abs_sig"])
+    d["q_abs_noise"] = torch.zeros_like(d["q_abs_noise"])
+    out = _gpu(d, max(lengths), window)
+    torch.cuda.synchronize()
+    cu = d["cu_seqlens_k"].cpu().long()
+    c = d["ckv"][:, :512].double().cpu()
+    means = torch.stack([c[max(int(cu[b]), int(cu[b + 1]) - window) if window > 0 else int(cu[b]):int(cu[b + 1])]
+                         .mean(0) for b in range(len(lengths))])                       # [B, 512]
+    h = torch.einsum("jde,be->bjd", d["w_uv"].double().cpu(), means).repeat_interleave(4, dim=1)
+    ref = torch.sigmoid(d["gate"].double().cpu()) * (1.0 - d["lam"].double().cpu())[..., None] * h
+    assert_close(out.float().cpu().numpy(), ref.numpy(), f"latent decode zero queries, window {window}")

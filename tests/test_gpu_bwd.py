@@ -141,3 +141,32 @@ def test_window_one_closed_form():
     scale = float(g["dv"].float().abs().max())
     for name in ("dq_sig", "dq_noise", "dk"):
         assert float(g[name].float().abs().max()) <= 1e-3 * scale, name
+
+
+def _permute_groups(x, perm, per_group):
+    """Reorder the KV-group blocks (of `per_group` heads each) along dim 1."""
+    n = x.shape[0]
+    blocks = x.reshape(n, len(perm), per_group, *x.shape[2:])
+    return blocks[:, list(perm)].reshape(x.shape).contiguous()
+
+
+def test_group_permutation_and_long_window_bitwise():
+    """Permuting the KV groups of every input permutes every gradient's groups bit for
+    bit, and a window no shorter than the sequences gives the full-causal gradients bit
+    for bit (the groups are independent and the masks drop nothing)."""
+    seqlens = (300, 77, 1)
+    hkv, perm = 3, (2, 0, 1)
+    t = gi.make_prefill_inputs(seqlens, hkv, 43, device="cuda")
+    dout = gi.make_prefill_grad(seqlens, hkv, 43, device="cuda")
+    a = gdla.attn_bwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"], dout, seqlens, 0)
+    sig = lambda x: _permute_groups(x, perm, 4)
+    one = lambda x: _permute_groups(x, perm, 1)
+    b = gdla.attn_bwd(sig(t["q_sig"]), one(t["q_noise"]), one(t["k"]), one(t["v"]), sig(t["lam"]),
+                      sig(t["gate"]), sig(dout), seqlens, 0)
+    c = gdla.attn_bwd(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"], dout, seqlens, 4096)
+    torch.cuda.synchronize()
+    assert gdla.device_error() == 0
+    for name in NAMES:
+        per = 1 if name in ("dq_noise", "dk", "dv") else 4
+        assert torch.equal(_permute_groups(a[name], perm, per), b[name]), name
+        assert torch.equal(a[name], c[name]), name

@@ -127,3 +127,23 @@ def test_zero_query_gives_the_projected_mean(window):
     h = torch.einsum("jde,be->bjd", d["w_uv"].double().cpu(), means).repeat_interleave(4, dim=1)
     ref = torch.sigmoid(d["gate"].double().cpu()) * (1.0 - d["lam"].double().cpu())[..., None] * h
     assert_close(out.float().cpu().numpy(), ref.numpy(), f"latent decode zero queries, window {window}")
+
+
+def test_group_permutation_equivariant_bitwise():
+    """Permuting the KV groups (their queries, W^UV_j, lambda and gate) permutes the
+    output groups bit for bit: every group's heads see the same cache rows."""
+    lengths = (1, 300, 2049, 77)
+    hkv, perm = 3, [2, 0, 1]
+    d = gi.make_latent_decode_inputs(lengths, hkv, 65, device="cuda")
+    a = _gpu(d, max(lengths), 0)
+
+    def grp(x, per):
+        b = x.shape[0]
+        return x.reshape(b, hkv, per, *x.shape[2:])[:, perm].reshape(x.shape).contiguous()
+
+    p = dict(d, q_abs_sig=grp(d["q_abs_sig"], 4), q_abs_noise=grp(d["q_abs_noise"], 1),
+             w_uv=d["w_uv"][perm].contiguous(), lam=grp(d["lam"], 4), gate=grp(d["gate"], 4))
+    b = _gpu(p, max(lengths), 0)
+    torch.cuda.synchronize()
+    assert gdla.device_error() == 0
+    assert torch.equal(grp(a, 4).view(torch.int16), b.view(torch.int16))

@@ -139,3 +139,35 @@ def test_planted_prologue_slip_is_caught(name, monkeypatch):
     ref = library_prologue(x, w, SEQLENS)
     got = _run_oracle(x, w)
     assert _worst(got, ref) > 1e-3, f"mutant {name} not caught"
+
+
+# Slips inside the body of oracle.prologue: each is a copy of its source with one
+# substitution, compiled in the oracle module's namespace.
+BODY_MUTANTS = {
+    "rope_on_content_dims": ("np.concatenate([q[..., :DQK - ROPE], rope(q[..., DQK - ROPE:], pos)], axis=-1)",
+                             "np.concatenate([rope(q[..., :ROPE], pos), q[..., ROPE:]], axis=-1)"),
+    "k_rope_from_latent_dims": ("k_rope = rope(ckv_full[:, DC:], pos)", "k_rope = rope(ckv_full[:, :ROPE], pos)"),
+    "w_uk_and_w_uv_swapped": ('k_nope = np.einsum("nc,hdc->nhd", ckv, _f64(w_uk))',
+                              'k_nope = np.einsum("nc,hdc->nhd", ckv, _f64(w_uv))'),
+    "lambda_without_sigmoid": ("lam = 1.0 / (1.0 + np.exp(-(x @ _f64(w_lambda).T)))", "lam = x @ _f64(w_lambda).T"),
+    "noise_heads_first": ('{"q_sig": q[:, :hs], "q_noise": q[:, hs:]', '{"q_sig": q[:, hkv:], "q_noise": q[:, :hkv]'),
+    "c_q_not_normalised": ("cq = rms_norm(x @ _f64(w_qa).T, gamma_q)", "cq = (x @ _f64(w_qa).T) * gamma_q"),
+    "k_rope_not_rotated": ("k_rope = rope(ckv_full[:, DC:], pos)", "k_rope = ckv_full[:, DC:]"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(BODY_MUTANTS))
+def test_planted_slip_in_the_prologue_body_is_caught(name, monkeypatch):
+    import inspect
+    import textwrap
+    old, new = BODY_MUTANTS[name]
+    src = textwrap.dedent(inspect.getsource(oracle.prologue))
+    assert src.count(old) == 1, name
+    scope = dict(vars(oracle))
+    exec(compile(src.replace(old, new), f"<mutant {name}>", "exec"), scope)
+    monkeypatch.setattr(oracle, "prologue", scope["prologue"])
+    w = _weights(3)
+    x = torch.randn(sum(SEQLENS), HIDDEN, generator=torch.Generator().manual_seed(4), dtype=torch.float64)
+    ref = library_prologue(x, w, SEQLENS)
+    got = _run_oracle(x, w)
+    assert _worst(got, ref) > 1e-3, f"mutant {name} not caught"

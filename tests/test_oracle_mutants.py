@@ -86,3 +86,48 @@ def test_mutant_is_caught(name, monkeypatch):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"mutant {name} passed every pin"
+
+
+# Slips in the decode path's own code (the prefill path untouched): each must break
+# "decode equals the last prefill row".
+DECODE_MUTANTS = {
+    "decode_window_off_by_one": (
+        "const int64_t t = len - 1;              /* the query's own position */\n        int64_t lo = 0;\n"
+        "        if (J->window > 0 && t - J->window + 1 > 0) lo = t - J->window + 1;",
+        "const int64_t t = len - 1;              /* the query's own position */\n        int64_t lo = 0;\n"
+        "        if (J->window > 0 && t - J->window + 2 > 0) lo = t - J->window + 2;"),
+    "decode_query_position": ("const int64_t t = len - 1;              /* the query's own position */",
+                              "const int64_t t = len - 2;              /* the query's own position */"),
+    "decode_noise_group_index": ("const uint16_t *qn = J->q_noise + (b * J->hkv + j) * DQK;",
+                                 "const uint16_t *qn = J->q_noise + (b * J->hkv + (J->hkv - 1 - j)) * DQK;"),
+    "decode_lambda_index": ("const float *lam = J->lambda + b * hs + GROUP * j;",
+                            "const float *lam = J->lambda + b * hs + j;"),
+    "decode_gate_group": ("const uint16_t *gate = J->gate + (b * hs + (long)GROUP * j) * DV;",
+                          "const uint16_t *gate = J->gate + (b * hs) * DV;"),
+    "decode_sequence_offset_dropped": ("const uint16_t *krow = J->k + (s0 + lo) * kstride + (long)j * DQK;\n"
+                                       "        const uint16_t *vrow = J->v + (s0 + lo) * vstride + (long)j * DV;\n"
+                                       "        const uint16_t *qs = J->q_sig + (b * hs",
+                                       "const uint16_t *krow = J->k + lo * kstride + (long)j * DQK;\n"
+                                       "        const uint16_t *vrow = J->v + lo * vstride + (long)j * DV;\n"
+                                       "        const uint16_t *qs = J->q_sig + (b * hs"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(DECODE_MUTANTS))
+def test_decode_mutant_is_caught(name, monkeypatch):
+    old, new = DECODE_MUTANTS[name]
+    assert open(SRC).read().count(old) == 1, name
+    path = _build_mutant(name, old, new)
+    real = oracle._load()
+    lib = ctypes.CDLL(path)
+    for fn in ("gdla_oracle_prefill", "gdla_oracle_decode"):
+        getattr(lib, fn).argtypes = getattr(real, fn).argtypes
+        getattr(lib, fn).restype = getattr(real, fn).restype
+    monkeypatch.setattr(oracle, "_lib", lib)
+    caught = []
+    for window in (0, 2, 300):
+        try:
+            P.test_decode_equals_last_prefill_row(window)
+        except AssertionError:
+            caught.append(window)
+    assert caught, f"decode mutant {name} passed every pin"

@@ -74,3 +74,45 @@ def test_chunks_equal_the_whole_sequence(mode, world, window):
     ref = _oracle_attn(t["q_sig"], t["q_noise"], t["k"], t["v"], t["lam"], t["gate"], (T,), window).numpy()
     assert got.shape == ref.shape
     assert np.array_equal(got, ref)
+
+
+def _error_worker(rank, world, port, q):
+    import torch.distributed as dist
+    from datetime import timedelta
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    from differential_latent_attention_b200 import context_parallel as cp
+    caught = []
+    for hkv, window, fn in ((4, 60, "swa"), (4, 0, "swa"), (3, 0, "ulysses")):
+        t = _inputs(96, hkv, 5)
+        c = 96 // world
+        chunk = [t[k][rank * c:(rank + 1) * c].contiguous() for k in ("q_sig", "q_noise", "k", "v", "lam", "gate")]
+        try:
+            if fn == "swa":
+                cp.swa_forward_cp(*chunk, window, attn=_oracle_attn)
+            else:
+                cp.full_forward_ulysses(*chunk, attn=_oracle_attn)
+        except ValueError:
+            caught.append((hkv, window, fn))
+    dist.barrier()   # every rank raised before any exchange, so the group is still in step
+    q.put((rank, caught))
+    dist.destroy_process_group()
+
+
+def test_unsupported_splits_raise_on_every_rank_before_any_exchange():
+    """A chunk shorter than the window's halo, a window of 0 for the halo scheme and a
+    KV-group count the world size does not divide each raise ValueError on every rank,
+    before any collective (the ranks stay in step and finish a barrier afterwards)."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_error_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=300) for _ in procs)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    for r in range(world):
+        assert res[r] == [(4, 60, "swa"), (4, 0, "swa"), (3, 0, "ulysses")], res[r]
